@@ -1,0 +1,13 @@
+"""fp64 CPU oracle for permuted block-sparse attention prefill.
+
+TEST INFRASTRUCTURE ONLY: imported by the tests, by the package smoke check
+and by the benchmark's CPU-baseline leg, never by the product path.
+"""
+from .pbs_oracle import *  # noqa: F401,F403
+from .pbs_oracle import (attn, attn_block, calibrate_thresholds, dense_lists,
+                         diagonal_blocks, forced_blocks, inverse_permutation,
+                         key_scores, key_tiles,
+                         lists_to_array, n_candidates, natural_key_block_sums,
+                         permute, permuted_key_block_sums, proxy_query,
+                         query_block_sums, segment_of_block, select,
+                         sort_segments, tile_maxima, topk_target)

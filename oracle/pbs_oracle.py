@@ -1,0 +1,400 @@
+"""fp64 CPU oracle for permuted block-sparse attention prefill.
+
+TEST INFRASTRUCTURE ONLY.  Only the test-suite, the package smoke check and
+the benchmark's CPU-baseline leg may import this module.  The product path
+(the CUDA library and its Python binding) never imports, calls or links it,
+and this module imports nothing from the product.
+
+It restates, step by step and in the pages' order, what the method computes:
+
+  1. proxy query + key scores   -- "Sparser Block-Sparse Attention via Token
+     Permutation", Technical Summary, 3. Global-Importance-Based Key
+     Permutation (Proxy Scoring: the last block of queries, mean-pooled
+     attention scores);
+  2. segmented stable sort      -- same page, 2. Segmented Permutation for
+     Causality and 3. (Sorting: descending within each segment);
+  3. block scores               -- same page, 4. Implementation (Block
+     Selection by mean pooling on the permuted keys);
+  4. top-k / cumulative-mass selection -- same page 4., and "SampleAttention"
+     (MLSys 2025 talk), Technical Deep Dive (the attention mass to preserve
+     per query);
+  5. masked softmax attention   -- "S2O: Early Stopping for Sparse Attention
+     via Online Permutation", Technical Summary, 3. Kernel Implementation
+     (Pass 1: dense causal window of the current segment; Pass 2: prefix
+     keys in permuted order), and the permutation invariance of attention
+     (PBS page, 1. Theoretical Foundation);
+  6. in-tile block-max gating   -- "Block Sparse Flash Attention", Approach
+     (exact QK^T in the tile; skip V and PV when the tile max is below a
+     calibrated threshold that keeps roughly the top-k blocks).
+
+Everything is fp64 on the same (bf16-exact) input values.  Where the pages
+leave a step open the plainest reading is taken; the readings are:
+
+  * proxy scores are pre-softmax logits of the pooled (summed) proxy query,
+    unscaled: the sort is invariant to the positive scale and divisor;
+  * the proxy query pools the last ``blk`` query rows of every query head of
+    the KV head's group, since keys (and hence the permutation) are per KV
+    head;
+  * sort ties keep ascending original position (stable);
+  * sink positions get score +inf, so they lead segment 0;
+  * a query block's own segment is attended densely, in natural order,
+    causally (Pass 1); listed permuted blocks come only from earlier
+    segments (Pass 2);
+  * block score = (sum of the block's query rows) . (sum of the permuted key
+    block's rows); for cumulative mass the softmax runs over these scores
+    divided by blk^2 * sqrt(d) (the mean tile logit);
+  * top-k budget k_i = max(D_i + |F_i|, ceil(rho * n_i)) with rho taken in
+    per-mille and the ceiling in integers; ties go to the lower block id;
+  * a gated tile is excluded entirely; the query block's own tile is never
+    gated; thresholds and tile maxima are raw (unscaled) q.k values.
+
+Parity pins: tests/test_oracle_pins.py checks every function here against
+brute force, closed forms, library routines and invariants.
+"""
+from __future__ import annotations
+
+import math
+from typing import Iterable, List, Optional, Sequence, Tuple
+
+import numpy as np
+
+F64 = np.float64
+
+
+# --------------------------------------------------------------------------
+# geometry helpers (plain integer bookkeeping)
+# --------------------------------------------------------------------------
+
+def segment_of_block(i: int, blk: int, seg: int) -> int:
+    """Segment index s(i) of query block i (segments hold seg/blk blocks)."""
+    return (i * blk) // seg
+
+
+def diagonal_blocks(i: int, blk: int, seg: int) -> range:
+    """Natural key blocks of block i's own segment that are causal for it."""
+    spb = seg // blk
+    s = segment_of_block(i, blk, seg)
+    return range(s * spb, i + 1)
+
+
+def n_candidates(i: int, blk: int, seg: int) -> int:
+    """Number of permuted key blocks in segments strictly before s(i)."""
+    spb = seg // blk
+    return segment_of_block(i, blk, seg) * spb
+
+
+def topk_target(n_causal: int, density: float) -> int:
+    """ceil(rho * n) with rho rounded to per-mille, computed in integers."""
+    r = int(round(1000.0 * density))
+    return -((-r * n_causal) // 1000)
+
+
+# --------------------------------------------------------------------------
+# 1-2. permutation
+# --------------------------------------------------------------------------
+
+def proxy_query(Q: np.ndarray, Hkv: int, blk: int) -> np.ndarray:
+    """qhat[b, hkv, :] = sum over the last ``blk`` query rows of every query
+    head in KV head hkv's group.  Q: [B, Hq, N, d].  Returns fp64 [B, Hkv, d]."""
+    B, Hq, N, d = Q.shape
+    G = Hq // Hkv
+    out = np.zeros((B, Hkv, d), F64)
+    for b in range(B):
+        for h in range(Hkv):
+            rows = Q[b, h * G:(h + 1) * G, N - blk:N, :].astype(F64)
+            out[b, h] = rows.reshape(-1, d).sum(axis=0)
+    return out
+
+
+def key_scores(qhat: np.ndarray, K: np.ndarray, n_sink: int = 0) -> np.ndarray:
+    """s[b, hkv, j] = qhat[b, hkv] . K[b, hkv, j] in fp64; sinks get +inf."""
+    B, Hkv, N, d = K.shape
+    s = np.zeros((B, Hkv, N), F64)
+    for b in range(B):
+        for h in range(Hkv):
+            s[b, h] = K[b, h].astype(F64) @ qhat[b, h]
+    if n_sink > 0:
+        s[:, :, :n_sink] = np.inf
+    return s
+
+
+def sort_segments(scores: np.ndarray, seg: int) -> np.ndarray:
+    """perm[b, h, p] = original position at logical position p.
+
+    Within each segment [t*seg, min((t+1)*seg, N)) positions are ordered by
+    descending score, equal scores in ascending position; segment order is
+    kept, so perm is a bijection of each segment onto itself."""
+    B, H, N = scores.shape
+    perm = np.empty((B, H, N), np.int32)
+    for b in range(B):
+        for h in range(H):
+            for lo in range(0, N, seg):
+                hi = min(lo + seg, N)
+                order = np.argsort(-scores[b, h, lo:hi], kind="stable")
+                perm[b, h, lo:hi] = lo + order
+    return perm
+
+
+def permute(Q: np.ndarray, K: np.ndarray, blk: int, seg: int, n_sink: int = 0) -> np.ndarray:
+    """The full permutation step: proxy query, key scores, segment sort."""
+    Hkv = K.shape[1]
+    qhat = proxy_query(Q, Hkv, blk)
+    return sort_segments(key_scores(qhat, K, n_sink), seg)
+
+
+# --------------------------------------------------------------------------
+# 3-4. block selection
+# --------------------------------------------------------------------------
+
+def query_block_sums(Q: np.ndarray, blk: int) -> np.ndarray:
+    """Qbar[b, hq, i] = sum of the blk rows of query block i (fp64)."""
+    B, H, N, d = Q.shape
+    return Q.astype(F64).reshape(B, H, N // blk, blk, d).sum(axis=3)
+
+
+def permuted_key_block_sums(K: np.ndarray, perm: np.ndarray, blk: int) -> np.ndarray:
+    """Kbar[b, hkv, pb] = sum of K rows perm[pb*blk .. pb*blk+blk-1] (fp64)."""
+    B, H, N, d = K.shape
+    out = np.zeros((B, H, N // blk, d), F64)
+    for b in range(B):
+        for h in range(H):
+            rows = K[b, h].astype(F64)[perm[b, h]]
+            out[b, h] = rows.reshape(N // blk, blk, d).sum(axis=1)
+    return out
+
+
+def natural_key_block_sums(K: np.ndarray, blk: int) -> np.ndarray:
+    B, H, N, d = K.shape
+    return K.astype(F64).reshape(B, H, N // blk, blk, d).sum(axis=3)
+
+
+def inverse_permutation(perm_row: np.ndarray) -> np.ndarray:
+    """inv[perm[p]] = p: the logical position of each original position."""
+    inv = np.empty_like(perm_row)
+    inv[perm_row] = np.arange(perm_row.shape[0], dtype=perm_row.dtype)
+    return inv
+
+
+def forced_blocks(i: int, inv_row: np.ndarray, blk: int, seg: int,
+                  band: int, n_sink: int) -> List[int]:
+    """Permuted blocks of earlier segments that must be listed for block i:
+    those holding a sink position (< n_sink) or a position among the ``band``
+    most recent keys of any query in the block.  ``inv_row`` is the inverse
+    of the KV head's permutation.  Ascending block ids."""
+    ncand = n_candidates(i, blk, seg)
+    if ncand == 0:
+        return []
+    s_start = segment_of_block(i, blk, seg) * seg
+    want = set()
+    if n_sink > 0:
+        for pos in range(0, min(n_sink, s_start)):
+            want.add(int(inv_row[pos]) // blk)
+    if band > 0:
+        lo = max(0, i * blk - band + 1)
+        for pos in range(lo, s_start):
+            want.add(int(inv_row[pos]) // blk)
+    return sorted(pb for pb in want if pb < ncand)
+
+
+def select(Q: np.ndarray, K: np.ndarray, perm: np.ndarray, blk: int, seg: int,
+           mode: str, density: float = 1.0, tau: float = 1.0, band: int = 0,
+           n_sink: int = 0, rows: Optional[Iterable[Tuple[int, int, int]]] = None):
+    """Per (b, hq, i) ascending lists of permuted key blocks to attend.
+
+    Returns (counts [B,Hq,nb] int32, lists dict {(b,hq,i): int32 array}).
+    With ``rows`` given, only those (b, hq, i) are computed (others count 0).
+    mode "topk": budget from ``density``; mode "tau": cumulative mass."""
+    B, Hq, N, d = Q.shape
+    Hkv = K.shape[1]
+    G = Hq // Hkv
+    nb = N // blk
+    if rows is None:
+        rows = [(b, h, i) for b in range(B) for h in range(Hq) for i in range(nb)]
+    rows = list(rows)
+    need_q = sorted({(b, h) for b, h, _ in rows})
+    counts = np.zeros((B, Hq, nb), np.int32)
+    lists = {}
+    kbar_p = {}
+    kbar_n = {}
+    inv = {}
+    for (b, h) in need_q:
+        hk = h // G
+        if (b, hk) not in kbar_p:
+            kbar_p[(b, hk)] = permuted_key_block_sums(K[b:b + 1, hk:hk + 1], perm[b:b + 1, hk:hk + 1], blk)[0, 0]
+            kbar_n[(b, hk)] = natural_key_block_sums(K[b:b + 1, hk:hk + 1], blk)[0, 0]
+            inv[(b, hk)] = inverse_permutation(perm[b, hk])
+    qbar_cache = {}
+    for (b, h, i) in rows:
+        hk = h // G
+        if (b, h) not in qbar_cache:
+            qbar_cache[(b, h)] = query_block_sums(Q[b:b + 1, h:h + 1], blk)[0, 0]
+        qb = qbar_cache[(b, h)][i]
+        ncand = n_candidates(i, blk, seg)
+        diag = list(diagonal_blocks(i, blk, seg))
+        D = len(diag)
+        if ncand == 0:
+            lists[(b, h, i)] = np.zeros(0, np.int32)
+            continue
+        S = kbar_p[(b, hk)][:ncand] @ qb                      # exact on lattice inputs
+        F = forced_blocks(i, inv[(b, hk)], blk, seg, band, n_sink)
+        rest = np.setdiff1d(np.arange(ncand, dtype=np.int64), np.array(F, np.int64))
+        # descending score, ties to the lower block id
+        order = rest[np.lexsort((rest, -S[rest]))] if rest.size else rest
+        if mode == "topk":
+            k = max(D + len(F), topk_target(i + 1, density))
+            take = k - D - len(F)
+            chosen = list(F) + [int(x) for x in order[:take]]
+        elif mode == "tau":
+            if tau >= 1.0:
+                chosen = list(range(ncand))
+            else:
+                scale = 1.0 / (blk * blk * math.sqrt(d))
+                lg_c = S * scale
+                lg_d = np.array([kbar_n[(b, hk)][j] @ qb for j in diag], F64) * scale
+                m = max(lg_c.max(), lg_d.max())
+                e_c = np.exp(lg_c - m)
+                e_d = np.exp(lg_d - m)
+                Z = e_c.sum() + e_d.sum()
+                cum = (e_d.sum() + e_c[F].sum()) / Z if F else e_d.sum() / Z
+                chosen = list(F)
+                for pb in order:
+                    if cum >= tau:
+                        break
+                    chosen.append(int(pb))
+                    cum += e_c[pb] / Z
+        else:
+            raise ValueError(mode)
+        arr = np.array(sorted(chosen), np.int32)
+        lists[(b, h, i)] = arr
+        counts[b, h, i] = arr.size
+    return counts, lists
+
+
+def lists_to_array(counts: np.ndarray, lists: dict, cap: int) -> np.ndarray:
+    """Pack lists into idx[B,Hq,nb,cap] (unused entries -1)."""
+    B, H, nb = counts.shape
+    idx = np.full((B, H, nb, cap), -1, np.int32)
+    for (b, h, i), arr in lists.items():
+        idx[b, h, i, :arr.size] = arr
+    return idx
+
+
+# --------------------------------------------------------------------------
+# 5-6. attention (optionally gated)
+# --------------------------------------------------------------------------
+
+def key_tiles(i: int, listed: Sequence[int], perm_row: np.ndarray, blk: int, seg: int):
+    """The tiles query block i visits: (kind, id, key positions).
+
+    kind "perm": permuted block of an earlier segment, keys perm[pb*blk ...];
+    kind "diag": natural block of the block's own segment."""
+    tiles = []
+    for pb in listed:
+        tiles.append(("perm", int(pb), perm_row[pb * blk:(pb + 1) * blk].astype(np.int64)))
+    for j in diagonal_blocks(i, blk, seg):
+        tiles.append(("diag", j, np.arange(j * blk, (j + 1) * blk, dtype=np.int64)))
+    return tiles
+
+
+def attn_block(Q, K, V, perm, listed, b, hq, i, blk, seg, scale,
+               gate_thr: Optional[float] = None):
+    """O and LSE (natural log of the softmax normaliser of the scaled logits)
+    for the ``blk`` query rows of block i of (b, hq), fp64.
+
+    The key set is the listed permuted blocks plus the causal part of the
+    block's own segment; with ``gate_thr`` every tile except block i's own is
+    dropped when its maximal raw q.k over visible entries is below it."""
+    Hq, Hkv = Q.shape[1], K.shape[1]
+    hk = hq // (Hq // Hkv)
+    q_pos = np.arange(i * blk, (i + 1) * blk)
+    q = Q[b, hq, i * blk:(i + 1) * blk].astype(F64)
+    keys, kmask = [], []
+    for kind, tid, pos in key_tiles(i, listed, perm[b, hk], blk, seg):
+        visible = pos[None, :] <= q_pos[:, None]
+        if gate_thr is not None and not (kind == "diag" and tid == i):
+            raw = q @ K[b, hk, pos].astype(F64).T
+            tmax = raw[visible].max() if visible.any() else -np.inf
+            if tmax < gate_thr:
+                continue
+        keys.append(pos)
+        kmask.append(visible)
+    keys = np.concatenate(keys)
+    vis = np.concatenate(kmask, axis=1)
+    logits = (q @ K[b, hk, keys].astype(F64).T) * scale
+    logits = np.where(vis, logits, -np.inf)
+    m = logits.max(axis=1, keepdims=True)
+    e = np.exp(logits - m)
+    l = e.sum(axis=1, keepdims=True)
+    O = (e @ V[b, hk, keys].astype(F64)) / l
+    lse = (m + np.log(l))[:, 0]
+    return O, lse
+
+
+def attn(Q, K, V, perm, lists: dict, blk: int, seg: int, scale: Optional[float] = None,
+         gate_thr: Optional[np.ndarray] = None, blocks: Optional[Iterable[Tuple[int, int, int]]] = None):
+    """O [B,Hq,N,d] and LSE [B,Hq,N] (fp64) over the given (b, hq, i) blocks
+    (all by default; rows of other blocks stay NaN).  ``lists`` maps
+    (b, hq, i) to its listed permuted blocks (missing = none)."""
+    B, Hq, N, d = Q.shape
+    nb = N // blk
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if blocks is None:
+        blocks = [(b, h, i) for b in range(B) for h in range(Hq) for i in range(nb)]
+    O = np.full((B, Hq, N, d), np.nan, F64)
+    L = np.full((B, Hq, N), np.nan, F64)
+    for (b, h, i) in blocks:
+        listed = lists.get((b, h, i), np.zeros(0, np.int32))
+        thr = None if gate_thr is None else float(gate_thr[b, h, i])
+        o, lse = attn_block(Q, K, V, perm, listed, b, h, i, blk, seg, scale, thr)
+        O[b, h, i * blk:(i + 1) * blk] = o
+        L[b, h, i * blk:(i + 1) * blk] = lse
+    return O, L
+
+
+# --------------------------------------------------------------------------
+# 6. gate calibration
+# --------------------------------------------------------------------------
+
+def tile_maxima(Q, K, b, hq, i, blk) -> np.ndarray:
+    """M[j] = max over visible (q, k) of raw q.k for natural tiles j <= i."""
+    Hq, Hkv = Q.shape[1], K.shape[1]
+    hk = hq // (Hq // Hkv)
+    q = Q[b, hq, i * blk:(i + 1) * blk].astype(F64)
+    k = K[b, hk, :(i + 1) * blk].astype(F64)
+    raw = q @ k.T
+    q_pos = np.arange(i * blk, (i + 1) * blk)[:, None]
+    k_pos = np.arange((i + 1) * blk)[None, :]
+    raw = np.where(k_pos <= q_pos, raw, -np.inf)
+    return raw.reshape(blk, i + 1, blk).max(axis=(0, 2))
+
+
+def calibrate_thresholds(Q, K, blk: int, keep: int,
+                         blocks: Optional[Iterable[Tuple[int, int, int]]] = None) -> np.ndarray:
+    """thr[b, hq, i] = the keep-th largest causal tile maximum of block i
+    (-inf when block i has at most ``keep`` causal tiles).  Unlisted blocks
+    (when ``blocks`` is given) get -inf."""
+    B, Hq, N, d = Q.shape
+    nb = N // blk
+    thr = np.full((B, Hq, nb), -np.inf, F64)
+    if blocks is None:
+        blocks = [(b, h, i) for b in range(B) for h in range(Hq) for i in range(nb)]
+    for (b, h, i) in blocks:
+        if i + 1 <= keep:
+            continue
+        M = tile_maxima(Q, K, b, h, i, blk)
+        thr[b, h, i] = np.sort(M)[::-1][keep - 1]
+    return thr
+
+
+def dense_lists(B: int, Hq: int, nb: int, blk: int, seg: int) -> Tuple[np.ndarray, dict]:
+    """Every candidate block listed (density 1): dense causal attention."""
+    counts = np.zeros((B, Hq, nb), np.int32)
+    lists = {}
+    for b in range(B):
+        for h in range(Hq):
+            for i in range(nb):
+                arr = np.arange(n_candidates(i, blk, seg), dtype=np.int32)
+                lists[(b, h, i)] = arr
+                counts[b, h, i] = arr.size
+    return counts, lists

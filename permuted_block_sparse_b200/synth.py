@@ -1,0 +1,154 @@
+"""Seeded synthetic inputs for permuted block-sparse attention prefill.
+
+This module only draws numbers: it holds none of the method's arithmetic
+(no pooling, scoring, sorting, selection or softmax).  Both the CPU oracle
+(through the tests) and the CUDA path consume its arrays.
+
+Workload structure follows the stripe observation of "S2O: Early Stopping
+for Sparse Attention via Online Permutation" (Technical Summary, Significance
+and Claims: attention maps are stripes, not blocks) and the heavy-hitter
+picture of "Sparser Block-Sparse Attention via Token Permutation" (Problem
+Statement: important keys scattered across many blocks).  Real model
+activations are not available, so a planted-stripe model stands in for them:
+
+  * Q, K, V ~ N(0, 1), drawn in float32 in the order Q, K, V;
+  * per KV head h a random unit direction u_h;
+  * a fraction ``stripe_frac`` of key positions per KV head, chosen uniformly
+    without replacement, get K += c * u_h, with c fixed or drawn per stripe
+    key from U[c_lo, c_hi];
+  * every query of the heads in that KV head's group gets Q += q_off * u_h;
+  * finally every value is rounded to a multiple of 1/8 and clipped to
+    +-31.875, so it is exact in bfloat16 ("lattice" values).  On lattice
+    inputs every pooled sum and block score of the method is exactly
+    representable in fp32, which is what makes bit-exact index parity
+    between the GPU and an fp64 oracle possible.
+
+Arrays are float32 numpy arrays holding bf16-exact values, layout
+Q[B,Hq,N,d], K/V[B,Hkv,N,d].
+"""
+from __future__ import annotations
+
+import dataclasses
+from typing import Optional, Tuple
+
+import numpy as np
+
+LATTICE_STEP = 0.125
+LATTICE_MAX = 31.875
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    """One synthetic prefill-attention problem and its selection settings."""
+
+    name: str
+    B: int
+    Hq: int
+    Hkv: int
+    N: int
+    d: int
+    blk: int
+    seg: int
+    mode: str                 # "topk", "tau" or "gate"
+    density: float = 1.0      # top-k density rho
+    tau: float = 1.0          # cumulative-mass target
+    band: int = 0             # most recent keys always kept (0 = none)
+    n_sink: int = 0           # leading sink keys always kept
+    gate_keep: int = 0        # gating: calibrate thresholds to keep this many tiles
+    stripe_frac: float = 0.0
+    c_lo: float = 4.0
+    c_hi: float = 4.0
+    q_off: float = 1.5
+    seed: int = 0
+
+    @property
+    def G(self) -> int:
+        return self.Hq // self.Hkv
+
+    @property
+    def nb(self) -> int:
+        return self.N // self.blk
+
+    def with_(self, **kw) -> "Workload":
+        return dataclasses.replace(self, **kw)
+
+
+# The five workloads.  Sizes, block/segment sizes, selection knobs and stripe
+# recipes are the ones the benchmark plan states; the query offset 1.5 is the
+# single-head case's value, reused for the others, which leave it open.
+WORKLOADS = {
+    "single_head_1k": Workload(
+        "single_head_1k", B=1, Hq=1, Hkv=1, N=1024, d=64, blk=64, seg=256,
+        mode="topk", density=0.30, stripe_frac=0.02, c_lo=4.0, c_hi=4.0),
+    "gqa_8k_band": Workload(
+        "gqa_8k_band", B=1, Hq=8, Hkv=2, N=8192, d=128, blk=128, seg=1024,
+        mode="topk", density=0.20, band=256, stripe_frac=0.01, c_lo=4.0, c_hi=4.0),
+    "llama8b_32k_tau": Workload(
+        "llama8b_32k_tau", B=1, Hq=32, Hkv=8, N=32768, d=128, blk=128, seg=2048,
+        mode="tau", tau=0.95, stripe_frac=0.005, c_lo=3.0, c_hi=6.0),
+    "llama8b_128k_sink": Workload(
+        "llama8b_128k_sink", B=1, Hq=32, Hkv=8, N=131072, d=128, blk=128, seg=4096,
+        mode="topk", density=0.10, n_sink=128, stripe_frac=0.0025, c_lo=4.0, c_hi=4.0),
+    "gate_b8_2k": Workload(
+        "gate_b8_2k", B=8, Hq=32, Hkv=8, N=2048, d=128, blk=128, seg=128,
+        mode="gate", gate_keep=64, stripe_frac=0.005, c_lo=3.0, c_hi=6.0),
+    "gate_b8_4k": Workload(
+        "gate_b8_4k", B=8, Hq=32, Hkv=8, N=4096, d=128, blk=128, seg=128,
+        mode="gate", gate_keep=64, stripe_frac=0.005, c_lo=3.0, c_hi=6.0),
+    "gate_b1_64k": Workload(
+        "gate_b1_64k", B=1, Hq=32, Hkv=8, N=65536, d=128, blk=128, seg=128,
+        mode="gate", gate_keep=64, stripe_frac=0.005, c_lo=3.0, c_hi=6.0),
+}
+
+
+def lattice(x: np.ndarray) -> np.ndarray:
+    """Round to the nearest multiple of 1/8 (ties to even) and clip: bf16-exact."""
+    y = np.round(x * (1.0 / LATTICE_STEP)).astype(np.float32)
+    np.clip(y, -LATTICE_MAX / LATTICE_STEP, LATTICE_MAX / LATTICE_STEP, out=y)
+    y *= np.float32(LATTICE_STEP)
+    return y
+
+
+def make_inputs(w: Workload, seed: Optional[int] = None) -> Tuple[np.ndarray, np.ndarray, np.ndarray, dict]:
+    """Draw Q, K, V for workload ``w``.  Returns (Q, K, V, info).
+
+    ``info`` records the planted structure (directions, stripe positions and
+    offsets) so tests can reason about it; nothing of the method is computed.
+    """
+    seed = w.seed if seed is None else seed
+    rng = np.random.default_rng(seed)
+    B, Hq, Hkv, N, d, G = w.B, w.Hq, w.Hkv, w.N, w.d, w.G
+    Q = rng.standard_normal((B, Hq, N, d), dtype=np.float32)
+    K = rng.standard_normal((B, Hkv, N, d), dtype=np.float32)
+    V = rng.standard_normal((B, Hkv, N, d), dtype=np.float32)
+    n_stripe = int(round(w.stripe_frac * N))
+    dirs = np.zeros((B, Hkv, d), np.float32)
+    stripes = np.zeros((B, Hkv, n_stripe), np.int64)
+    offsets = np.zeros((B, Hkv, n_stripe), np.float32)
+    for b in range(B):
+        for h in range(Hkv):
+            u = rng.standard_normal(d).astype(np.float64)
+            u /= np.linalg.norm(u)
+            u = u.astype(np.float32)
+            pos = np.sort(rng.choice(N, size=n_stripe, replace=False)) if n_stripe else np.zeros(0, np.int64)
+            if w.c_hi > w.c_lo:
+                c = rng.uniform(w.c_lo, w.c_hi, size=n_stripe).astype(np.float32)
+            else:
+                c = np.full(n_stripe, w.c_lo, np.float32)
+            if n_stripe:
+                K[b, h, pos, :] += c[:, None] * u[None, :]
+            Q[b, h * G:(h + 1) * G, :, :] += np.float32(w.q_off) * u
+            dirs[b, h] = u
+            stripes[b, h] = pos
+            offsets[b, h] = c
+    Q = lattice(Q)
+    K = lattice(K)
+    V = lattice(V)
+    info = {"seed": seed, "dirs": dirs, "stripes": stripes, "offsets": offsets}
+    return Q, K, V, info
+
+
+def random_lattice(shape, seed: int, scale: float = 1.0) -> np.ndarray:
+    """Plain N(0, scale^2) lattice values (no planted structure)."""
+    rng = np.random.default_rng(seed)
+    return lattice(rng.standard_normal(shape, dtype=np.float32) * np.float32(scale))
