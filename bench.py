@@ -1,0 +1,430 @@
+#!/usr/bin/env python3
+"""Benchmark: permuted block-sparse attention prefill on B200.
+
+One step = pbs_permute + pbs_select + pbs_attn_fwd over one batch of the
+128K-token GQA workload (B=1, Hq=32, Hkv=8, d=128, blk 128, seg 4096, 10 %
+top-k density, 128 sink keys; planted-stripe lattice inputs), inputs
+resident in HBM.  Prints ONE JSON line (rank 0).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl pbs|reference]
+
+Under torchrun each rank runs its own copy of the workload on its own GPU
+(weak scaling: the path shards by independent problems, no collective on
+the data path); times are the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "prefill attention ms & effective TFLOP/s (% bf16 TC peak) at 128K vs dense"
+DEFAULT_WORKLOAD = "llama8b_128k_sink"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="pbs", choices=["pbs", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--no-dense", action="store_true", help="skip the dense same-kernel comparison run")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def dense_causal_flops(w) -> float:
+    return 2.0 * w.d * w.N * w.N * w.Hq * w.B
+
+
+def tile_flops(w) -> float:
+    return 4.0 * w.blk * w.blk * w.d
+
+
+# --------------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples SM clock and throttle reasons with NVML (read-only) while running."""
+
+    REASONS = {
+        0x0000000000000001: "gpu_idle", 0x0000000000000002: "applications_clocks_setting",
+        0x0000000000000004: "sw_power_cap", 0x0000000000000008: "hw_slowdown",
+        0x0000000000000010: "sync_boost", 0x0000000000000020: "sw_thermal_slowdown",
+        0x0000000000000040: "hw_thermal_slowdown", 0x0000000000000080: "hw_power_brake_slowdown",
+        0x0000000000000100: "display_clock_setting",
+    }
+
+    def __init__(self, device_index: int, period: float = 0.02):
+        self.samples, self.reasons = [], set()
+        self.max_mhz = None
+        self.period = period
+        self._stop = threading.Event()
+        self._ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self._ok = True
+        except Exception:
+            self._ok = False
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                mask = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if mask & bit and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self._ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self._ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self._ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": len(self.samples)}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------ CPU baseline
+def oracle_baseline(w, Q, K, V, budget_s: float = 20.0, n_blocks: int = 48):
+    """Time the fp64 oracle on a bounded sample of the workload and scale it
+    to the whole workload (effective TFLOP/s of dense-causal-equivalent work).
+
+    Sample: the permutation of one KV head (scaled by B*Hkv), selection and
+    attention of ``n_blocks`` query blocks of one query head spread evenly
+    over the sequence (scaled by the workload's executed tiles per tile of
+    the sample)."""
+    import oracle
+    t0 = time.perf_counter()
+    perm1 = oracle.permute(Q[:, :w.G], K[:, :1], w.blk, w.seg, w.n_sink)
+    t_perm = (time.perf_counter() - t0) * w.B * w.Hkv
+    perm = np.zeros((w.B, w.Hkv, w.N), np.int32)
+    perm[:, 0] = perm1[:, 0]
+    blocks = [(0, 0, int(i)) for i in np.linspace(0, w.nb - 1, n_blocks).round().astype(int)]
+    t0 = time.perf_counter()
+    counts, lists = oracle.select(Q, K, perm, w.blk, w.seg, w.mode, density=w.density, tau=w.tau,
+                                  band=w.band, n_sink=w.n_sink, rows=blocks)
+    t_sel = (time.perf_counter() - t0) * (w.B * w.Hq * w.nb) / len(blocks)
+    t0 = time.perf_counter()
+    done = []
+    tiles_sample = 0
+    spb = w.seg // w.blk
+    for key in blocks:
+        oracle.attn_blocks(Q, K, V, perm, lists, w.blk, w.seg, [key])
+        i = key[2]
+        tiles_sample += len(lists.get(key, ())) + (i - (i // spb) * spb + 1)
+        done.append(key)
+        if time.perf_counter() - t0 > budget_s:
+            break
+    t_attn_sample = time.perf_counter() - t0
+    # executed tiles of the whole workload, estimated from the sample's density
+    n_rows = w.B * w.Hq * w.nb
+    t_attn = t_attn_sample / max(len(done), 1) * n_rows
+    total = t_perm + t_sel + t_attn
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([int(x.get("num_threads", 1)) for x in threadpool_info()] + [1])
+    except Exception:
+        cores = os.cpu_count() or 1
+    return {
+        "value": dense_causal_flops(w) / total / 1e12,
+        "unit": "TFLOP/s",
+        "cores": cores,
+        "kind": "oracle",
+        "sample": (f"fp64 numpy oracle: permutation of 1 of {w.B * w.Hkv} KV heads, selection + attention of "
+                   f"{len(done)} query blocks of head 0 spread over N={w.N}; scaled to all "
+                   f"{n_rows} query blocks; est. full run {total:.0f} s"),
+        "est_total_s": total,
+    }
+
+
+# ------------------------------------------------------------------- GPU arm
+def run_pbs(args):
+    import torch
+    import torch.distributed as dist
+
+    import permuted_block_sparse_b200 as pbs
+    from permuted_block_sparse_b200 import synth
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    dev = torch.device("cuda", local if world > 1 else torch.cuda.current_device())
+    torch.cuda.set_device(dev)
+    pbs.load()
+
+    w = synth.WORKLOADS[args.workload]
+    Qn, Kn, Vn, _ = synth.make_inputs(w, seed=w.seed + rank)
+    Q = torch.from_numpy(Qn).to(torch.bfloat16).to(dev)
+    K = torch.from_numpy(Kn).to(torch.bfloat16).to(dev)
+    V = torch.from_numpy(Vn).to(torch.bfloat16).to(dev)
+    s = torch.cuda.current_stream()
+    dt = w.tau if w.mode == "tau" else w.density
+    cap = max(1, pbs.select_capacity(w.N, w.blk, w.seg, w.mode, dt, w.band, w.n_sink))
+    perm = torch.empty((w.B, w.Hkv, w.N), dtype=torch.int32, device=dev)
+    counts = torch.empty((w.B, w.Hq, w.nb), dtype=torch.int32, device=dev)
+    idx = torch.empty((w.B, w.Hq, w.nb, cap), dtype=torch.int32, device=dev)
+    O = torch.empty_like(Q)
+    lse = torch.empty((w.B, w.Hq, w.N), dtype=torch.float32, device=dev)
+    ws_p = torch.empty(pbs.workspace_size(pbs.PBS_OP_PERMUTE, Q, K, w.blk, w.seg) + 256, dtype=torch.uint8, device=dev)
+    ws_s = torch.empty(pbs.workspace_size(pbs.PBS_OP_SELECT, Q, K, w.blk, w.seg) + 256, dtype=torch.uint8, device=dev)
+    stats = torch.zeros(2, dtype=torch.int64, device=dev)
+    launches_per_step = 6   # 2 permute + 3 select + 1 attention kernels
+
+    ev = {k: [] for k in ("p0", "p1", "s1", "a1")}
+
+    def step(record=False, st=None):
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(4)] if record else None
+        if record:
+            e[0].record(s)
+        pbs.pbs_permute(Q, K, w.blk, w.seg, w.n_sink, perm=perm, ws=ws_p)
+        if record:
+            e[1].record(s)
+        pbs.pbs_select(Q, K, perm, w.blk, w.seg, w.mode, dt, w.band, w.n_sink, cap=cap, counts=counts,
+                       idx=idx, ws=ws_s)
+        if record:
+            e[2].record(s)
+        pbs.pbs_attn_fwd(Q, K, V, perm, counts, idx, w.blk, w.seg, out=O, lse=lse, stats=st)
+        if record:
+            e[3].record(s)
+            for k, x in zip(("p0", "p1", "s1", "a1"), e):
+                ev[k].append(x)
+
+    # executed tiles (one counted run, outside the timed region)
+    step(st=stats)
+    pbs.pbs_check_device()
+    n_qk, n_gated = int(stats[0]), int(stats[1])
+    executed_flops = (n_qk - n_gated) * tile_flops(w) + n_gated * tile_flops(w) / 2
+    causal_tiles = w.B * w.Hq * w.nb * (w.nb + 1) // 2
+
+    for _ in range(max(args.warmup, 0)):
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev.index) as clk:
+        t_start.record(s)
+        for _ in range(args.steps):
+            step(record=True)
+        t_end.record(s)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    pbs.pbs_check_device()
+    ms_total = t_start.elapsed_time(t_end)
+    ms_step = ms_total / args.steps
+    ms_perm = statistics.mean(a.elapsed_time(b) for a, b in zip(ev["p0"], ev["p1"]))
+    ms_sel = statistics.mean(a.elapsed_time(b) for a, b in zip(ev["p1"], ev["s1"]))
+    ms_attn = statistics.mean(a.elapsed_time(b) for a, b in zip(ev["s1"], ev["a1"]))
+    if world > 1:
+        t = torch.tensor([ms_step, ms_attn], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_step, ms_attn = float(t[0]), float(t[1])
+
+    value = dense_causal_flops(w) * world / (ms_step * 1e-3) / 1e12
+
+    # dense causal run of the same kernel: identity permutation, seg = blk,
+    # every earlier block listed
+    dense = None
+    if not args.no_dense and rank == 0:
+        ident = torch.arange(w.N, dtype=torch.int32, device=dev).expand(w.B, w.Hkv, w.N).contiguous()
+        nb = w.nb
+        d_counts = torch.arange(nb, dtype=torch.int32, device=dev).expand(w.B, w.Hq, nb).contiguous()
+        d_idx = torch.arange(max(nb - 1, 1), dtype=torch.int32, device=dev).expand(w.B, w.Hq, nb, max(nb - 1, 1)).contiguous()
+        Od = torch.empty_like(Q)
+        for _ in range(2):
+            pbs.pbs_attn_fwd(Q, K, V, ident, d_counts, d_idx, w.blk, w.blk, out=Od, want_lse=False)
+        torch.cuda.synchronize()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        reps = 3
+        a.record(s)
+        for _ in range(reps):
+            pbs.pbs_attn_fwd(Q, K, V, ident, d_counts, d_idx, w.blk, w.blk, out=Od, want_lse=False)
+        b.record(s)
+        torch.cuda.synchronize()
+        pbs.pbs_check_device()
+        dms = a.elapsed_time(b) / reps
+        dense = {"ms": dms, "tflops": causal_tiles * tile_flops(w) / (dms * 1e-3) / 1e12,
+                 "speedup_of_sparse_step": dms / ms_step}
+        del d_idx, Od
+
+    # end to end through the C ABI with host buffers: H2D of Q, K, V from
+    # pinned memory and D2H of O inside the timed region
+    e2e = None
+    if not args.no_e2e:
+        Qh = torch.from_numpy(Qn).to(torch.bfloat16).pin_memory()
+        Kh = torch.from_numpy(Kn).to(torch.bfloat16).pin_memory()
+        Vh = torch.from_numpy(Vn).to(torch.bfloat16).pin_memory()
+        Oh = torch.empty(Qh.shape, dtype=torch.bfloat16).pin_memory()
+        Qd, Kd, Vd = torch.empty_like(Q), torch.empty_like(K), torch.empty_like(V)
+
+        def e2e_step():
+            Qd.copy_(Qh, non_blocking=True)
+            Kd.copy_(Kh, non_blocking=True)
+            Vd.copy_(Vh, non_blocking=True)
+            pbs.pbs_permute(Qd, Kd, w.blk, w.seg, w.n_sink, perm=perm, ws=ws_p)
+            pbs.pbs_select(Qd, Kd, perm, w.blk, w.seg, w.mode, dt, w.band, w.n_sink, cap=cap, counts=counts,
+                           idx=idx, ws=ws_s)
+            pbs.pbs_attn_fwd(Qd, Kd, Vd, perm, counts, idx, w.blk, w.seg, out=O, lse=lse)
+            Oh.copy_(O, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        k_e2e = max(1, min(args.steps, 5))
+        a.record(s)
+        for _ in range(k_e2e):
+            e2e_step()
+        b.record(s)
+        torch.cuda.synchronize()
+        ems = a.elapsed_time(b) / k_e2e
+        if world > 1:
+            t = torch.tensor([ems], device=dev, dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ems = float(t[0])
+        e2e = {"value": dense_causal_flops(w) * world / (ems * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "ms_per_step": ems,
+               "h2d_bytes_per_step": int(Qh.numel() * 2 + Kh.numel() * 2 + Vh.numel() * 2),
+               "d2h_bytes_per_step": int(Oh.numel() * 2)}
+
+    peaks, peak_src = load_peaks()
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    achieved = executed_flops / (ms_attn * 1e-3) / 1e12
+    traffic = None
+    tpath = os.path.join(ROOT, "profiles", "attn_fwd_traffic.json")
+    try:
+        with open(os.path.join(ROOT, "permuted_block_sparse_b200", "csrc", "attn_fwd.cu"), "rb") as f:
+            h = hashlib.sha256(f.read()).hexdigest()[:16]
+        with open(tpath) as f:
+            tj = json.load(f)
+        if tj.get("attn_fwd_sha") == h and tj.get("workload") == w.name:
+            traffic = tj.get("bytes_per_launch")
+    except Exception:
+        traffic = None
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        cpu = oracle_baseline(w, Qn, Kn, Vn)
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    out = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d, "blk": w.blk,
+                   "seg": w.seg, "selection": f"{w.mode} density={w.density} n_sink={w.n_sink}",
+                   "per_gpu": "one full workload per GPU",
+                   "l2": "inputs larger than L2 (Q alone is %.2f GB)" % (Q.numel() * 2 / 1e9)},
+        "breakdown": {"permute_ms": ms_perm, "select_ms": ms_sel, "attn_ms": ms_attn,
+                      "executed_tiles": n_qk, "gated_tiles": n_gated, "causal_tiles": causal_tiles,
+                      "density": n_qk / causal_tiles, "executed_tflops": achieved,
+                      "effective_tflops": value / world},
+        "dense_same_kernel": dense,
+        "roofline": {"bound": "tensor", "kernel": "attn_fwd", "achieved": achieved, "peak": peak,
+                     "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
+                     "peak_source": f"bf16_tflops (burst) of {peak_src}"},
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "clocks": clk.summary(),
+        "gpu_launches": launches_per_step * args.steps,
+    }
+    print(json.dumps(out), flush=True)
+
+
+# ------------------------------------------------------------ reference arm
+def run_reference(args):
+    """The oracle, as it stands, on the host cores (rank 0 only)."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from permuted_block_sparse_b200 import synth
+    w = synth.WORKLOADS[args.workload]
+    Qn, Kn, Vn, _ = synth.make_inputs(w)
+    per_step = max(2.0, 60.0 / max(args.steps + args.warmup, 1))
+    for _ in range(args.warmup):
+        oracle_baseline(w, Qn, Kn, Vn, budget_s=per_step, n_blocks=8)
+    vals, totals = [], []
+    cpu = None
+    for _ in range(args.steps):
+        cpu = oracle_baseline(w, Qn, Kn, Vn, budget_s=per_step, n_blocks=8)
+        vals.append(cpu["value"])
+        totals.append(cpu["est_total_s"])
+    value = statistics.median(vals)
+    out = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": statistics.median(totals) * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d, "blk": w.blk,
+                   "seg": w.seg},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cpu["cores"], "kind": "oracle",
+                         "sample": cpu["sample"]},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_pbs(args)
+
+
+if __name__ == "__main__":
+    main()

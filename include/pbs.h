@@ -1,0 +1,159 @@
+/*
+ * pbs.h -- C ABI of the permuted block-sparse attention prefill library
+ * (libpbs.so, sm_100a).
+ *
+ * Three calls make up one prefill-attention pass:
+ *
+ *   pbs_permute   per-segment stable sort of keys by a pooled-query score.
+ *                 "Sparser Block-Sparse Attention via Token Permutation",
+ *                 Technical Summary, 2. Segmented Permutation for Causality
+ *                 and 3. Global-Importance-Based Key Permutation.
+ *   pbs_select    per-query-block lists of permuted key blocks, by top-k
+ *                 density or by cumulative attention mass on block-pooled
+ *                 scores.  Same page, 4. Implementation (Block Selection);
+ *                 cumulative mass as in "SampleAttention", Technical Deep Dive.
+ *   pbs_attn_fwd  FlashAttention-style forward over the block's own segment
+ *                 (dense, causal, natural order) and the listed permuted
+ *                 blocks of earlier segments, gathered through the index
+ *                 list; optional exact in-tile block-max gating.
+ *                 "S2O: Early Stopping for Sparse Attention via Online
+ *                 Permutation", Technical Summary, 1. Online Permutation via
+ *                 Index-Driven Loading and 3. Kernel Implementation;
+ *                 "Block Sparse Flash Attention", Approach.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - Tensors are described by pbs_tensor: a DEVICE pointer to bfloat16
+ *    elements with logical shape [B, H, N, D] and element strides sB, sH,
+ *    sN; the D stride is 1.  Q is [B, Hq, N, D]; K, V and O are
+ *    [B, Hkv, N, D] / [B, Hq, N, D].  Hq must be a multiple of Hkv; query
+ *    head h uses KV head h / (Hq / Hkv).
+ *  - Supported: D in {64, 128}; blk in {64, 128}; seg a multiple of blk,
+ *    seg <= 8192; N a multiple of blk, N < 2^31; pointers 16-byte aligned;
+ *    strides multiples of 8 elements.  Anything else returns
+ *    PBS_ERR_UNSUPPORTED or PBS_ERR_INVALID_ARG and leaves outputs untouched.
+ *  - Index arrays are DEVICE int32, dense row-major, shapes as stated.
+ *  - Ownership: the caller owns every buffer, the stream and the workspace.
+ *    The library allocates no memory, never synchronises the stream (except
+ *    pbs_check_device) and never throws across this boundary.  Work is
+ *    enqueued on `stream` (a cudaStream_t; NULL = legacy default stream) of
+ *    the current device.
+ *  - Workspace: `ws` is a DEVICE buffer of at least pbs_workspace_size()
+ *    bytes, 256-byte aligned, used as scratch for the duration of the
+ *    enqueued work only.  Concurrent calls need distinct workspaces.
+ *  - Errors: every call returns PBS_OK (0) or a negative pbs_status; the
+ *    message of the most recent failure on the calling host thread is
+ *    returned by pbs_get_last_error().  Host-side checks happen before
+ *    anything is enqueued.  Device-side checks (an index outside its
+ *    segment or causal range, a list count above capacity, a bounded wait
+ *    that gave up) never fault: the offending access is skipped and a
+ *    sticky device error word is set, which pbs_check_device() reports.
+ */
+#ifndef PBS_H_
+#define PBS_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct pbs_tensor {
+  void* ptr;              /* device pointer to bf16 elements                 */
+  int64_t B, H, N, D;     /* logical shape                                    */
+  int64_t sB, sH, sN;     /* element strides of B, H, N (D stride is 1)       */
+} pbs_tensor;
+
+typedef enum pbs_status {
+  PBS_OK = 0,
+  PBS_ERR_INVALID_ARG = -1,   /* null pointer, inconsistent shapes          */
+  PBS_ERR_UNSUPPORTED = -2,   /* valid but outside the supported envelope   */
+  PBS_ERR_CAPACITY = -3,      /* idx capacity below the required bound      */
+  PBS_ERR_CUDA = -4,          /* a CUDA runtime call failed                 */
+  PBS_ERR_TIMEOUT = -5,       /* device: a bounded wait gave up             */
+  PBS_ERR_DEVICE_CHECK = -6   /* device: an index failed its bounds check   */
+} pbs_status;
+
+enum { PBS_OP_PERMUTE = 0, PBS_OP_SELECT = 1, PBS_OP_ATTN = 2 };
+enum { PBS_SELECT_TOPK = 0, PBS_SELECT_TAU = 1 };
+
+/* Bytes of workspace the given op needs for these shapes (0 if none).
+ * Q and K may not be NULL; only their shapes are read.                     */
+size_t pbs_workspace_size(int op, const pbs_tensor* Q, const pbs_tensor* K,
+                          int blk, int seg);
+
+/* pbs_permute: perm[b, hkv, p] = original key position at logical position
+ * p, for every (b, hkv).
+ *   1. proxy query qhat[b,hkv] = sum of the last `blk` query rows of every
+ *      query head of KV head hkv's group (fp32);
+ *   2. score s_j = qhat . K[b,hkv,j] (fp32); positions j < n_sink get +inf;
+ *   3. within each segment [t*seg, (t+1)*seg) keys are ordered by descending
+ *      score, equal scores by ascending position.  Segment order is kept, so
+ *      perm maps each segment onto itself.
+ * perm: device int32 [B, Hkv, N].  Requires N >= blk.                      */
+int pbs_permute(const pbs_tensor* Q, const pbs_tensor* K, int blk, int seg,
+                int n_sink, int32_t* perm, void* ws, size_t ws_bytes,
+                void* stream);
+
+/* Upper bound on the list length pbs_select can produce for these settings
+ * (host-only arithmetic).  Pass at least this as `cap`.                    */
+int pbs_select_capacity(int64_t N, int blk, int seg, int mode,
+                        double density_or_tau, int band, int n_sink);
+
+/* pbs_select: for each query block i of every (b, hq), the ascending list
+ * of permuted key blocks pb (blocks of segments before block i's own) that
+ * pbs_attn_fwd shall visit besides block i's own segment.
+ *   Qbar_i = sum of the rows of query block i; Kbar_pb = sum of K rows
+ *   perm[pb*blk .. pb*blk+blk-1]; block score S = Qbar_i . Kbar_pb (fp32).
+ *   Forced blocks: those holding a sink position (< n_sink) or one of the
+ *   `band` most recent keys of any query of the block.
+ *   mode PBS_SELECT_TOPK: listed count = max(|forced|, ceil(rho*(i+1)) - D_i)
+ *     with rho = density rounded to per-mille, D_i = causal blocks of block
+ *     i's own segment; forced first, then highest S, ties to lower pb.
+ *   mode PBS_SELECT_TAU: softmax (fp64) over S/(blk^2 sqrt(D)) of the
+ *     candidates and of the natural blocks of the own segment; after the
+ *     forced blocks, add candidates by descending S while the accumulated
+ *     mass (own segment included) is below tau.  tau >= 1 lists all.
+ * counts: device int32 [B, Hq, N/blk]; idx: device int32
+ * [B, Hq, N/blk, cap]; entries at and after counts[...] are unspecified.
+ * Returns PBS_ERR_CAPACITY if cap < pbs_select_capacity(...).               */
+int pbs_select(const pbs_tensor* Q, const pbs_tensor* K, const int32_t* perm,
+               int blk, int seg, int mode, double density_or_tau, int band,
+               int n_sink, int32_t* counts, int32_t* idx, int cap, void* ws,
+               size_t ws_bytes, void* stream);
+
+/* pbs_attn_fwd: O[b,hq,q] = sum_k softmax_k(scale * Q[q].K[k]) V[k] over the
+ * key set of q's block i: the keys of i's own segment up to q (natural
+ * order, causal) plus, for each listed pb, keys perm[b,hkv,pb*blk + r].
+ *   perm: device int32 [B, Hkv, N] (any source; each permuted block must
+ *     map into its own segment); counts/idx as produced by pbs_select.
+ *   gate_thr: NULL, or device fp32 [B, Hq, N/blk] in raw q.k units: a tile
+ *     other than block i's own whose largest visible raw q.k is below
+ *     gate_thr[b,hq,i] is skipped entirely (no V load, no PV, no softmax
+ *     update).
+ *   O: bf16 output, same shape as Q.  lse: NULL or device fp32 [B, Hq, N],
+ *     natural-log normaliser of the scaled logits.
+ *   stats: NULL or device int64[2], incremented by (tiles whose QK^T was
+ *     computed, tiles gated off); the caller zeroes it.
+ * Result depends on the set of listed blocks, not on their order.          */
+int pbs_attn_fwd(const pbs_tensor* Q, const pbs_tensor* K, const pbs_tensor* V,
+                 const int32_t* perm, const int32_t* counts, const int32_t* idx,
+                 int cap, int blk, int seg, const float* gate_thr,
+                 float softmax_scale, pbs_tensor* O, float* lse,
+                 long long* stats, void* ws, size_t ws_bytes, void* stream);
+
+/* Synchronises `stream`, then returns and clears the sticky device error
+ * word of the current device (PBS_OK if no device-side check failed).      */
+int pbs_check_device(void* stream);
+
+/* Message of the most recent failing call on this host thread ("" if none). */
+const char* pbs_get_last_error(void);
+
+/* Library version string. */
+const char* pbs_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* PBS_H_ */

@@ -198,12 +198,16 @@ def forced_blocks(i: int, inv_row: np.ndarray, blk: int, seg: int,
 
 def select(Q: np.ndarray, K: np.ndarray, perm: np.ndarray, blk: int, seg: int,
            mode: str, density: float = 1.0, tau: float = 1.0, band: int = 0,
-           n_sink: int = 0, rows: Optional[Iterable[Tuple[int, int, int]]] = None):
+           n_sink: int = 0, rows: Optional[Iterable[Tuple[int, int, int]]] = None,
+           trace: Optional[dict] = None):
     """Per (b, hq, i) ascending lists of permuted key blocks to attend.
 
     Returns (counts [B,Hq,nb] int32, lists dict {(b,hq,i): int32 array}).
     With ``rows`` given, only those (b, hq, i) are computed (others count 0).
-    mode "topk": budget from ``density``; mode "tau": cumulative mass."""
+    mode "topk": budget from ``density``; mode "tau": cumulative mass.
+    With ``trace`` (a dict), tau mode records per row the accumulated mass
+    before the last added block and after it, so callers can check how far
+    each stopping decision is from tau."""
     B, Hq, N, d = Q.shape
     Hkv = K.shape[1]
     G = Hq // Hkv
@@ -257,11 +261,15 @@ def select(Q: np.ndarray, K: np.ndarray, perm: np.ndarray, blk: int, seg: int,
                 Z = e_c.sum() + e_d.sum()
                 cum = (e_d.sum() + e_c[F].sum()) / Z if F else e_d.sum() / Z
                 chosen = list(F)
+                before = cum
                 for pb in order:
                     if cum >= tau:
                         break
                     chosen.append(int(pb))
+                    before = cum
                     cum += e_c[pb] / Z
+                if trace is not None:
+                    trace[(b, h, i)] = (before, cum)
         else:
             raise ValueError(mode)
         arr = np.array(sorted(chosen), np.int32)
@@ -350,6 +358,20 @@ def attn(Q, K, V, perm, lists: dict, blk: int, seg: int, scale: Optional[float] 
         O[b, h, i * blk:(i + 1) * blk] = o
         L[b, h, i * blk:(i + 1) * blk] = lse
     return O, L
+
+
+def attn_blocks(Q, K, V, perm, lists: dict, blk: int, seg: int, blocks: Iterable[Tuple[int, int, int]],
+                scale: Optional[float] = None, gate_thr: Optional[np.ndarray] = None) -> dict:
+    """{(b, hq, i): (O [blk, d], LSE [blk])} for the given query blocks only."""
+    d = Q.shape[3]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    out = {}
+    for (b, h, i) in blocks:
+        listed = lists.get((b, h, i), np.zeros(0, np.int32))
+        thr = None if gate_thr is None else float(gate_thr[b, h, i])
+        out[(b, h, i)] = attn_block(Q, K, V, perm, listed, b, h, i, blk, seg, scale, thr)
+    return out
 
 
 # --------------------------------------------------------------------------

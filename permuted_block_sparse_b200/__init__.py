@@ -1,0 +1,10 @@
+"""Permuted block-sparse attention prefill on B200 (sm_100a).
+
+The compute lives in libpbs.so (hand-written CUDA behind a C ABI, see
+include/pbs.h); this package is its Python binding plus the seeded synthetic
+input generator used by the tests and the benchmark.
+"""
+from ._binding import (EXPORTS, LIB_PATH, PBS_OP_ATTN, PBS_OP_PERMUTE, PBS_OP_SELECT,  # noqa: F401
+                       PBS_SELECT_TAU, PBS_SELECT_TOPK, PbsError, PbsTensor, describe, load,
+                       pbs_attn_fwd, pbs_check_device, pbs_permute, pbs_select, select_capacity,
+                       version, workspace_size)

@@ -1,0 +1,53 @@
+// Internal launcher interface between the C-ABI front end (api.cu) and the
+// kernel translation units.  Host-only; not part of the public ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/pbs.h"
+
+namespace pbs {
+
+struct TensorDesc {       // validated pbs_tensor, strides in elements
+  const void* ptr;
+  int64_t B, H, N, D, sB, sH, sN;
+};
+
+// pbs_permute launchers ---------------------------------------------------
+cudaError_t launch_pool_proxy_query(const TensorDesc& Q, int Hkv, int blk, float* qhat,
+                                    cudaStream_t s);
+cudaError_t launch_score_sort(const TensorDesc& K, int seg, int n_sink, const float* qhat,
+                              int32_t* perm, int* err, cudaStream_t s);
+
+// pbs_select launchers ----------------------------------------------------
+cudaError_t launch_pool_query_blocks(const TensorDesc& Q, int blk, float* qbar, cudaStream_t s);
+cudaError_t launch_pool_key_blocks(const TensorDesc& K, const int32_t* perm, int blk, int seg,
+                                   bool natural, float* kbar_perm, float* kbar_nat,
+                                   int32_t* inv, int* err, cudaStream_t s);
+struct SelectParams {
+  int B, Hq, Hkv, D, blk, seg, nb, mode, band, n_sink, cap;
+  int64_t N;
+  int64_t rho_permille;   // top-k density in per-mille
+  double tau;
+};
+cudaError_t launch_select_blocks(const SelectParams& p, const float* qbar, const float* kbar_perm,
+                                 const float* kbar_nat, const int32_t* inv, int32_t* counts,
+                                 int32_t* idx, int* err, cudaStream_t s);
+
+// pbs_attn_fwd launcher ---------------------------------------------------
+struct AttnParams {
+  TensorDesc Q, K, V, O;
+  const int32_t* perm;
+  const int32_t* counts;
+  const int32_t* idx;
+  int cap, blk, seg, nb, G;
+  const float* gate_thr;
+  float scale_log2;       // softmax scale * log2(e)
+  float* lse;
+  long long* stats;
+  int* err;
+};
+cudaError_t launch_attn_fwd(const AttnParams& p, cudaStream_t s);
+
+}  // namespace pbs

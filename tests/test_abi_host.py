@@ -1,0 +1,128 @@
+"""Host-only checks of the C ABI: the library loads, exports every function
+include/pbs.h declares, and rejects bad arguments before touching a GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import permuted_block_sparse_b200 as pbs
+from permuted_block_sparse_b200 import _binding as bd
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADERS = [os.path.join(ROOT, "include", f) for f in os.listdir(os.path.join(ROOT, "include")) if f.endswith(".h")]
+
+
+def _declared():
+    names = set()
+    for h in HEADERS:
+        text = open(h).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        for m in re.finditer(r"\b(pbs_[a-z0-9_]+)\s*\(", text):
+            names.add(m.group(1))
+    return names
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from permuted_block_sparse_b200 import build
+    build.build()
+    return pbs.load()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    declared = _declared()
+    assert {"pbs_permute", "pbs_select", "pbs_attn_fwd"} <= declared
+    for name in declared:
+        assert hasattr(lib, name), name
+    assert set(bd.EXPORTS) <= declared
+
+
+def test_version_and_last_error(lib):
+    assert "sm_100a" in pbs.version()
+    assert lib.pbs_get_last_error() is not None
+
+
+def _desc(B=1, H=2, N=256, D=128, ptr=0x1000):
+    return bd.PbsTensor(ptr, B, H, N, D, H * N * D, N * D, D)
+
+
+@pytest.mark.parametrize("mutate,code", [
+    (dict(ptr=0), -1),                 # null data
+    (dict(D=96), -2),                  # unsupported head dim
+    (dict(ptr=0x1008), -2),            # misaligned
+])
+def test_permute_rejects_bad_tensors(lib, mutate, code):
+    kw = dict(B=1, H=2, N=256, D=128, ptr=0x1000)
+    kw.update(mutate)
+    q = _desc(**kw)
+    k = _desc(B=1, H=1, N=256, D=kw["D"])
+    rc = lib.pbs_permute(ctypes.byref(q), ctypes.byref(k), 128, 256, 0, ctypes.c_void_p(0x2000),
+                         ctypes.c_void_p(0x4000), 1 << 20, None)
+    assert rc == code
+    assert lib.pbs_get_last_error()
+
+
+def test_geometry_checks(lib):
+    q, k = _desc(H=4), _desc(H=3)
+    rc = lib.pbs_permute(ctypes.byref(q), ctypes.byref(k), 128, 256, 0, ctypes.c_void_p(0x2000),
+                         ctypes.c_void_p(0x4000), 1 << 20, None)
+    assert rc == -1 and b"multiple" in lib.pbs_get_last_error()
+    q, k = _desc(H=2), _desc(H=1)
+    for blk, seg, code in ((96, 192, -2), (128, 192, -1), (128, 16384, -2)):
+        rc = lib.pbs_permute(ctypes.byref(q), ctypes.byref(k), blk, seg, 0, ctypes.c_void_p(0x2000),
+                             ctypes.c_void_p(0x4000), 1 << 20, None)
+        assert rc == code, (blk, seg)
+    # workspace too small / misaligned
+    rc = lib.pbs_permute(ctypes.byref(q), ctypes.byref(k), 128, 256, 0, ctypes.c_void_p(0x2000),
+                         ctypes.c_void_p(0x4000), 16, None)
+    assert rc == -1
+    rc = lib.pbs_permute(ctypes.byref(q), ctypes.byref(k), 128, 256, 0, ctypes.c_void_p(0x2000),
+                         ctypes.c_void_p(0x4010), 1 << 20, None)
+    assert rc == -1
+
+
+def test_select_capacity_and_errors(lib):
+    # 128K, 10 % density, one sink block: budget 100 at block 992 minus 1 own block
+    assert pbs.select_capacity(131072, 128, 4096, "topk", 0.10, 0, 128) == 99
+    assert pbs.select_capacity(32768, 128, 2048, "tau", 0.95) == 240
+    assert pbs.select_capacity(1024, 64, 256, "topk", 1.0) == 12
+    q, k = _desc(H=2, N=1024), _desc(H=1, N=1024)
+    cap = pbs.select_capacity(1024, 128, 256, "topk", 0.5)
+    rc = lib.pbs_select(ctypes.byref(q), ctypes.byref(k), ctypes.c_void_p(0x2000), 128, 256, 0, 0.5, 0, 0,
+                        ctypes.c_void_p(0x3000), ctypes.c_void_p(0x5000), cap - 1, ctypes.c_void_p(0x4000),
+                        1 << 30, None)
+    assert rc == -3
+    rc = lib.pbs_select(ctypes.byref(q), ctypes.byref(k), ctypes.c_void_p(0x2000), 128, 256, 7, 0.5, 0, 0,
+                        ctypes.c_void_p(0x3000), ctypes.c_void_p(0x5000), cap, ctypes.c_void_p(0x4000),
+                        1 << 30, None)
+    assert rc == -1
+
+
+def test_workspace_sizes(lib):
+    q, k = _desc(B=1, H=32, N=131072), _desc(B=1, H=8, N=131072)
+    assert lib.pbs_workspace_size(0, ctypes.byref(q), ctypes.byref(k), 128, 4096) == 8 * 128 * 4
+    nb = 1024
+    expect = 32 * nb * 128 * 4 + 2 * 8 * nb * 128 * 4 + 8 * 131072 * 4
+    assert lib.pbs_workspace_size(1, ctypes.byref(q), ctypes.byref(k), 128, 4096) == expect
+
+
+def test_attn_rejects_mismatched_output(lib):
+    q, k, v = _desc(H=2), _desc(H=1), _desc(H=1)
+    o = _desc(H=2, N=128)
+    rc = lib.pbs_attn_fwd(ctypes.byref(q), ctypes.byref(k), ctypes.byref(v), ctypes.c_void_p(0x2000),
+                          ctypes.c_void_p(0x3000), ctypes.c_void_p(0x5000), 4, 128, 256, None, 0.088,
+                          ctypes.byref(o), None, None, None, 0, None)
+    assert rc == -1 and b"O shape" in lib.pbs_get_last_error()
+    o = _desc(H=2)
+    rc = lib.pbs_attn_fwd(ctypes.byref(q), ctypes.byref(k), ctypes.byref(v), ctypes.c_void_p(0x2000),
+                          ctypes.c_void_p(0x3000), ctypes.c_void_p(0x5000), 4, 128, 256, None, -1.0,
+                          ctypes.byref(o), None, None, None, 0, None)
+    assert rc == -1
+
+
+def test_binding_refuses_cpu_tensors(lib):
+    import torch
+    x = torch.zeros(1, 1, 128, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        pbs.pbs_permute(x, x, 64, 128)
