@@ -96,6 +96,22 @@ int pbs_permute(const pbs_tensor* Q, const pbs_tensor* K, int blk, int seg,
                 int n_sink, int32_t* perm, void* ws, size_t ws_bytes,
                 void* stream);
 
+/* pbs_permute_noalloc: the same permutation as pbs_permute, for callers
+ * that cannot allocate device memory when they call (for example a runtime
+ * whose device memory is all reserved by its own allocator, or a plugin
+ * interface that passes a kernel its inputs and outputs but no workspace).
+ * The pages have no counterpart: this is a deployment convenience.
+ * Its scratch is a fixed 256 KiB device array inside libpbs.so (held by
+ * every GPU that loads the library until the process exits), so
+ * B * Hkv * D must not exceed 65536; larger inputs return PBS_ERR_CAPACITY.
+ * The call allocates nothing.  Its first call on a device looks up the
+ * array's device address with that device current; make that first call
+ * before any stream capture.  All calls on a device share the array and it
+ * keeps the last call's contents (each call overwrites what it reads), so
+ * calls whose GPU work may overlap race and must not be issued together.    */
+int pbs_permute_noalloc(const pbs_tensor* Q, const pbs_tensor* K, int blk, int seg,
+                        int n_sink, int32_t* perm, void* stream);
+
 /* Upper bound on the list length pbs_select can produce for these settings
  * (host-only arithmetic).  Pass at least this as `cap`.                    */
 int pbs_select_capacity(int64_t N, int blk, int seg, int mode,

@@ -112,6 +112,26 @@ int64_t rho_permille(double density) { return static_cast<int64_t>(std::llround(
 
 }  // namespace
 
+namespace pbs {
+
+int api_fail(int code, const char* msg) { return fail(code, "%s", msg); }
+
+int api_ok() { return ok(); }
+
+int* api_device_error_word() { return device_error_word(); }
+
+int api_validate_permute(const pbs_tensor* Qt, const pbs_tensor* Kt, int blk, int seg, int n_sink,
+                         const int32_t* perm, TensorDesc* Q, TensorDesc* K) {
+  int rc;
+  if ((rc = check_tensor(Qt, "Q", Q)) || (rc = check_tensor(Kt, "K", K))) return rc;
+  if ((rc = check_geometry(*Q, *K, blk, seg))) return rc;
+  if (!perm) return fail(PBS_ERR_INVALID_ARG, "perm is null");
+  if (n_sink < 0) return fail(PBS_ERR_INVALID_ARG, "n_sink %d < 0", n_sink);
+  return PBS_OK;
+}
+
+}  // namespace pbs
+
 extern "C" {
 
 const char* pbs_version(void) { return "pbs 0.1 (sm_100a)"; }

@@ -35,6 +35,15 @@ cudaError_t launch_select_blocks(const SelectParams& p, const float* qbar, const
                                  const float* kbar_nat, const int32_t* inv, int32_t* counts,
                                  int32_t* idx, int* err, cudaStream_t s);
 
+// Front-end helpers shared by C-ABI entry points defined outside api.cu.
+// They set the calling thread's last-error message like the entry points in
+// api.cu do.
+int api_fail(int code, const char* msg);
+int api_ok();
+int* api_device_error_word();
+int api_validate_permute(const pbs_tensor* Qt, const pbs_tensor* Kt, int blk, int seg, int n_sink,
+                         const int32_t* perm, TensorDesc* Q, TensorDesc* K);
+
 // pbs_attn_fwd launcher ---------------------------------------------------
 struct AttnParams {
   TensorDesc Q, K, V, O;
