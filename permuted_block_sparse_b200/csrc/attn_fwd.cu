@@ -4,23 +4,37 @@
 // Technical Summary:
 //   1. Online Permutation via Index-Driven Loading -- K/V stay in their HBM
 //      layout; an index list says which (non-contiguous) rows to load, and
-//      the kernel gathers those rows into shared memory;
+//      the kernel gathers those rows into on-chip memory;
 //   3. Kernel Implementation -- Pass 1 runs dense causal attention over the
 //      query block's own segment and builds the online-softmax state
-//      (m, l, acc); Pass 2 continues from that state over prefix key blocks
+//      (m, l, acc); Pass 2 continues from that state over earlier key blocks
 //      in permuted order.
 // "Block Sparse Flash Attention", Approach: the exact tile maximum of QK^T
 // is compared with a per-(head, query block) threshold; below it the tile
-// is dropped before the V load and the PV product.
+// adds nothing (no PV product, no softmax update).
 //
-// sm_100a design (this file): one CTA per (query block, query head, batch),
-// 128 threads.  K/V rows of a tile (natural or permuted) are gathered with
-// 16-byte cp.async into 128B-swizzled shared-memory tiles; QK^T and PV run
-// on the 5th-generation tensor cores (tcgen05.mma, bf16 in, fp32 in tensor
-// memory); each thread owns one query row of S / O in tensor memory, so the
-// online softmax needs no cross-thread reduction; P is written back to
-// tensor memory as bf16 and consumed directly as the A operand of PV.
+// sm_100a design.  One CTA per work item = (query block i, batch b, a pair
+// of query heads h0, h0+1 of the same GQA group).  The two heads share K/V,
+// so the CTA walks the UNION of their tile lists (the own segment's natural
+// blocks, then the listed permuted blocks in ascending order) and gathers
+// every K/V tile once for both heads.  Roles (384 threads):
+//   warp 0       tcgen05 MMA issuer (one thread) and tensor-memory owner;
+//   warps 1-3    producer: 16-byte cp.async row gathers of Q once and of the
+//                K and V tiles into a 2-stage ring of 128B-swizzled tiles;
+//   warps 4-7    softmax for head slot 0, warps 8-11 for head slot 1: each
+//                thread owns one query row of S and O in tensor memory.
+// Tensor memory (512 columns): S0 | S1 | O0 | O1, 128 columns each; P (bf16)
+// overwrites the first half of S and feeds PV as the A operand straight
+// from tensor memory.  K and V have separate 2-stage rings: a K stage is
+// released as soon as the QK^T of its tile are done, a V stage after the
+// PVs, so each gather has about two tiles of time to land.  The MMA thread
+// is event driven: it issues whichever QK^T or PV is ready, so that while
+// one softmax warpgroup works on its tile the tensor core works for the
+// other head.  All waits are bounded; a shared abort flag makes
+// every role of the CTA give up together.
 #include <math.h>
+
+#include <algorithm>
 
 #include "pbs_common.cuh"
 #include "pbs_internal.h"
@@ -28,23 +42,23 @@
 namespace pbs {
 namespace {
 
-constexpr int kThreads = 128;
+constexpr int kThreads = 384;
 constexpr int kM = 128;               // query rows per MMA tile
-constexpr uint32_t kTmemCols = 256;   // S/P: cols [0,128), O: cols [128, 128+D)
+constexpr int kProducerThreads = 96;  // warps 1-3
+constexpr int kStages = 2;
 constexpr float kRescaleSlack = 8.0f; // keep the running max while within 2^8
 
 template <int D, int BLK>
-struct Smem {
+struct Cfg {
   static constexpr int kQBytes = (D / 64) * kM * 128;
   static constexpr int kKVBytes = (D / 64) * BLK * 128;
-  static constexpr int kQ = 0;
-  static constexpr int kK = kQ + kQBytes;
-  static constexpr int kV = kK + kKVBytes;
-  static constexpr int kEnd = kV + kKVBytes;
-  // + alignment slack; at least 90 KB so that no more than two CTAs share an
-  // SM, which keeps their tensor-memory allocations (256 columns each) within
-  // the SM's 512 columns and tcgen05.alloc never has to wait.
-  static constexpr int kTotal = (kEnd + 1024) > 92160 ? (kEnd + 1024) : 92160;
+  static constexpr int kQ0 = 0;
+  static constexpr int kK = 2 * kQBytes;
+  static constexpr int kV = kK + kStages * kKVBytes;
+  static constexpr int kEnd = kV + kStages * kKVBytes;
+  // Above half the SM's shared memory, so one CTA per SM: its 512 tensor-
+  // memory columns are then always available and tcgen05.alloc never waits.
+  static constexpr int kMinSmem = 120 * 1024;
 };
 
 __device__ __forceinline__ float warp_max(float v) {
@@ -52,279 +66,494 @@ __device__ __forceinline__ float warp_max(float v) {
   return v;
 }
 
+struct Shared {
+  uint64_t bar_q;
+  uint64_t bar_k[kStages], bar_v[kStages], bar_kempty[kStages], bar_vempty[kStages];
+  uint64_t bar_s[2], bar_p[2], bar_o[2], bar_fin;
+  uint32_t tmem_base;
+  int abort;
+  int n_union;
+  int skip[2][2];
+  float red[2][4];
+};
+
 template <int D, int BLK>
-__global__ void __launch_bounds__(kThreads) attn_fwd_kernel(AttnParams p) {
-  using L = Smem<D, BLK>;
+__global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
+  using C = Cfg<D, BLK>;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  __shared__ uint64_t mma_bar;
-  __shared__ uint32_t tmem_slot;
-  __shared__ int32_t rowpos[BLK];
-  __shared__ float red[4];
+  uint32_t* sched = reinterpret_cast<uint32_t*>(smem + C::kEnd);
+  __shared__ Shared sh;
+  __shared__ uint32_t bm[2][256];          // candidate bitmaps (ncand <= 8192)
+  __shared__ int32_t rowbuf[kStages][BLK];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  // Heavy query blocks (more tiles) first.
-  const int i = p.nb - 1 - static_cast<int>(blockIdx.x);
-  const int hq = blockIdx.y, b = blockIdx.z;
-  const int hk = hq / p.G;
+  const int Hq = p.G * static_cast<int>(p.K.H);
+  const int npair = (p.G + 1) / 2;
+  // Work order: all items of one (batch, KV head) before the next, so that
+  // head's K/V (the tiles every item gathers) stays resident in L2; within
+  // it, heavy query blocks (more tiles) first, then the head pair.
+  const int per_bh = p.nb * npair;
+  const int bh = static_cast<int>(blockIdx.x) / per_bh;
+  const int rem = static_cast<int>(blockIdx.x) % per_bh;
+  const int i = p.nb - 1 - rem / npair;
+  const int pr = rem % npair;
+  const int b = bh / static_cast<int>(p.K.H);
+  const int hk = bh % static_cast<int>(p.K.H);
+  const int h0 = hk * p.G + 2 * pr;
+  const bool has1 = 2 * pr + 1 < p.G;
   const int spb = p.seg / BLK;
   const int s = i / spb;
+  const int ncand = s * spb;
+  const int n_diag = i - s * spb + 1;
   const int64_t q0 = static_cast<int64_t>(i) * BLK;
   const int64_t N = p.Q.N;
 
-  const uint32_t sQ = smem_u32(smem + L::kQ);
-  const uint32_t sK = smem_u32(smem + L::kK);
-  const uint32_t sV = smem_u32(smem + L::kV);
+  const uint32_t sQ0 = smem_u32(smem + C::kQ0);
+  const uint32_t sK = smem_u32(smem + C::kK);
+  const uint32_t sV = smem_u32(smem + C::kV);
 
+  // ------------------------------------------------------------------ setup
   if (warp == 0) {
-    tmem_alloc(&tmem_slot, kTmemCols);
+    tmem_alloc(&sh.tmem_base, 512);
     tmem_relinquish();
-  }
-  if (tid == 0) {
-    mbar_init(&mma_bar, 1);
-    fence_mbar_init();
+    // union of the two heads' lists as a bitmap, then an ascending schedule
+    int cnt[2] = {0, 0};
+    for (int h = 0; h < 2; ++h) {
+      if (h == 1 && !has1) break;
+      const int64_t row = (static_cast<int64_t>(b) * Hq + h0 + h) * p.nb + i;
+      int c = p.counts[row];
+      if (c < 0 || c > p.cap) {
+        if (lane == 0) set_error(p.err, kErrDeviceCheck);
+        c = 0;
+      }
+      cnt[h] = c;
+    }
+    const int words = (ncand + 31) >> 5;
+    for (int w = lane; w < words; w += 32) {
+      bm[0][w] = 0u;
+      bm[1][w] = 0u;
+    }
+    __syncwarp();
+    for (int h = 0; h < 2; ++h) {
+      const int32_t* list = p.idx + ((static_cast<int64_t>(b) * Hq + h0 + h) * p.nb + i) * p.cap;
+      for (int e = lane; e < cnt[h]; e += 32) {
+        const int pb = list[e];
+        if (pb < 0 || pb >= ncand) {
+          set_error(p.err, kErrDeviceCheck);
+          continue;
+        }
+        atomicOr(&bm[h][pb >> 5], 1u << (pb & 31));
+      }
+    }
+    __syncwarp();
+    int total = 0;
+    for (int base = 0; base < words; base += 32) {
+      const int w = base + lane;
+      const uint32_t m0 = w < words ? bm[0][w] : 0u, m1 = w < words ? bm[1][w] : 0u;
+      uint32_t u = m0 | m1;
+      const int c = __popc(u);
+      int incl = c;
+      for (int off = 1; off < 32; off <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += y;
+      }
+      int o = total + incl - c;
+      while (u) {
+        const int bit = __ffs(u) - 1;
+        u &= u - 1;
+        const uint32_t mask = ((m0 >> bit) & 1u) | (((m1 >> bit) & 1u) << 1);
+        sched[o++] = static_cast<uint32_t>(w * 32 + bit) | (mask << 30);
+      }
+      total += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) {
+      sh.n_union = total;
+      sh.abort = 0;
+      mbar_init(&sh.bar_q, kProducerThreads);
+      for (int st = 0; st < kStages; ++st) {
+        mbar_init(&sh.bar_k[st], kProducerThreads);
+        mbar_init(&sh.bar_v[st], kProducerThreads);
+        mbar_init(&sh.bar_kempty[st], 1);
+        mbar_init(&sh.bar_vempty[st], 1);
+      }
+      for (int h = 0; h < 2; ++h) {
+        mbar_init(&sh.bar_s[h], 1);
+        mbar_init(&sh.bar_p[h], 128);
+        mbar_init(&sh.bar_o[h], 1);
+      }
+      mbar_init(&sh.bar_fin, 1);
+      fence_mbar_init();
+    }
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = tmem_slot;
-  const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-  const uint32_t tS = tmem, tP = tmem, tO = tmem + 128;
+  const uint32_t tmem = sh.tmem_base;
+  const int T = n_diag + sh.n_union;
+  const uint32_t both = has1 ? 3u : 1u;
+  volatile int* abort_flag = &sh.abort;
+  // tile t: natural block i-t for t < n_diag, else sched[t - n_diag]
+  auto tile_mask = [&](int t) -> uint32_t { return t < n_diag ? both : (sched[t - n_diag] >> 30); };
 
-  // ---- Q tile: rows q0 .. q0+BLK-1, padded with zeros to 128 rows.
-  {
-    const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(p.Q.ptr) + b * p.Q.sB + hq * p.Q.sH;
+  if (warp >= 1 && warp <= 3) {
+    // ============================================================ producer
+    const int pt = tid - 32;
+    const __nv_bfloat16* kb = static_cast<const __nv_bfloat16*>(p.K.ptr) + b * p.K.sB + hk * p.K.sH;
+    const __nv_bfloat16* vb = static_cast<const __nv_bfloat16*>(p.V.ptr) + b * p.V.sB + hk * p.V.sH;
+    const int32_t* prow = p.perm + (static_cast<int64_t>(b) * p.K.H + hk) * N;
     constexpr int CH = D / 8;
-    for (int id = tid; id < kM * CH; id += kThreads) {
-      const int r = id / CH, c = id % CH;
-      const bool valid = r < BLK;
-      const __nv_bfloat16* src = valid ? qb + (q0 + r) * p.Q.sN + c * 8 : qb;
-      cp_async16_zfill(sQ + (c / 8) * (kM * 128) + sw128_offset(r, c % 8), src, valid);
-    }
-    cp_async_commit();
-  }
-
-  const int cnt_raw = p.counts[(static_cast<int64_t>(b) * (p.G * p.K.H) + hq) * p.nb + i];
-  int cnt = cnt_raw;
-  if (cnt < 0 || cnt > p.cap) {
-    if (tid == 0) set_error(p.err, kErrDeviceCheck);
-    cnt = 0;
-  }
-  const int32_t* list = p.idx + ((static_cast<int64_t>(b) * (p.G * p.K.H) + hq) * p.nb + i) * p.cap;
-  const int32_t* prow = p.perm + (static_cast<int64_t>(b) * p.K.H + hk) * N;
-  const int n_diag = i - s * spb + 1;
-  const int n_tiles = n_diag + cnt;
-  const float thr = p.gate_thr ? p.gate_thr[(static_cast<int64_t>(b) * (p.G * p.K.H) + hq) * p.nb + i]
-                               : -INFINITY;
-
-  const __nv_bfloat16* kb = static_cast<const __nv_bfloat16*>(p.K.ptr) + b * p.K.sB + hk * p.K.sH;
-  const __nv_bfloat16* vb = static_cast<const __nv_bfloat16*>(p.V.ptr) + b * p.V.sB + hk * p.V.sH;
-
-  const int r = warp * 32 + lane;      // this thread's query row in the tile
-  float m_run = -INFINITY, l_run = 0.f;
-  bool o_init = false;
-  uint32_t phase = 0;
-  int n_qk = 0, n_gated = 0;
-  bool aborted = false;
-
-  for (int t = 0; t < n_tiles && !aborted; ++t) {
-    // Pass 1 (t < n_diag): natural blocks of the own segment, from block i
-    // down; Pass 2: listed permuted blocks of earlier segments.
-    const bool is_diag = t < n_diag;
-    const int j = is_diag ? i - t : 0;
-    int pb = -1;
-    if (!is_diag) {
-      pb = list[t - n_diag];
-      if (pb < 0 || pb >= s * spb) {
-        if (tid == 0) set_error(p.err, kErrDeviceCheck);
-        continue;
+    // Q tiles of both heads (rows >= BLK zero-filled when BLK < 128)
+    for (int h = 0; h < (has1 ? 2 : 1); ++h) {
+      const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(p.Q.ptr) + b * p.Q.sB + (h0 + h) * p.Q.sH;
+      const uint32_t dst = sQ0 + h * C::kQBytes;
+      for (int id = pt; id < kM * CH; id += kProducerThreads) {
+        const int r = id / CH, c = id % CH;
+        const bool valid = r < BLK;
+        cp_async16_zfill(dst + (c / 8) * (kM * 128) + sw128_offset(r, c % 8),
+                         valid ? qb + (q0 + r) * p.Q.sN + c * 8 : qb, valid);
       }
     }
-    if (tid < BLK) {
-      int64_t x;
-      if (is_diag) {
-        x = static_cast<int64_t>(j) * BLK + tid;
-      } else {
-        const int64_t lp = static_cast<int64_t>(pb) * BLK + tid;
-        const int64_t lo = (lp / p.seg) * p.seg;
-        x = prow[lp];
-        if (x < lo || x >= lo + p.seg || x >= N) {
-          set_error(p.err, kErrDeviceCheck);
-          x = lo;                      // in bounds, inside the segment
+    cp_async_mbar_arrive(&sh.bar_q);
+    // Row indices of a tile: natural rows, or the permutation's entries for
+    // a permuted block.  Loaded one tile ahead into registers and checked
+    // when used, so the load latency overlaps the previous tile.
+    constexpr int RPT = (BLK + kProducerThreads - 1) / kProducerThreads;
+    int32_t nxt[RPT];
+    auto fetch_rows = [&](int t) {
+#pragma unroll
+      for (int q = 0; q < RPT; ++q) {
+        const int r = pt + q * kProducerThreads;
+        if (r < BLK && t >= n_diag)
+          nxt[q] = prow[static_cast<int64_t>(sched[t - n_diag] & 0x3FFFFFFFu) * BLK + r];
+      }
+    };
+    if (T > 0) fetch_rows(0);
+    for (int t = 0; t < T; ++t) {
+      const int st = t & 1;
+      const bool ok = t < kStages || mbar_wait_or_abort(&sh.bar_kempty[st], ((t >> 1) - 1) & 1, p.err, abort_flag);
+      if (named_sync_or(1, kProducerThreads, !ok)) break;   // all producer threads leave together
+      const bool nat = t < n_diag;
+      const int id0 = nat ? i - t : static_cast<int>(sched[t - n_diag] & 0x3FFFFFFFu);
+#pragma unroll
+      for (int q = 0; q < RPT; ++q) {
+        const int r = pt + q * kProducerThreads;
+        if (r >= BLK) continue;
+        int64_t x;
+        if (nat) {
+          x = static_cast<int64_t>(id0) * BLK + r;
+        } else {
+          const int64_t lo = ((static_cast<int64_t>(id0) * BLK + r) / p.seg) * p.seg;
+          x = nxt[q];
+          if (x < lo || x >= lo + p.seg || x >= N) {
+            set_error(p.err, kErrDeviceCheck);
+            x = lo;
+          }
+        }
+        rowbuf[st][r] = static_cast<int32_t>(x);
+      }
+      named_sync(1, kProducerThreads);
+      const uint32_t dk = sK + st * C::kKVBytes, dv = sV + st * C::kKVBytes;
+      for (int id = pt; id < BLK * CH; id += kProducerThreads) {
+        const int r = id / CH, c = id % CH;
+        cp_async16(dk + (c / 8) * (BLK * 128) + sw128_offset(r, c % 8), kb + rowbuf[st][r] * p.K.sN + c * 8);
+      }
+      cp_async_mbar_arrive(&sh.bar_k[st]);        // arrives when this thread's copies land
+      const bool okv = t < kStages || mbar_wait_or_abort(&sh.bar_vempty[st], ((t >> 1) - 1) & 1, p.err, abort_flag);
+      if (named_sync_or(1, kProducerThreads, !okv)) break;
+      for (int id = pt; id < BLK * CH; id += kProducerThreads) {
+        const int r = id / CH, c = id % CH;
+        cp_async16(dv + (c / 8) * (BLK * 128) + sw128_offset(r, c % 8), vb + rowbuf[st][r] * p.V.sN + c * 8);
+      }
+      cp_async_mbar_arrive(&sh.bar_v[st]);
+      if (t + 1 < T) fetch_rows(t + 1);
+    }
+    cp_async_wait_all();
+  } else if (warp == 0) {
+    // ========================================================= MMA issuer
+    if (lane == 0) {
+      bool ok = mbar_wait_or_abort(&sh.bar_q, 0, p.err, abort_flag);
+      fence_proxy_async();   // cp.async (generic proxy) writes -> tensor-core reads
+      tc_fence_after();
+      constexpr uint32_t idesc_qk = idesc_bf16(kM, BLK, false);
+      constexpr uint32_t idesc_pv = idesc_bf16(kM, D, true);
+      const int nh = has1 ? 2 : 1;
+      // Per head: next tile needing QK^T, tile whose PV is pending, QK count.
+      int nq[2] = {T, T}, pend[2] = {-1, -1}, kh[2] = {0, 0};
+      bool o_init[2] = {false, false};
+      auto next_tile = [&](int h, int from) {
+        int t = from;
+        while (t < T && !((tile_mask(t) >> h) & 1u)) ++t;
+        return t;
+      };
+      for (int h = 0; h < nh; ++h) nq[h] = next_tile(h, 0);
+      // Per ring stage: the tile it holds and how many heads still need it,
+      // and how many of its fill phases have been observed.  A stage holds
+      // tiles st, st+2, st+4, ... in turn; a tile's phase is tested only when
+      // it is the next one due on its stage, since a parity test cannot tell
+      // a phase two fills ahead from the current one.
+      int ktile[kStages] = {-1, -1}, kleft[kStages] = {0, 0}, kseen[kStages] = {0, 0};
+      int vtile[kStages] = {-1, -1}, vleft[kStages] = {0, 0}, vseen[kStages] = {0, 0};
+      auto landed = [&](uint64_t* bars, int* seen, int t) -> bool {
+        const int st = t & 1, due = st + 2 * seen[st];
+        if (t < due) return true;                        // observed earlier, still held
+        if (t > due) return false;                       // an earlier fill is not observed yet
+        if (!mbar_test_wait(&bars[st], seen[st] & 1)) return false;
+        ++seen[st];
+        fence_proxy_async();   // the fill's cp.async (generic proxy) writes -> tensor-core reads
+        return true;
+      };
+      uint32_t idle = 0;
+      // Event-driven issue: whichever of PV_h (P ready, V landed) or QK_h
+      // (previous PV_h issued, K landed) can go, goes.  QK_h(t) is always
+      // issued after PV_h of the head's previous tile, so P (which lives in
+      // S's columns) has been consumed before S is overwritten.
+      while (ok) {
+        bool pending = false, progress = false;
+        for (int h = 0; h < nh; ++h) {
+          if (pend[h] >= 0) {
+            pending = true;
+            const int t = pend[h], st = t & 1;
+            if (mbar_test_wait(&sh.bar_p[h], (kh[h] - 1) & 1) && landed(sh.bar_v, vseen, t)) {
+              tc_fence_after();
+              if (!sh.skip[h][(kh[h] - 1) & 1]) {
+                const uint32_t tP = tmem + h * 128;
+                const uint32_t tO = tmem + 256 + h * 128;
+                const uint32_t vbase = sV + st * C::kKVBytes;
+#pragma unroll
+                for (int kk = 0; kk < BLK / 16; ++kk) {
+                  const uint64_t bd = sdesc_sw128(vbase + kk * 2048, BLK * 128, 1024);
+                  mma_ts(tO, tP + kk * 8, bd, idesc_pv, (o_init[h] || kk > 0) ? 1u : 0u);
+                }
+                o_init[h] = true;
+              }
+              if (vtile[st] != t) {
+                vtile[st] = t;
+                vleft[st] = __popc(tile_mask(t));
+              }
+              if (--vleft[st] == 0) tc_commit(&sh.bar_vempty[st]);
+              pend[h] = -1;
+              progress = true;
+            }
+          }
+          if (pend[h] < 0 && nq[h] < T) {
+            pending = true;
+            const int t = nq[h], st = t & 1;
+            if (landed(sh.bar_k, kseen, t)) {
+              tc_fence_after();
+              const uint32_t qbase = sQ0 + h * C::kQBytes;
+              const uint32_t kbase = sK + st * C::kKVBytes;
+              const uint32_t tS = tmem + h * 128;
+#pragma unroll
+              for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t half = kk / 4, koff = (kk % 4) * 32;
+                const uint64_t a = sdesc_sw128(qbase + half * (kM * 128) + koff, 16, 1024);
+                const uint64_t bd = sdesc_sw128(kbase + half * (BLK * 128) + koff, 16, 1024);
+                mma_ss(tS, a, bd, idesc_qk, kk > 0 ? 1u : 0u);
+              }
+              tc_commit(&sh.bar_s[h]);
+              ++kh[h];
+              if (ktile[st] != t) {
+                ktile[st] = t;
+                kleft[st] = __popc(tile_mask(t));
+              }
+              if (--kleft[st] == 0) tc_commit(&sh.bar_kempty[st]);
+              pend[h] = t;
+              nq[h] = next_tile(h, t + 1);
+              progress = true;
+            }
+          }
+        }
+        if (!pending) break;
+        if (progress) {
+          idle = 0;
+        } else if (++idle >= 4u * kSpinLimit) {
+          set_error(p.err, kErrTimeout);
+          *abort_flag = 1;
+          ok = false;
+        } else if ((idle & 63u) == 0 && *abort_flag) {
+          ok = false;
         }
       }
-      rowpos[tid] = static_cast<int32_t>(x);
+      for (int h = 0; h < nh; ++h)
+        if (kh[h] > 0) tc_commit(&sh.bar_o[h]);
+      tc_commit(&sh.bar_fin);
+      // drain: every MMA of this CTA has completed before tensor memory is freed
+      mbar_wait(&sh.bar_fin, 0, p.err);
     }
-    __syncthreads();
-    {
-      constexpr int CH = D / 8;
-      for (int id = tid; id < BLK * CH; id += kThreads) {
-        const int rr = id / CH, c = id % CH;
-        const int64_t x = rowpos[rr];
-        const uint32_t off = (c / 8) * (BLK * 128) + sw128_offset(rr, c % 8);
-        cp_async16(sK + off, kb + x * p.K.sN + c * 8);
-        cp_async16(sV + off, vb + x * p.V.sN + c * 8);
-      }
-      cp_async_commit();
-      cp_async_wait_all();
-      fence_proxy_async();
-    }
-    __syncthreads();
-
-    // ---- S = Q K^T into tensor memory.
-    if (tid == 0) {
+    __syncwarp();
+  } else {
+    // ============================================================ softmax
+    const int h = (warp - 4) >> 2;                  // head slot
+    const int r = tid - 128 - h * 128;              // query row = TMEM lane
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + h * 128 + lane_off;
+    const uint32_t tO = tmem + 256 + h * 128 + lane_off;
+    const int hq = h0 + h;
+    const bool active = h == 0 || has1;
+    const float thr =
+        (active && p.gate_thr) ? p.gate_thr[(static_cast<int64_t>(b) * Hq + hq) * p.nb + i] : -INFINITY;
+    float m_run = -INFINITY, l_run = 0.f;
+    bool o_init = false;
+    int k = 0, n_qk = 0, n_gated = 0;
+    bool ok = true;
+    for (int t = 0; active && ok && t < T; ++t) {
+      if (!((tile_mask(t) >> h) & 1u)) continue;
+      ok = mbar_wait_or_abort(&sh.bar_s[h], k & 1, p.err, abort_flag);
+      ok = !named_sync_or(2 + h, 128, !ok);          // the warpgroup leaves together
+      if (!ok) break;
       tc_fence_after();
-      constexpr uint32_t idesc = idesc_bf16(kM, BLK, false);
+      ++n_qk;
+      // One pass over S in 32-column chunks.  P = 2^(s*scale - m) is taken
+      // against a running max m that starts at the row's max so far; when a
+      // chunk's max exceeds m by more than 2^8, m moves up and the P columns
+      // already written for this tile are rescaled in place (rare after the
+      // first tile).  So P stays below 2^8 and S is read once.  The tile's
+      // raw max decides the gate at the end; a gated tile leaves m, l and O
+      // as they were.
+      const bool causal = t == 0;
+      float rmax = -INFINITY, psum = 0.f, m_t = m_run;
+#pragma unroll 1
+      for (int c = 0; c < BLK / 32; ++c) {
+        uint32_t x[32], u[16];
+        tmem_ld32(tS + c * 32, x);
+        float cmax = -INFINITY;
 #pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        const uint32_t half = kk / 4, koff = (kk % 4) * 32;
-        const uint64_t a = sdesc_sw128(sQ + half * (kM * 128) + koff, 16, 1024);
-        const uint64_t bd = sdesc_sw128(sK + half * (BLK * 128) + koff, 16, 1024);
-        mma_ss(tS, a, bd, idesc, kk > 0 ? 1u : 0u);
+        for (int e = 0; e < 32; ++e) {
+          float v = __uint_as_float(x[e]);
+          if (causal && c * 32 + e > r) v = -INFINITY;
+          x[e] = __float_as_uint(v);
+          cmax = fmaxf(cmax, v);
+        }
+        rmax = fmaxf(rmax, cmax);
+        const float cm = cmax * p.scale_log2;
+        const bool up = cm > (m_t == -INFINITY ? -INFINITY : m_t + kRescaleSlack);
+        if (__any_sync(0xffffffffu, up)) {
+          const float m_new = up ? cm : m_t;
+          const float beta = ex2(m_t - m_new);       // 0 when m_t was -inf
+          if (c > 0 && __any_sync(0xffffffffu, beta != 1.0f)) {
+            tmem_st_wait();                           // earlier P stores of this thread landed
+            for (int q = 0; q < c; ++q) {             // rescale this tile's P so far
+              uint32_t w[32];
+              tmem_ld32(tS + q * 16, w);             // columns q*16 .. q*16+31 hold P
+#pragma unroll
+              for (int e = 0; e < 16; ++e) {
+                const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[e]));
+                w[e] = pack_bf16x2(f.x * beta, f.y * beta);
+              }
+              tmem_st16(tS + q * 16, *reinterpret_cast<const uint32_t(*)[16]>(&w[0]));
+            }
+          }
+          psum *= beta;
+          m_t = m_new;
+        }
+        const float m_use = m_t == -INFINITY ? 0.f : m_t;
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float a0 = ex2(fmaf(__uint_as_float(x[2 * e]), p.scale_log2, -m_use));
+          const float a1 = ex2(fmaf(__uint_as_float(x[2 * e + 1]), p.scale_log2, -m_use));
+          psum += a0 + a1;
+          u[e] = pack_bf16x2(a0, a1);
+        }
+        tmem_st16(tS + c * 16, u);
       }
-      tc_commit(&mma_bar);
-    }
-    const bool ok1 = mbar_wait(&mma_bar, phase, p.err);
-    phase ^= 1;
-    if (__syncthreads_or(!ok1)) {
-      aborted = true;
-      break;
-    }
-    tc_fence_after();
-    ++n_qk;
-
-    // ---- softmax on this thread's row.
-    float sv[BLK];
-#pragma unroll
-    for (int c = 0; c < BLK / 32; ++c) {
-      uint32_t u[32];
-      tmem_ld32(tS + lane_off + c * 32, u);
-#pragma unroll
-      for (int e = 0; e < 32; ++e) sv[c * 32 + e] = __uint_as_float(u[e]);
-    }
-    const bool causal_tile = is_diag && j == i;
-    float rmax = -INFINITY;
-#pragma unroll
-    for (int c = 0; c < BLK; ++c) {
-      const bool vis = !causal_tile || c <= r;
-      if (!vis) sv[c] = -INFINITY;
-      rmax = fmaxf(rmax, sv[c]);
-    }
-    if (p.gate_thr && !causal_tile) {
-      float wm = warp_max(r < BLK ? rmax : -INFINITY);
-      if (lane == 0) red[warp] = wm;
-      __syncthreads();
-      const float tmax = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
-      __syncthreads();
-      if (tmax < thr) {
-        ++n_gated;
-        tc_fence_before();             // S reads done before the next QK^T overwrites S
-        continue;                      // tile dropped: no V, no PV, no state update
+      if (p.gate_thr && !causal) {
+        const float wm = warp_max(r < BLK ? rmax : -INFINITY);
+        if (lane == 0) sh.red[h][warp & 3] = wm;
+        named_sync(2 + h, 128);
+        const float tmax = fmaxf(fmaxf(sh.red[h][0], sh.red[h][1]), fmaxf(sh.red[h][2], sh.red[h][3]));
+        named_sync(2 + h, 128);
+        if (tmax < thr) {
+          ++n_gated;
+          tmem_st_wait();
+          if (r == 0) sh.skip[h][k & 1] = 1;
+          tc_fence_before();
+          mbar_arrive(&sh.bar_p[h]);
+          ++k;
+          continue;
+        }
       }
-    }
-    const float mx = rmax * p.scale_log2;
-    const float m_new = (m_run == -INFINITY || mx > m_run + kRescaleSlack) ? fmaxf(mx, m_run) : m_run;
-    const float alpha = ex2(m_run - m_new);
-    float psum = 0.f;
-    uint32_t packed[BLK / 2];
+      const float m_new = m_t;
+      const float alpha = ex2(m_run - m_new);
+      if (o_init && __any_sync(0xffffffffu, alpha != 1.0f)) {
+        // PV of this head's previous tile has completed: the S-ready barrier
+        // tracks every MMA issued before this tile's QK^T.
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t u[32];
+          tmem_ld32(tO + c * 32, u);
 #pragma unroll
-    for (int c = 0; c < BLK; c += 2) {
-      const float p0 = ex2(fmaf(sv[c], p.scale_log2, -m_new));
-      const float p1 = ex2(fmaf(sv[c + 1], p.scale_log2, -m_new));
-      psum += p0 + p1;
-      packed[c / 2] = pack_bf16x2(p0, p1);
+          for (int e = 0; e < 32; ++e) u[e] = __float_as_uint(__uint_as_float(u[e]) * alpha);
+          tmem_st32(tO + c * 32, u);
+        }
+      }
+      l_run = l_run * alpha + psum;
+      m_run = m_new;
+      tmem_st_wait();
+      if (r == 0) sh.skip[h][k & 1] = 0;
+      tc_fence_before();
+      mbar_arrive(&sh.bar_p[h]);
+      o_init = true;
+      ++k;
     }
-    l_run = l_run * alpha + psum;
-    m_run = m_new;
-    if (o_init && __any_sync(0xffffffffu, alpha != 1.0f)) {
-#pragma unroll
+    // ---- epilogue: O / l -> bf16, LSE
+    if (active && ok && k > 0) {
+      ok = mbar_wait_or_abort(&sh.bar_o[h], 0, p.err, abort_flag);
+      ok = !named_sync_or(2 + h, 128, !ok);
+      tc_fence_after();
+    }
+    if (active && ok && o_init) {
+      const float inv_l = 1.0f / l_run;
+      __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(const_cast<void*>(p.O.ptr)) + b * p.O.sB +
+                          hq * p.O.sH + (q0 + r) * p.O.sN;
+#pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
         uint32_t u[32];
-        tmem_ld32(tO + lane_off + c * 32, u);
+        tmem_ld32(tO + c * 32, u);
+        if (r < BLK) {
 #pragma unroll
-        for (int e = 0; e < 32; ++e) u[e] = __float_as_uint(__uint_as_float(u[e]) * alpha);
-        tmem_st32(tO + lane_off + c * 32, u);
-      }
-    }
-#pragma unroll
-    for (int c = 0; c < BLK / 64; ++c) {
-      uint32_t u[32];
-#pragma unroll
-      for (int e = 0; e < 32; ++e) u[e] = packed[c * 32 + e];
-      tmem_st32(tP + lane_off + c * 32, u);
-    }
-    tmem_st_wait();
-    tc_fence_before();
-    __syncthreads();
-
-    // ---- O += P V.
-    if (tid == 0) {
-      tc_fence_after();
-      constexpr uint32_t idesc = idesc_bf16(kM, D, true);
-#pragma unroll
-      for (int kk = 0; kk < BLK / 16; ++kk) {
-        const uint64_t bd = sdesc_sw128(sV + kk * 2048, BLK * 128, 1024);
-        mma_ts(tO, tP + kk * 8, bd, idesc, (o_init || kk > 0) ? 1u : 0u);
-      }
-      tc_commit(&mma_bar);
-    }
-    const bool ok2 = mbar_wait(&mma_bar, phase, p.err);
-    phase ^= 1;
-    if (__syncthreads_or(!ok2)) {
-      aborted = true;
-      break;
-    }
-    tc_fence_after();
-    o_init = true;
-  }
-
-  // ---- epilogue: O / l -> bf16, LSE.
-  if (!aborted && o_init) {
-    const float inv_l = 1.0f / l_run;
-    __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(const_cast<void*>(p.O.ptr)) + b * p.O.sB +
-                        hq * p.O.sH + (q0 + r) * p.O.sN;
-#pragma unroll
-    for (int c = 0; c < D / 32; ++c) {
-      uint32_t u[32];
-      tmem_ld32(tO + lane_off + c * 32, u);
-      if (r < BLK) {
-#pragma unroll
-        for (int e = 0; e < 32; e += 8) {
-          uint4 v;
-          v.x = pack_bf16x2(__uint_as_float(u[e + 0]) * inv_l, __uint_as_float(u[e + 1]) * inv_l);
-          v.y = pack_bf16x2(__uint_as_float(u[e + 2]) * inv_l, __uint_as_float(u[e + 3]) * inv_l);
-          v.z = pack_bf16x2(__uint_as_float(u[e + 4]) * inv_l, __uint_as_float(u[e + 5]) * inv_l);
-          v.w = pack_bf16x2(__uint_as_float(u[e + 6]) * inv_l, __uint_as_float(u[e + 7]) * inv_l);
-          *reinterpret_cast<uint4*>(ob + c * 32 + e) = v;
+          for (int e = 0; e < 32; e += 8) {
+            uint4 v;
+            v.x = pack_bf16x2(__uint_as_float(u[e + 0]) * inv_l, __uint_as_float(u[e + 1]) * inv_l);
+            v.y = pack_bf16x2(__uint_as_float(u[e + 2]) * inv_l, __uint_as_float(u[e + 3]) * inv_l);
+            v.z = pack_bf16x2(__uint_as_float(u[e + 4]) * inv_l, __uint_as_float(u[e + 5]) * inv_l);
+            v.w = pack_bf16x2(__uint_as_float(u[e + 6]) * inv_l, __uint_as_float(u[e + 7]) * inv_l);
+            *reinterpret_cast<uint4*>(ob + c * 32 + e) = v;
+          }
         }
       }
+      if (p.lse && r < BLK)
+        p.lse[(static_cast<int64_t>(b) * Hq + hq) * N + q0 + r] = (m_run + log2f(l_run)) * 0.69314718055994531f;
     }
-    if (p.lse && r < BLK)
-      p.lse[(static_cast<int64_t>(b) * (p.G * p.K.H) + hq) * N + q0 + r] =
-          (m_run + log2f(l_run)) * 0.69314718055994531f;
-  }
-  if (tid == 0 && p.stats) {
-    atomicAdd(reinterpret_cast<unsigned long long*>(p.stats), static_cast<unsigned long long>(n_qk));
-    atomicAdd(reinterpret_cast<unsigned long long*>(p.stats) + 1,
-              static_cast<unsigned long long>(n_gated));
+    if (active && r == 0 && p.stats) {
+      atomicAdd(reinterpret_cast<unsigned long long*>(p.stats), static_cast<unsigned long long>(n_qk));
+      atomicAdd(reinterpret_cast<unsigned long long*>(p.stats) + 1, static_cast<unsigned long long>(n_gated));
+    }
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
+    tmem_dealloc(tmem, 512);
   }
 }
 
 template <int D, int BLK>
 cudaError_t launch_typed(const AttnParams& p, cudaStream_t s) {
-  using L = Smem<D, BLK>;
+  using C = Cfg<D, BLK>;
+  // schedule: at most min(candidates, 2 * cap) permuted tiles per item
+  const int max_union = std::min(p.nb, 2 * p.cap);
+  int smem = 1024 + C::kEnd + 4 * max_union;
+  smem = smem < C::kMinSmem ? C::kMinSmem : smem;
+  if (smem + 4096 > 227 * 1024) return cudaErrorInvalidValue;   // + static shared memory
   cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D, BLK>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, L::kTotal);
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  dim3 grid(static_cast<unsigned>(p.nb), static_cast<unsigned>(p.Q.H), static_cast<unsigned>(p.Q.B));
-  attn_fwd_kernel<D, BLK><<<grid, kThreads, L::kTotal, s>>>(p);
+  const int npair = (p.G + 1) / 2;
+  const int64_t items = static_cast<int64_t>(p.nb) * p.Q.B * p.K.H * npair;
+  if (items >= (1ll << 31)) return cudaErrorInvalidValue;
+  attn_fwd_kernel<D, BLK><<<static_cast<unsigned>(items), kThreads, smem, s>>>(p);
   return cudaGetLastError();
 }
 
@@ -332,6 +561,7 @@ cudaError_t launch_typed(const AttnParams& p, cudaStream_t s) {
 
 cudaError_t launch_attn_fwd(const AttnParams& p, cudaStream_t s) {
   const int D = static_cast<int>(p.Q.D);
+  if (p.nb > 8192) return cudaErrorInvalidValue;
   if (D == 128 && p.blk == 128) return launch_typed<128, 128>(p, s);
   if (D == 128 && p.blk == 64) return launch_typed<128, 64>(p, s);
   if (D == 64 && p.blk == 128) return launch_typed<64, 128>(p, s);
