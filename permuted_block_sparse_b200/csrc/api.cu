@@ -86,7 +86,7 @@ int check_geometry(const pbs::TensorDesc& Q, const pbs::TensorDesc& K, int blk, 
 }
 
 struct SelectWs {
-  size_t qbar, kperm, knat, inv, total;
+  size_t qbar, kperm, knat, inv, scores, total;
 };
 
 SelectWs select_ws(const pbs::TensorDesc& Q, const pbs::TensorDesc& K, int blk) {
@@ -96,7 +96,8 @@ SelectWs select_ws(const pbs::TensorDesc& Q, const pbs::TensorDesc& K, int blk) 
   w.kperm = w.qbar + align256(static_cast<size_t>(Q.B * Q.H) * nb * Q.D * 4);
   w.knat = w.kperm + align256(static_cast<size_t>(K.B * K.H) * nb * K.D * 4);
   w.inv = w.knat + align256(static_cast<size_t>(K.B * K.H) * nb * K.D * 4);
-  w.total = w.inv + align256(static_cast<size_t>(K.B * K.H) * K.N * 4);
+  w.scores = w.inv + align256(static_cast<size_t>(K.B * K.H) * K.N * 4);
+  w.total = w.scores + align256(static_cast<size_t>(Q.B * Q.H) * nb * nb * 4);
   return w;
 }
 
@@ -228,6 +229,7 @@ int pbs_select(const pbs_tensor* Qt, const pbs_tensor* Kt, const int32_t* perm, 
   float* kperm = reinterpret_cast<float*>(base + w.kperm);
   float* knat = reinterpret_cast<float*>(base + w.knat);
   int32_t* inv = reinterpret_cast<int32_t*>(base + w.inv);
+  float* scores = reinterpret_cast<float*>(base + w.scores);
   cudaError_t e = pbs::launch_pool_query_blocks(Q, blk, qbar, s);
   if (e != cudaSuccess) return cuda_fail(e, "pool_query_blocks launch");
   e = pbs::launch_pool_key_blocks(K, perm, blk, seg, mode == PBS_SELECT_TAU, kperm, knat, inv, err, s);
@@ -247,7 +249,7 @@ int pbs_select(const pbs_tensor* Qt, const pbs_tensor* Kt, const int32_t* perm, 
   p.N = Q.N;
   p.rho_permille = rho_permille(density_or_tau);
   p.tau = density_or_tau;
-  e = pbs::launch_select_blocks(p, qbar, kperm, knat, inv, counts, idx, err, s);
+  e = pbs::launch_select_blocks(p, qbar, kperm, knat, inv, scores, counts, idx, err, s);
   if (e != cudaSuccess) return cuda_fail(e, "select_blocks launch");
   return ok();
 }

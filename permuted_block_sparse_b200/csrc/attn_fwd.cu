@@ -272,10 +272,24 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
     cp_async_wait_all();
   } else if (warp == 0) {
     // ========================================================= MMA issuer
-    if (lane == 0) {
-      bool ok = mbar_wait_or_abort(&sh.bar_q, 0, p.err, abort_flag);
-      fence_proxy_async();   // cp.async (generic proxy) writes -> tensor-core reads
+    // The whole warp runs the issue loop with warp-uniform state, so MMA
+    // descriptors stay warp-uniform; lane 0 observes each barrier (and so
+    // acquires the data) and alone issues the MMAs and commits.
+    const bool leader = lane == 0;
+    auto test = [&](uint64_t* bar, uint32_t parity) -> bool {
+      bool v = false;
+      if (leader) v = mbar_test_wait(bar, parity);
+      return __shfl_sync(0xffffffffu, v, 0);
+    };
+    bool ok = true;
+    {
+      bool v = true;
+      if (leader) v = mbar_wait_or_abort(&sh.bar_q, 0, p.err, abort_flag);
+      ok = __shfl_sync(0xffffffffu, v, 0);
+      if (leader) fence_proxy_async();   // cp.async (generic proxy) writes -> tensor-core reads
       tc_fence_after();
+    }
+    {
       constexpr uint32_t idesc_qk = idesc_bf16(kM, BLK, false);
       constexpr uint32_t idesc_pv = idesc_bf16(kM, D, true);
       const int nh = has1 ? 2 : 1;
@@ -299,9 +313,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
         const int st = t & 1, due = st + 2 * seen[st];
         if (t < due) return true;                        // observed earlier, still held
         if (t > due) return false;                       // an earlier fill is not observed yet
-        if (!mbar_test_wait(&bars[st], seen[st] & 1)) return false;
+        if (!test(&bars[st], seen[st] & 1)) return false;
         ++seen[st];
-        fence_proxy_async();   // the fill's cp.async (generic proxy) writes -> tensor-core reads
+        if (leader) fence_proxy_async();                 // fill's cp.async writes -> tensor-core reads
         return true;
       };
       uint32_t idle = 0;
@@ -315,16 +329,20 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
           if (pend[h] >= 0) {
             pending = true;
             const int t = pend[h], st = t & 1;
-            if (mbar_test_wait(&sh.bar_p[h], (kh[h] - 1) & 1) && landed(sh.bar_v, vseen, t)) {
+            if (test(&sh.bar_p[h], (kh[h] - 1) & 1) && landed(sh.bar_v, vseen, t)) {
               tc_fence_after();
-              if (!sh.skip[h][(kh[h] - 1) & 1]) {
+              int skip = 0;
+              if (leader) skip = sh.skip[h][(kh[h] - 1) & 1];      // lane 0 acquired bar_p
+              if (!__shfl_sync(0xffffffffu, skip, 0)) {
                 const uint32_t tP = tmem + h * 128;
                 const uint32_t tO = tmem + 256 + h * 128;
                 const uint32_t vbase = sV + st * C::kKVBytes;
+                if (leader) {
+                  const uint64_t bd0 = sdesc_sw128(vbase, BLK * 128, 1024);
+                  mma_ts(tO, tP, bd0, idesc_pv, o_init[h] ? 1u : 0u);
 #pragma unroll
-                for (int kk = 0; kk < BLK / 16; ++kk) {
-                  const uint64_t bd = sdesc_sw128(vbase + kk * 2048, BLK * 128, 1024);
-                  mma_ts(tO, tP + kk * 8, bd, idesc_pv, (o_init[h] || kk > 0) ? 1u : 0u);
+                  for (int kk = 1; kk < BLK / 16; ++kk)
+                    mma_ts(tO, tP + kk * 8, sdesc_add(bd0, kk * 2048), idesc_pv, 1u);
                 }
                 o_init[h] = true;
               }
@@ -332,7 +350,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
                 vtile[st] = t;
                 vleft[st] = __popc(tile_mask(t));
               }
-              if (--vleft[st] == 0) tc_commit(&sh.bar_vempty[st]);
+              if (--vleft[st] == 0 && leader) tc_commit(&sh.bar_vempty[st]);
               pend[h] = -1;
               progress = true;
             }
@@ -345,20 +363,23 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
               const uint32_t qbase = sQ0 + h * C::kQBytes;
               const uint32_t kbase = sK + st * C::kKVBytes;
               const uint32_t tS = tmem + h * 128;
+              if (leader) {
+                const uint64_t a0 = sdesc_sw128(qbase, 16, 1024);
+                const uint64_t b0 = sdesc_sw128(kbase, 16, 1024);
 #pragma unroll
-              for (int kk = 0; kk < D / 16; ++kk) {
-                const uint32_t half = kk / 4, koff = (kk % 4) * 32;
-                const uint64_t a = sdesc_sw128(qbase + half * (kM * 128) + koff, 16, 1024);
-                const uint64_t bd = sdesc_sw128(kbase + half * (BLK * 128) + koff, 16, 1024);
-                mma_ss(tS, a, bd, idesc_qk, kk > 0 ? 1u : 0u);
+                for (int kk = 0; kk < D / 16; ++kk) {
+                  const uint32_t half = kk / 4, koff = (kk % 4) * 32;
+                  mma_ss(tS, sdesc_add(a0, half * (kM * 128) + koff), sdesc_add(b0, half * (BLK * 128) + koff),
+                         idesc_qk, kk > 0 ? 1u : 0u);
+                }
+                tc_commit(&sh.bar_s[h]);
               }
-              tc_commit(&sh.bar_s[h]);
               ++kh[h];
               if (ktile[st] != t) {
                 ktile[st] = t;
                 kleft[st] = __popc(tile_mask(t));
               }
-              if (--kleft[st] == 0) tc_commit(&sh.bar_kempty[st]);
+              if (--kleft[st] == 0 && leader) tc_commit(&sh.bar_kempty[st]);
               pend[h] = t;
               nq[h] = next_tile(h, t + 1);
               progress = true;
@@ -369,18 +390,22 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
         if (progress) {
           idle = 0;
         } else if (++idle >= 4u * kSpinLimit) {
-          set_error(p.err, kErrTimeout);
-          *abort_flag = 1;
+          if (leader) {
+            set_error(p.err, kErrTimeout);
+            *abort_flag = 1;
+          }
           ok = false;
-        } else if ((idle & 63u) == 0 && *abort_flag) {
-          ok = false;
+        } else if ((idle & 63u) == 0) {
+          ok = !__shfl_sync(0xffffffffu, *abort_flag, 0);
         }
       }
-      for (int h = 0; h < nh; ++h)
-        if (kh[h] > 0) tc_commit(&sh.bar_o[h]);
-      tc_commit(&sh.bar_fin);
-      // drain: every MMA of this CTA has completed before tensor memory is freed
-      mbar_wait(&sh.bar_fin, 0, p.err);
+      if (leader) {
+        for (int h = 0; h < nh; ++h)
+          if (kh[h] > 0) tc_commit(&sh.bar_o[h]);
+        tc_commit(&sh.bar_fin);
+        // drain: every MMA of this CTA has completed before tensor memory is freed
+        mbar_wait(&sh.bar_fin, 0, p.err);
+      }
     }
     __syncwarp();
   } else {
@@ -405,7 +430,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
       if (!ok) break;
       tc_fence_after();
       ++n_qk;
-      // One pass over S in 32-column chunks.  P = 2^(s*scale - m) is taken
+      // One pass over S in 64-column chunks.  P = 2^(s*scale - m) is taken
       // against a running max m that starts at the row's max so far; when a
       // chunk's max exceeds m by more than 2^8, m moves up and the P columns
       // already written for this tile are rescaled in place (rare after the
@@ -415,16 +440,25 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
       const bool causal = t == 0;
       float rmax = -INFINITY, psum = 0.f, m_t = m_run;
 #pragma unroll 1
-      for (int c = 0; c < BLK / 32; ++c) {
-        uint32_t x[32], u[16];
-        tmem_ld32(tS + c * 32, x);
+      for (int c = 0; c < BLK / 64; ++c) {
+        uint32_t x[64], u[32];
+        tmem_ld64(tS + c * 64, x);
         float cmax = -INFINITY;
+        if (causal) {
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          float v = __uint_as_float(x[e]);
-          if (causal && c * 32 + e > r) v = -INFINITY;
-          x[e] = __float_as_uint(v);
-          cmax = fmaxf(cmax, v);
+          for (int e = 0; e < 64; ++e) {
+            const float v = c * 64 + e > r ? -INFINITY : __uint_as_float(x[e]);
+            x[e] = __float_as_uint(v);
+            cmax = fmaxf(cmax, v);
+          }
+        } else {
+          // Eight independent partial maxima (a single chain is latency bound).
+          float mm[8];
+#pragma unroll
+          for (int q = 0; q < 8; ++q) mm[q] = __uint_as_float(x[q]);
+#pragma unroll
+          for (int e = 8; e < 64; ++e) mm[e & 7] = fmaxf(mm[e & 7], __uint_as_float(x[e]));
+          cmax = fmaxf(fmaxf(fmaxf(mm[0], mm[1]), fmaxf(mm[2], mm[3])), fmaxf(fmaxf(mm[4], mm[5]), fmaxf(mm[6], mm[7])));
         }
         rmax = fmaxf(rmax, cmax);
         const float cm = cmax * p.scale_log2;
@@ -434,29 +468,43 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
           const float beta = ex2(m_t - m_new);       // 0 when m_t was -inf
           if (c > 0 && __any_sync(0xffffffffu, beta != 1.0f)) {
             tmem_st_wait();                           // earlier P stores of this thread landed
-            for (int q = 0; q < c; ++q) {             // rescale this tile's P so far
-              uint32_t w[32];
-              tmem_ld32(tS + q * 16, w);             // columns q*16 .. q*16+31 hold P
+            for (int q = 0; q < 2 * c; ++q) {         // rescale this tile's P so far
+              uint32_t w[16];
+              tmem_ld16(tS + q * 16, w);             // columns q*16 .. q*16+15 hold P
 #pragma unroll
               for (int e = 0; e < 16; ++e) {
                 const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[e]));
                 w[e] = pack_bf16x2(f.x * beta, f.y * beta);
               }
-              tmem_st16(tS + q * 16, *reinterpret_cast<const uint32_t(*)[16]>(&w[0]));
+              tmem_st16(tS + q * 16, w);
             }
           }
           psum *= beta;
           m_t = m_new;
         }
         const float m_use = m_t == -INFINITY ? 0.f : m_t;
+        if (causal) {
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const float a0 = ex2(fmaf(__uint_as_float(x[2 * e]), p.scale_log2, -m_use));
-          const float a1 = ex2(fmaf(__uint_as_float(x[2 * e + 1]), p.scale_log2, -m_use));
-          psum += a0 + a1;
-          u[e] = pack_bf16x2(a0, a1);
+          for (int e = 0; e < 32; ++e) {
+            const float a0 = ex2(fmaf(__uint_as_float(x[2 * e]), p.scale_log2, -m_use));
+            const float a1 = ex2(fmaf(__uint_as_float(x[2 * e + 1]), p.scale_log2, -m_use));
+            psum += a0 + a1;
+            u[e] = pack_bf16x2(a0, a1);
+          }
+        } else {
+          // Eight independent partial sums: one running sum would make the
+          // row's 64 additions a serial chain of FADD latencies.
+          float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const float a0 = ex2(fmaf(__uint_as_float(x[2 * e]), p.scale_log2, -m_use));
+            const float a1 = ex2(fmaf(__uint_as_float(x[2 * e + 1]), p.scale_log2, -m_use));
+            ps[e & 7] += a0 + a1;
+            u[e] = pack_bf16x2(a0, a1);
+          }
+          psum += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
         }
-        tmem_st16(tS + c * 16, u);
+        tmem_st32(tS + c * 32, u);
       }
       if (p.gate_thr && !causal) {
         const float wm = warp_max(r < BLK ? rmax : -INFINITY);

@@ -32,7 +32,7 @@ struct SelectParams {
   double tau;
 };
 cudaError_t launch_select_blocks(const SelectParams& p, const float* qbar, const float* kbar_perm,
-                                 const float* kbar_nat, const int32_t* inv, int32_t* counts,
+                                 const float* kbar_nat, const int32_t* inv, float* scores, int32_t* counts,
                                  int32_t* idx, int* err, cudaStream_t s);
 
 // Front-end helpers shared by C-ABI entry points defined outside api.cu.

@@ -13,6 +13,8 @@
 #include "pbs_common.cuh"
 #include "pbs_internal.h"
 
+#include <algorithm>
+
 namespace pbs {
 namespace {
 
@@ -134,9 +136,208 @@ __device__ __forceinline__ double block_max_f64(double v, double* red) {
   return t;
 }
 
-// One CTA per (query block i, query head, batch).
-__global__ void __launch_bounds__(kSelThreads) select_blocks_kernel(
-    SelectParams p, const float* __restrict__ qbar, const float* __restrict__ kbar_perm,
+// Block scores S[b, hq, i, pb] = Qbar_i . Kbar_pb for every candidate
+// pb < candidates(i), as a register-tiled fp32 GEMM per (batch, query head):
+// 64 x 64 output tiles, 4 x 4 per thread, d in chunks of 32.  Tiles wholly
+// above the candidate triangle are skipped.  On lattice inputs every
+// partial sum is exact, so any accumulation order gives the same scores.
+constexpr int kTile = 64;
+
+__global__ void __launch_bounds__(256) block_scores_kernel(SelectParams p, const float* __restrict__ qbar,
+                                                           const float* __restrict__ kbar_perm,
+                                                           float* __restrict__ S) {
+  const int ct = blockIdx.x, rt = blockIdx.y, bh = blockIdx.z;
+  const int b = bh / p.Hq, h = bh % p.Hq, hk = h / (p.Hq / p.Hkv);
+  const int spb = p.seg / p.blk;
+  const int i_last = min((rt + 1) * kTile, p.nb) - 1;
+  const int pb0 = ct * kTile;
+  if (pb0 >= (i_last / spb) * spb) return;
+  __shared__ __align__(16) float qs[32][kTile + 4];     // [d][row]
+  __shared__ __align__(16) float ks[32][kTile + 4];     // [d][candidate]
+  const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
+  float acc[4][4];
+#pragma unroll
+  for (int u = 0; u < 4; ++u)
+#pragma unroll
+    for (int v = 0; v < 4; ++v) acc[u][v] = 0.f;
+  const float* qsrc = qbar + (static_cast<int64_t>(b) * p.Hq + h) * p.nb * p.D;
+  const float* ksrc = kbar_perm + (static_cast<int64_t>(b) * p.Hkv + hk) * p.nb * p.D;
+  for (int d0 = 0; d0 < p.D; d0 += 32) {
+    for (int x = threadIdx.x; x < kTile * 8; x += 256) {
+      const int r = x / 8, d4 = x % 8;
+      const int i = rt * kTile + r, pb = pb0 + r;
+      const float4 qv = i < p.nb ? *reinterpret_cast<const float4*>(qsrc + static_cast<int64_t>(i) * p.D + d0 + 4 * d4)
+                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+      const float4 kv = pb < p.nb ? *reinterpret_cast<const float4*>(ksrc + static_cast<int64_t>(pb) * p.D + d0 + 4 * d4)
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+      qs[4 * d4 + 0][r] = qv.x; qs[4 * d4 + 1][r] = qv.y; qs[4 * d4 + 2][r] = qv.z; qs[4 * d4 + 3][r] = qv.w;
+      ks[4 * d4 + 0][r] = kv.x; ks[4 * d4 + 1][r] = kv.y; ks[4 * d4 + 2][r] = kv.z; ks[4 * d4 + 3][r] = kv.w;
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int dd = 0; dd < 32; ++dd) {
+      const float4 a = *reinterpret_cast<const float4*>(&qs[dd][ty * 4]);
+      const float4 c = *reinterpret_cast<const float4*>(&ks[dd][tx * 4]);
+      const float av[4] = {a.x, a.y, a.z, a.w}, cv[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int v = 0; v < 4; ++v) acc[u][v] = fmaf(av[u], cv[v], acc[u][v]);
+    }
+    __syncthreads();
+  }
+  float* out = S + (static_cast<int64_t>(b) * p.Hq + h) * p.nb * p.nb;
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int i = rt * kTile + ty * 4 + u;
+    if (i >= p.nb) continue;
+    const int nc = (i / spb) * spb;
+#pragma unroll
+    for (int v = 0; v < 4; ++v) {
+      const int pb = pb0 + tx * 4 + v;
+      if (pb < nc) out[static_cast<int64_t>(i) * p.nb + pb] = acc[u][v];
+    }
+  }
+}
+
+// Forced blocks of row i as a bitmap over candidates (one warp).
+__device__ __forceinline__ void forced_bitmap(const SelectParams& p, const int32_t* irow, int i, int ncand,
+                                              uint32_t* fbits, int lane) {
+  const int words = (ncand + 31) >> 5;
+  for (int w = lane; w < words; w += 32) fbits[w] = 0u;
+  __syncwarp();
+  const int spb = p.seg / p.blk;
+  const int64_t s_start = static_cast<int64_t>(i / spb) * p.seg;
+  const int64_t sink_hi = min(static_cast<int64_t>(p.n_sink), s_start);
+  for (int64_t pos = lane; pos < sink_hi; pos += 32) {
+    const int32_t lp = irow[pos];
+    if (lp >= 0 && lp < static_cast<int64_t>(ncand) * p.blk) atomicOr(&fbits[(lp / p.blk) >> 5], 1u << ((lp / p.blk) & 31));
+  }
+  if (p.band > 0) {
+    const int64_t band_lo = max(static_cast<int64_t>(0), static_cast<int64_t>(i) * p.blk - p.band + 1);
+    for (int64_t pos = band_lo + lane; pos < s_start; pos += 32) {
+      const int32_t lp = irow[pos];
+      if (lp >= 0 && lp < static_cast<int64_t>(ncand) * p.blk) atomicOr(&fbits[(lp / p.blk) >> 5], 1u << ((lp / p.blk) & 31));
+    }
+  }
+  __syncwarp();
+}
+
+// Top-k selection, one warp per (b, hq, i) row: radix select of the `want`
+// smallest sort keys, where a forced block's key is 0 and any other block's
+// is the order-inverted score (descending score); ties at the threshold go
+// to the lowest block ids.  The chosen ids are written in ascending order.
+constexpr int kWarpsPerCta = 8;
+
+__global__ void __launch_bounds__(kWarpsPerCta * 32) select_topk_kernel(
+    SelectParams p, const float* __restrict__ S_all, const int32_t* __restrict__ inv,
+    int32_t* __restrict__ counts, int32_t* __restrict__ idx, int* err) {
+  extern __shared__ __align__(16) uint32_t fb_all[];                 // kWarpsPerCta x nbw
+  __shared__ uint32_t hist_all[kWarpsPerCta][256];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nbw = p.nb / 32 + 1;
+  uint32_t* fbits = fb_all + warp * nbw;
+  uint32_t* hist = hist_all[warp];
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * kWarpsPerCta + warp;
+  if (row >= static_cast<int64_t>(p.B) * p.Hq * p.nb) return;
+  const int i = static_cast<int>(row % p.nb);
+  const int h = static_cast<int>((row / p.nb) % p.Hq);
+  const int b = static_cast<int>(row / (static_cast<int64_t>(p.nb) * p.Hq));
+  const int hk = h / (p.Hq / p.Hkv);
+  const int spb = p.seg / p.blk;
+  const int s = i / spb, ncand = s * spb, Di = i - s * spb + 1;
+  if (ncand == 0) {
+    if (lane == 0) counts[row] = 0;
+    return;
+  }
+  const float* S = S_all + row * p.nb;
+  forced_bitmap(p, inv + (static_cast<int64_t>(b) * p.Hkv + hk) * p.N, i, ncand, fbits, lane);
+  const int words = (ncand + 31) >> 5;
+  int nf = 0;
+  for (int w = lane; w < words; w += 32) nf += __popc(fbits[w]);
+  for (int off = 16; off > 0; off >>= 1) nf += __shfl_xor_sync(0xffffffffu, nf, off);
+  const int64_t target = (p.rho_permille * (i + 1) + 999) / 1000;
+  const int want = static_cast<int>(min(max(static_cast<int64_t>(Di + nf), target) - Di, static_cast<int64_t>(ncand)));
+  if (want > p.cap) {
+    if (lane == 0) {
+      set_error(err, kErrDeviceCheck);
+      counts[row] = 0;
+    }
+    return;
+  }
+  auto key_hi = [&](int t) -> uint32_t {
+    return ((fbits[t >> 5] >> (t & 31)) & 1u) ? 0u : ~ordered_u32(S[t]);
+  };
+  uint32_t prefix = 0, pmask = 0;
+  int rank = want;
+  if (want > 0) {
+    for (int shift = 24; shift >= 0; shift -= 8) {
+      for (int q = lane; q < 256; q += 32) hist[q] = 0u;
+      __syncwarp();
+      for (int t = lane; t < ncand; t += 32) {
+        const uint32_t k = key_hi(t);
+        if ((k & pmask) == prefix) atomicAdd(&hist[(k >> shift) & 255u], 1u);
+      }
+      __syncwarp();
+      uint32_t loc[8], sum = 0;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        loc[q] = hist[lane * 8 + q];
+        sum += loc[q];
+      }
+      uint32_t incl = sum;
+      for (int off = 1; off < 32; off <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += y;
+      }
+      const uint32_t excl = incl - sum;
+      const bool mine = excl < static_cast<uint32_t>(rank) && static_cast<uint32_t>(rank) <= incl;
+      const int src = __ffs(__ballot_sync(0xffffffffu, mine)) - 1;
+      uint32_t bucket = 0, below = 0;
+      if (lane == src) {
+        uint32_t c = excl;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          if (c + loc[q] >= static_cast<uint32_t>(rank)) {
+            bucket = lane * 8 + q;
+            below = c;
+            break;
+          }
+          c += loc[q];
+        }
+      }
+      bucket = __shfl_sync(0xffffffffu, bucket, src);
+      below = __shfl_sync(0xffffffffu, below, src);
+      prefix |= bucket << shift;
+      pmask |= 255u << shift;
+      rank -= static_cast<int>(below);
+      __syncwarp();
+    }
+  }
+  int32_t* out = idx + row * p.cap;
+  int written = 0, ties = 0;
+  for (int base = 0; base < ncand && want > 0; base += 32) {
+    const int t = base + lane;
+    const uint32_t k = t < ncand ? key_hi(t) : 0xffffffffu;
+    const bool lt = t < ncand && k < prefix;
+    const bool eq = t < ncand && k == prefix;
+    const uint32_t eqm = __ballot_sync(0xffffffffu, eq);
+    const int my_tie = ties + __popc(eqm & ((1u << lane) - 1u));
+    const bool take = lt || (eq && my_tie < rank);
+    const uint32_t tm = __ballot_sync(0xffffffffu, take);
+    if (take) out[written + __popc(tm & ((1u << lane) - 1u))] = t;
+    written += __popc(tm);
+    ties += __popc(eqm);
+  }
+  if (lane == 0) counts[row] = want;
+}
+
+// Cumulative-mass selection, one CTA per (query block, query head, batch):
+// the row's candidates are sorted by (forced first, descending score, lower
+// block id) and taken in that order while the accumulated softmax mass (fp64,
+// own segment included) is below tau.
+__global__ void __launch_bounds__(kSelThreads) select_tau_kernel(
+    SelectParams p, const float* __restrict__ S_all, const float* __restrict__ qbar,
     const float* __restrict__ kbar_nat, const int32_t* __restrict__ inv,
     int32_t* __restrict__ counts, int32_t* __restrict__ idx, int* err) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -154,13 +355,14 @@ __global__ void __launch_bounds__(kSelThreads) select_blocks_kernel(
   int n2 = 1;
   while (n2 < ncand) n2 <<= 1;
   uint64_t* keys = reinterpret_cast<uint64_t*>(smem_raw);           // n2
-  double* ev = reinterpret_cast<double*>(keys + n2);                 // n2 (tau)
+  double* ev = reinterpret_cast<double*>(keys + n2);                 // n2
   float* S = reinterpret_cast<float*>(ev + n2);                      // n2
   float* q = S + n2;                                                 // D
   int* flag = reinterpret_cast<int*>(q + p.D);                       // n2
   __shared__ double red[kSelThreads / 32];
   __shared__ int sh_int[4];
-
+  const float* srow = S_all + row * p.nb;
+  for (int t = threadIdx.x; t < ncand; t += blockDim.x) S[t] = srow[t];
   const float* qsrc = qbar + row * p.D;
   for (int c = threadIdx.x; c < p.D; c += blockDim.x) q[c] = qsrc[c];
   for (int t = threadIdx.x; t < n2; t += blockDim.x) flag[t] = 0;
@@ -169,16 +371,7 @@ __global__ void __launch_bounds__(kSelThreads) select_blocks_kernel(
     sh_int[1] = ncand;
   }
   __syncthreads();
-
-  // Exact block scores (lattice inputs): one warp per candidate.
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const float* kb = kbar_perm + (static_cast<int64_t>(b) * p.Hkv + hk) * p.nb * p.D;
-  for (int pb = warp; pb < ncand; pb += kSelThreads / 32) {
-    float acc = 0.f;
-    for (int c = lane; c < p.D; c += 32) acc = fmaf(q[c], kb[static_cast<int64_t>(pb) * p.D + c], acc);
-    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-    if (lane == 0) S[pb] = acc;
-  }
   // Forced blocks: sinks and the recent-key band that fall before the own segment.
   const int64_t s_start = static_cast<int64_t>(s) * p.seg;
   const int32_t* irow = inv + (static_cast<int64_t>(b) * p.Hkv + hk) * p.N;
@@ -348,23 +541,30 @@ cudaError_t launch_pool_key_blocks(const TensorDesc& K, const int32_t* perm, int
   return cudaGetLastError();
 }
 
-size_t select_smem_bytes(int nb, int D) {
-  int n2 = 1;
-  while (n2 < nb) n2 <<= 1;
-  return static_cast<size_t>(n2) * (8 + 8 + 4 + 4) + static_cast<size_t>(D) * 4;
-}
-
 cudaError_t launch_select_blocks(const SelectParams& p, const float* qbar, const float* kbar_perm,
-                                 const float* kbar_nat, const int32_t* inv, int32_t* counts,
+                                 const float* kbar_nat, const int32_t* inv, float* scores, int32_t* counts,
                                  int32_t* idx, int* err, cudaStream_t s) {
-  const size_t smem = select_smem_bytes(p.nb, p.D);
-  cudaError_t e = cudaFuncSetAttribute(select_blocks_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
+  const int tiles = (p.nb + kTile - 1) / kTile;
+  dim3 g1(static_cast<unsigned>(tiles), static_cast<unsigned>(tiles), static_cast<unsigned>(p.B * p.Hq));
+  block_scores_kernel<<<g1, 256, 0, s>>>(p, qbar, kbar_perm, scores);
+  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  dim3 grid(static_cast<unsigned>(p.nb), static_cast<unsigned>(p.Hq), static_cast<unsigned>(p.B));
-  select_blocks_kernel<<<grid, kSelThreads, smem, s>>>(p, qbar, kbar_perm, kbar_nat, inv, counts,
-                                                       idx, err);
+  if (p.mode == PBS_SELECT_TOPK) {
+    const size_t smem = static_cast<size_t>(kWarpsPerCta) * (p.nb / 32 + 1) * 4;
+    e = cudaFuncSetAttribute(select_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    const int64_t rows = static_cast<int64_t>(p.B) * p.Hq * p.nb;
+    select_topk_kernel<<<static_cast<unsigned>((rows + kWarpsPerCta - 1) / kWarpsPerCta), kWarpsPerCta * 32, smem, s>>>(
+        p, scores, inv, counts, idx, err);
+    return cudaGetLastError();
+  }
+  int n2 = 1;
+  while (n2 < p.nb) n2 <<= 1;
+  const size_t smem = static_cast<size_t>(n2) * (8 + 8 + 4 + 4) + static_cast<size_t>(p.D) * 4;
+  e = cudaFuncSetAttribute(select_tau_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  dim3 g2(static_cast<unsigned>(p.nb), static_cast<unsigned>(p.Hq), static_cast<unsigned>(p.B));
+  select_tau_kernel<<<g2, kSelThreads, smem, s>>>(p, scores, qbar, kbar_nat, inv, counts, idx, err);
   return cudaGetLastError();
 }
 

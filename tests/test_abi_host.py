@@ -103,7 +103,9 @@ def test_workspace_sizes(lib):
     q, k = _desc(B=1, H=32, N=131072), _desc(B=1, H=8, N=131072)
     assert lib.pbs_workspace_size(0, ctypes.byref(q), ctypes.byref(k), 128, 4096) == 8 * 128 * 4
     nb = 1024
-    expect = 32 * nb * 128 * 4 + 2 * 8 * nb * 128 * 4 + 8 * 131072 * 4
+    # pooled query blocks, pooled permuted and natural key blocks, inverse
+    # permutation, block-score matrix
+    expect = 32 * nb * 128 * 4 + 2 * 8 * nb * 128 * 4 + 8 * 131072 * 4 + 32 * nb * nb * 4
     assert lib.pbs_workspace_size(1, ctypes.byref(q), ctypes.byref(k), 128, 4096) == expect
 
 
