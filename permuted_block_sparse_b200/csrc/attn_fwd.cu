@@ -337,12 +337,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
                 const uint32_t tP = tmem + h * 128;
                 const uint32_t tO = tmem + 256 + h * 128;
                 const uint32_t vbase = sV + st * C::kKVBytes;
-                if (leader) {
-                  const uint64_t bd0 = sdesc_sw128(vbase, BLK * 128, 1024);
-                  mma_ts(tO, tP, bd0, idesc_pv, o_init[h] ? 1u : 0u);
+                const uint64_t bd0 = sdesc_sw128(vbase, BLK * 128, 1024);
+                const uint32_t acc0 = o_init[h] ? 1u : 0u;
 #pragma unroll
-                  for (int kk = 1; kk < BLK / 16; ++kk)
-                    mma_ts(tO, tP + kk * 8, sdesc_add(bd0, kk * 2048), idesc_pv, 1u);
+                for (int kk = 0; kk < BLK / 16; ++kk) {
+                  const uint64_t bd = sdesc_add(bd0, kk * 2048);
+                  if (elect_one()) mma_ts(tO, tP + kk * 8, bd, idesc_pv, kk > 0 ? 1u : acc0);
                 }
                 o_init[h] = true;
               }
@@ -350,7 +350,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
                 vtile[st] = t;
                 vleft[st] = __popc(tile_mask(t));
               }
-              if (--vleft[st] == 0 && leader) tc_commit(&sh.bar_vempty[st]);
+              if (--vleft[st] == 0 && elect_one()) tc_commit(&sh.bar_vempty[st]);
               pend[h] = -1;
               progress = true;
             }
@@ -363,23 +363,22 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
               const uint32_t qbase = sQ0 + h * C::kQBytes;
               const uint32_t kbase = sK + st * C::kKVBytes;
               const uint32_t tS = tmem + h * 128;
-              if (leader) {
-                const uint64_t a0 = sdesc_sw128(qbase, 16, 1024);
-                const uint64_t b0 = sdesc_sw128(kbase, 16, 1024);
+              const uint64_t a0 = sdesc_sw128(qbase, 16, 1024);
+              const uint64_t b0 = sdesc_sw128(kbase, 16, 1024);
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                  const uint32_t half = kk / 4, koff = (kk % 4) * 32;
-                  mma_ss(tS, sdesc_add(a0, half * (kM * 128) + koff), sdesc_add(b0, half * (BLK * 128) + koff),
-                         idesc_qk, kk > 0 ? 1u : 0u);
-                }
-                tc_commit(&sh.bar_s[h]);
+              for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t half = kk / 4, koff = (kk % 4) * 32;
+                const uint64_t ad = sdesc_add(a0, half * (kM * 128) + koff);
+                const uint64_t bd = sdesc_add(b0, half * (BLK * 128) + koff);
+                if (elect_one()) mma_ss(tS, ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
               }
+              if (elect_one()) tc_commit(&sh.bar_s[h]);
               ++kh[h];
               if (ktile[st] != t) {
                 ktile[st] = t;
                 kleft[st] = __popc(tile_mask(t));
               }
-              if (--kleft[st] == 0 && leader) tc_commit(&sh.bar_kempty[st]);
+              if (--kleft[st] == 0 && elect_one()) tc_commit(&sh.bar_kempty[st]);
               pend[h] = t;
               nq[h] = next_tile(h, t + 1);
               progress = true;

@@ -4,6 +4,7 @@
 // PTX ISA's description of each instruction.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -79,6 +80,19 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
 }
 
 
+// One lane of a converged warp (elect.sync).  Issuing tcgen05.mma under it,
+// from warp-uniform control flow with warp-uniform operands, keeps the
+// per-instruction issue cost low.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n\t.reg .pred P;\n\t"
+      "elect.sync _|P, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, P;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
+}
+
 // Named barrier over `nthreads` threads (a multiple of 32); id 0 is
 // __syncthreads.
 __device__ __forceinline__ void named_sync(uint32_t id, uint32_t nthreads) {
@@ -124,6 +138,25 @@ __device__ __forceinline__ bool mbar_wait_or_abort(uint64_t* bar, uint32_t parit
   set_error(err, kErrTimeout);
   *abort = 1;
   return false;
+}
+
+// ------------------------------------------------------------------- TMA
+// Post `bytes` of expected transaction bytes on `bar` and arrive once.
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+// Gather four rows y0..y3 (each one box of the 2D tensor map: `x` .. x+63
+// columns) into 4 consecutive 128-byte rows at `dst`; the map's 128-byte
+// swizzle is applied by shared-memory address, so 4-row groups may start
+// at any 512-byte boundary of a swizzle atom.  Completes on `bar`.
+__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap* map, int x, int y0, int y1,
+                                            int y2, int y3, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3), "r"(smem_u32(bar))
+      : "memory");
 }
 
 // ---------------------------------------------------------------- cp.async
