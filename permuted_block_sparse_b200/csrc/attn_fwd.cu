@@ -70,6 +70,8 @@ struct Shared {
   uint64_t bar_q;
   uint64_t bar_k[kStages], bar_v[kStages], bar_kempty[kStages], bar_vempty[kStages];
   uint64_t bar_s[2], bar_p[2], bar_o[2], bar_fin;
+  uint64_t bar_g[2];       // gate decisions, one arrival per decided tile of a head
+  int gkeep[2][2];         // [head][decision parity]: tile kept by this head
   uint32_t tmem_base;
   int abort;
   int n_union;
@@ -184,6 +186,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
         mbar_init(&sh.bar_o[h], 1);
       }
       mbar_init(&sh.bar_fin, 1);
+      mbar_init(&sh.bar_g[0], 1);
+      mbar_init(&sh.bar_g[1], 1);
       fence_mbar_init();
     }
   }
@@ -230,43 +234,68 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
       }
     };
     if (T > 0) fetch_rows(0);
-    for (int t = 0; t < T; ++t) {
-      const int st = t & 1;
-      const bool ok = t < kStages || mbar_wait_or_abort(&sh.bar_kempty[st], ((t >> 1) - 1) & 1, p.err, abort_flag);
-      if (named_sync_or(1, kProducerThreads, !ok)) break;   // all producer threads leave together
-      const bool nat = t < n_diag;
-      const int id0 = nat ? i - t : static_cast<int>(sched[t - n_diag] & 0x3FFFFFFFu);
+    // With gating, V of tile t-1 is issued after K of tile t, once every
+    // head visiting tile t-1 has decided: a tile all of them dropped is not
+    // loaded at all (its PVs are skipped too).
+    const bool gate = p.gate_thr != nullptr;
+    int gk[2] = {0, 0};
+    for (int t = 0; t <= T; ++t) {
+      if (t < T) {
+        const int st = t & 1;
+        const bool ok = t < kStages || mbar_wait_or_abort(&sh.bar_kempty[st], ((t >> 1) - 1) & 1, p.err, abort_flag);
+        if (named_sync_or(1, kProducerThreads, !ok)) break;   // all producer threads leave together
+        const bool nat = t < n_diag;
+        const int id0 = nat ? i - t : static_cast<int>(sched[t - n_diag] & 0x3FFFFFFFu);
 #pragma unroll
-      for (int q = 0; q < RPT; ++q) {
-        const int r = pt + q * kProducerThreads;
-        if (r >= BLK) continue;
-        int64_t x;
-        if (nat) {
-          x = static_cast<int64_t>(id0) * BLK + r;
-        } else {
-          const int64_t lo = ((static_cast<int64_t>(id0) * BLK + r) / p.seg) * p.seg;
-          x = nxt[q];
-          if (x < lo || x >= lo + p.seg || x >= N) {
-            set_error(p.err, kErrDeviceCheck);
-            x = lo;
+        for (int q = 0; q < RPT; ++q) {
+          const int r = pt + q * kProducerThreads;
+          if (r >= BLK) continue;
+          int64_t x;
+          if (nat) {
+            x = static_cast<int64_t>(id0) * BLK + r;
+          } else {
+            const int64_t lo = ((static_cast<int64_t>(id0) * BLK + r) / p.seg) * p.seg;
+            x = nxt[q];
+            if (x < lo || x >= lo + p.seg || x >= N) {
+              set_error(p.err, kErrDeviceCheck);
+              x = lo;
+            }
+          }
+          rowbuf[st][r] = static_cast<int32_t>(x);
+        }
+        named_sync(1, kProducerThreads);
+        const uint32_t dk = sK + st * C::kKVBytes;
+        for (int id = pt; id < BLK * CH; id += kProducerThreads) {
+          const int r = id / CH, c = id % CH;
+          cp_async16(dk + (c / 8) * (BLK * 128) + sw128_offset(r, c % 8), kb + rowbuf[st][r] * p.K.sN + c * 8);
+        }
+        cp_async_mbar_arrive(&sh.bar_k[st]);      // arrives when this thread's copies land
+      }
+      const int tv = gate ? t - 1 : t;            // tile whose V goes now
+      if (tv >= 0 && tv < T) {
+        const int sv = tv & 1;
+        bool okv = tv < kStages || mbar_wait_or_abort(&sh.bar_vempty[sv], ((tv >> 1) - 1) & 1, p.err, abort_flag);
+        bool keep = true;
+        if (gate) {
+          keep = false;
+          const uint32_t mask = tile_mask(tv);
+          for (int h = 0; h < 2; ++h) {
+            if (!((mask >> h) & 1u)) continue;
+            okv = okv && mbar_wait_or_abort(&sh.bar_g[h], gk[h] & 1, p.err, abort_flag);
+            keep = keep || (okv && sh.gkeep[h][gk[h] & 1]);
+            ++gk[h];
           }
         }
-        rowbuf[st][r] = static_cast<int32_t>(x);
+        if (named_sync_or(1, kProducerThreads, !okv)) break;
+        if (keep) {
+          const uint32_t dv = sV + sv * C::kKVBytes;
+          for (int id = pt; id < BLK * CH; id += kProducerThreads) {
+            const int r = id / CH, c = id % CH;
+            cp_async16(dv + (c / 8) * (BLK * 128) + sw128_offset(r, c % 8), vb + rowbuf[sv][r] * p.V.sN + c * 8);
+          }
+        }
+        cp_async_mbar_arrive(&sh.bar_v[sv]);
       }
-      named_sync(1, kProducerThreads);
-      const uint32_t dk = sK + st * C::kKVBytes, dv = sV + st * C::kKVBytes;
-      for (int id = pt; id < BLK * CH; id += kProducerThreads) {
-        const int r = id / CH, c = id % CH;
-        cp_async16(dk + (c / 8) * (BLK * 128) + sw128_offset(r, c % 8), kb + rowbuf[st][r] * p.K.sN + c * 8);
-      }
-      cp_async_mbar_arrive(&sh.bar_k[st]);        // arrives when this thread's copies land
-      const bool okv = t < kStages || mbar_wait_or_abort(&sh.bar_vempty[st], ((t >> 1) - 1) & 1, p.err, abort_flag);
-      if (named_sync_or(1, kProducerThreads, !okv)) break;
-      for (int id = pt; id < BLK * CH; id += kProducerThreads) {
-        const int r = id / CH, c = id % CH;
-        cp_async16(dv + (c / 8) * (BLK * 128) + sw128_offset(r, c % 8), vb + rowbuf[st][r] * p.V.sN + c * 8);
-      }
-      cp_async_mbar_arrive(&sh.bar_v[st]);
       if (t + 1 < T) fetch_rows(t + 1);
     }
     cp_async_wait_all();
@@ -513,6 +542,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
         named_sync(2 + h, 128);
         if (tmax < thr) {
           ++n_gated;
+          if (r == 0) {
+            sh.gkeep[h][k & 1] = 0;
+            mbar_arrive(&sh.bar_g[h]);
+          }
           tmem_st_wait();
           if (r == 0) sh.skip[h][k & 1] = 1;
           tc_fence_before();
@@ -520,6 +553,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
           ++k;
           continue;
         }
+      }
+      if (p.gate_thr && r == 0) {               // kept (the diagonal tile always is)
+        sh.gkeep[h][k & 1] = 1;
+        mbar_arrive(&sh.bar_g[h]);
       }
       const float m_new = m_t;
       const float alpha = ex2(m_run - m_new);
