@@ -195,8 +195,9 @@ def run_pbs(args):
     torch.cuda.set_device(dev)
     pbs.load()
 
+    from permuted_block_sparse_b200 import shard
     w = synth.WORKLOADS[args.workload]
-    Qn, Kn, Vn, _ = synth.make_inputs(w, seed=w.seed + rank)
+    Qn, Kn, Vn, _ = synth.make_inputs(w, seed=shard.seed_for_rank(w.seed, rank))
     Q = torch.from_numpy(Qn).to(torch.bfloat16).to(dev)
     K = torch.from_numpy(Kn).to(torch.bfloat16).to(dev)
     V = torch.from_numpy(Vn).to(torch.bfloat16).to(dev)
@@ -263,9 +264,7 @@ def run_pbs(args):
     ms_sel = statistics.mean(a.elapsed_time(b) for a, b in zip(ev["p1"], ev["s1"]))
     ms_attn = statistics.mean(a.elapsed_time(b) for a, b in zip(ev["s1"], ev["a1"]))
     if world > 1:
-        t = torch.tensor([ms_step, ms_attn], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_step, ms_attn = float(t[0]), float(t[1])
+        ms_step, ms_attn = shard.max_over_ranks([ms_step, ms_attn], dist)
 
     value = dense_causal_flops(w) * world / (ms_step * 1e-3) / 1e12
 
@@ -329,9 +328,7 @@ def run_pbs(args):
         torch.cuda.synchronize()
         ems = a.elapsed_time(b) / k_e2e
         if world > 1:
-            t = torch.tensor([ems], device=dev, dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ems = float(t[0])
+            ems = shard.max_over_ranks([ems], dist)[0]
         e2e = {"value": dense_causal_flops(w) * world / (ems * 1e-3) / 1e12, "unit": "TFLOP/s",
                "ms_per_step": ems,
                "h2d_bytes_per_step": int(Qh.numel() * 2 + Kh.numel() * 2 + Vh.numel() * 2),

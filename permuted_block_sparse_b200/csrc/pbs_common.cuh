@@ -4,7 +4,6 @@
 // PTX ISA's description of each instruction.
 #pragma once
 
-#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -114,18 +113,6 @@ __device__ __forceinline__ bool named_sync_or(uint32_t id, uint32_t nthreads, bo
   return r != 0;
 }
 
-// Per-warpgroup register re-allocation (all 128 threads of the warpgroup
-// execute it).  The sum over warpgroups must not exceed what the block was
-// launched with, or the increase waits forever; launchers check that.
-template <uint32_t N>
-__device__ __forceinline__ void regs_inc() {
-  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
-}
-template <uint32_t N>
-__device__ __forceinline__ void regs_dec() {
-  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
-}
-
 // Bounded wait that also gives up as soon as another role of the CTA has
 // raised `abort` (a shared-memory flag).  Returns false if it gave up; on a
 // timeout it raises `abort` itself and sets the error word.
@@ -138,25 +125,6 @@ __device__ __forceinline__ bool mbar_wait_or_abort(uint64_t* bar, uint32_t parit
   set_error(err, kErrTimeout);
   *abort = 1;
   return false;
-}
-
-// ------------------------------------------------------------------- TMA
-// Post `bytes` of expected transaction bytes on `bar` and arrive once.
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
-               : "memory");
-}
-// Gather four rows y0..y3 (each one box of the 2D tensor map: `x` .. x+63
-// columns) into 4 consecutive 128-byte rows at `dst`; the map's 128-byte
-// swizzle is applied by shared-memory address, so 4-row groups may start
-// at any 512-byte boundary of a swizzle atom.  Completes on `bar`.
-__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap* map, int x, int y0, int y1,
-                                            int y2, int y3, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3), "r"(smem_u32(bar))
-      : "memory");
 }
 
 // ---------------------------------------------------------------- cp.async
@@ -291,39 +259,6 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
       : "r"(taddr)
       : "memory");
 }
-// tmem_ld32 that also takes a value computed from the previous chunk, so
-// the compiler cannot hoist the load above that computation (which would
-// keep several chunks' registers live at once).
-__device__ __forceinline__ void tmem_ld32_after(uint32_t taddr, uint32_t (&r)[32], float dep) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n\t"
-      "tcgen05.wait::ld.sync.aligned;"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
-        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
-        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr), "f"(dep)
-      : "memory");
-}
-
-// Asynchronous 32x32b.x32 load: the registers are NOT valid until
-// tmem_wait_ld(r) below, which names them as in/out operands so that the
-// compiler neither reads them earlier nor reuses them before the wait.
-__device__ __forceinline__ void tmem_ld32_async(uint32_t taddr, uint32_t (&r)[32]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr)
-      : "memory");
-}
-__device__ __forceinline__ void tmem_wait_ld(uint32_t (&r)[32]) {
-  asm volatile("tcgen05.wait::ld.sync.aligned;" : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31]) : : "memory");
-}
-
 // 32 lanes x 64 columns -> 64 registers per thread, wait included.
 __device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
   asm volatile(
@@ -389,24 +324,6 @@ __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
-}
-
-// 2^x on the FMA pipe, to take load off the SFU.  Cody-Waite split
-// x = n + f with n = round(x), obtained by adding and subtracting 1.5 * 2^23
-// (which rounds to an integer in fp32 and leaves n in the low mantissa bits
-// of the sum), f in [-1/2, 1/2]; 2^f from a cubic fitted for minimal
-// relative error on [-1/2, 1/2] (max 7.7e-5, below bf16's 2^-9 rounding of
-// P); 2^n applied by adding n to the exponent field (Schraudolph, "A fast,
-// compact approximation of the exponential function", 1999).  Valid for
-// -126 <= x <= 127; smaller x is clamped and gives a value below 2^-126.
-__device__ __forceinline__ float ex2_fma(float x) {
-  x = fmaxf(x, -127.0f);
-  const float t = x + 12582912.0f;
-  const float n = t - 12582912.0f;
-  const float f = x - n;
-  const float q = fmaf(fmaf(fmaf(0.05522261559963226f, f, 0.24261537194252014f), f, 0.6932516098022461f), f,
-                       0.9999275803565979f);
-  return __int_as_float(__float_as_int(q) + (__float_as_int(t) << 23));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
