@@ -61,6 +61,13 @@ def dense_causal_flops(w) -> float:
     return 2.0 * w.d * w.N * w.N * w.Hq * w.B
 
 
+def selection_label(w) -> str:
+    if w.mode == "gate":
+        return f"all earlier blocks, block-max gate calibrated to keep {w.gate_keep} tiles"
+    sel = f"topk density={w.density}" if w.mode == "topk" else f"tau={w.tau}"
+    return sel + (f" band={w.band}" if w.band else "") + (f" n_sink={w.n_sink}" if w.n_sink else "")
+
+
 def tile_flops(w) -> float:
     return 4.0 * w.blk * w.blk * w.d
 
@@ -134,22 +141,31 @@ def oracle_baseline(w, Q, K, V, budget_s: float = 20.0, n_blocks: int = 48):
     over the sequence (scaled by the workload's executed tiles per tile of
     the sample)."""
     import oracle
-    t0 = time.perf_counter()
-    perm1 = oracle.permute(Q[:, :w.G], K[:, :1], w.blk, w.seg, w.n_sink)
-    t_perm = (time.perf_counter() - t0) * w.B * w.Hkv
-    perm = np.zeros((w.B, w.Hkv, w.N), np.int32)
-    perm[:, 0] = perm1[:, 0]
     blocks = [(0, 0, int(i)) for i in np.linspace(0, w.nb - 1, n_blocks).round().astype(int)]
-    t0 = time.perf_counter()
-    counts, lists = oracle.select(Q, K, perm, w.blk, w.seg, w.mode, density=w.density, tau=w.tau,
-                                  band=w.band, n_sink=w.n_sink, rows=blocks)
-    t_sel = (time.perf_counter() - t0) * (w.B * w.Hq * w.nb) / len(blocks)
+    thr = None
+    if w.mode == "gate":
+        # no permutation or selection step: identity order, every earlier
+        # block listed, offline-calibrated thresholds
+        t_perm = t_sel = 0.0
+        perm = np.broadcast_to(np.arange(w.N, dtype=np.int32), (w.B, w.Hkv, w.N)).copy()
+        lists = {key: np.arange(key[2], dtype=np.int32) for key in blocks}
+        thr = np.load(os.path.join(ROOT, "tests", "golden", f"gate_thr_{w.name}.npy")).astype(np.float64)
+    else:
+        t0 = time.perf_counter()
+        perm1 = oracle.permute(Q[:, :w.G], K[:, :1], w.blk, w.seg, w.n_sink)
+        t_perm = (time.perf_counter() - t0) * w.B * w.Hkv
+        perm = np.zeros((w.B, w.Hkv, w.N), np.int32)
+        perm[:, 0] = perm1[:, 0]
+        t0 = time.perf_counter()
+        counts, lists = oracle.select(Q, K, perm, w.blk, w.seg, w.mode, density=w.density, tau=w.tau,
+                                      band=w.band, n_sink=w.n_sink, rows=blocks)
+        t_sel = (time.perf_counter() - t0) * (w.B * w.Hq * w.nb) / len(blocks)
     t0 = time.perf_counter()
     done = []
     tiles_sample = 0
     spb = w.seg // w.blk
     for key in blocks:
-        oracle.attn_blocks(Q, K, V, perm, lists, w.blk, w.seg, [key])
+        oracle.attn_blocks(Q, K, V, perm, lists, w.blk, w.seg, [key], gate_thr=thr)
         i = key[2]
         tiles_sample += len(lists.get(key, ())) + (i - (i // spb) * spb + 1)
         done.append(key)
@@ -170,8 +186,9 @@ def oracle_baseline(w, Q, K, V, budget_s: float = 20.0, n_blocks: int = 48):
         "unit": "TFLOP/s",
         "cores": cores,
         "kind": "oracle",
-        "sample": (f"fp64 numpy oracle: permutation of 1 of {w.B * w.Hkv} KV heads, selection + attention of "
-                   f"{len(done)} query blocks of head 0 spread over N={w.N}; scaled to all "
+        "sample": (f"fp64 numpy oracle: "
+                   + ("" if w.mode == "gate" else f"permutation of 1 of {w.B * w.Hkv} KV heads, selection + ")
+                   + f"attention of {len(done)} query blocks of head 0 spread over N={w.N}; scaled to all "
                    f"{n_rows} query blocks; est. full run {total:.0f} s"),
         "est_total_s": total,
     }
@@ -213,6 +230,19 @@ def run_pbs(args):
     ws_s = torch.empty(pbs.workspace_size(pbs.PBS_OP_SELECT, Q, K, w.blk, w.seg) + 256, dtype=torch.uint8, device=dev)
     stats = torch.zeros(2, dtype=torch.int64, device=dev)
     launches_per_step = 6   # 2 permute + 3 select + 1 attention kernels
+    # Block-max gating workloads: no permutation or selection step; every
+    # earlier block is listed and the thresholds (calibrated offline by the
+    # oracle, stored beside the tests) decide per tile.
+    gate = w.mode == "gate"
+    thr = None
+    if gate:
+        thr_path = os.path.join(ROOT, "tests", "golden", f"gate_thr_{w.name}.npy")
+        thr = torch.from_numpy(np.load(thr_path).astype(np.float32)).to(dev)
+        perm.copy_(torch.arange(w.N, dtype=torch.int32, device=dev).expand(w.B, w.Hkv, w.N))
+        counts.copy_(torch.arange(w.nb, dtype=torch.int32, device=dev).expand(w.B, w.Hq, w.nb))
+        cap = max(w.nb - 1, 1)
+        idx = torch.arange(cap, dtype=torch.int32, device=dev).expand(w.B, w.Hq, w.nb, cap).contiguous()
+        launches_per_step = 1
 
     ev = {k: [] for k in ("p0", "p1", "s1", "a1")}
 
@@ -220,14 +250,16 @@ def run_pbs(args):
         e = [torch.cuda.Event(enable_timing=True) for _ in range(4)] if record else None
         if record:
             e[0].record(s)
-        pbs.pbs_permute(Q, K, w.blk, w.seg, w.n_sink, perm=perm, ws=ws_p)
+        if not gate:
+            pbs.pbs_permute(Q, K, w.blk, w.seg, w.n_sink, perm=perm, ws=ws_p)
         if record:
             e[1].record(s)
-        pbs.pbs_select(Q, K, perm, w.blk, w.seg, w.mode, dt, w.band, w.n_sink, cap=cap, counts=counts,
-                       idx=idx, ws=ws_s)
+        if not gate:
+            pbs.pbs_select(Q, K, perm, w.blk, w.seg, w.mode, dt, w.band, w.n_sink, cap=cap, counts=counts,
+                           idx=idx, ws=ws_s)
         if record:
             e[2].record(s)
-        pbs.pbs_attn_fwd(Q, K, V, perm, counts, idx, w.blk, w.seg, out=O, lse=lse, stats=st)
+        pbs.pbs_attn_fwd(Q, K, V, perm, counts, idx, w.blk, w.seg, out=O, lse=lse, stats=st, gate_thr=thr)
         if record:
             e[3].record(s)
             for k, x in zip(("p0", "p1", "s1", "a1"), e):
@@ -308,10 +340,11 @@ def run_pbs(args):
             Qd.copy_(Qh, non_blocking=True)
             Kd.copy_(Kh, non_blocking=True)
             Vd.copy_(Vh, non_blocking=True)
-            pbs.pbs_permute(Qd, Kd, w.blk, w.seg, w.n_sink, perm=perm, ws=ws_p)
-            pbs.pbs_select(Qd, Kd, perm, w.blk, w.seg, w.mode, dt, w.band, w.n_sink, cap=cap, counts=counts,
-                           idx=idx, ws=ws_s)
-            pbs.pbs_attn_fwd(Qd, Kd, Vd, perm, counts, idx, w.blk, w.seg, out=O, lse=lse)
+            if not gate:
+                pbs.pbs_permute(Qd, Kd, w.blk, w.seg, w.n_sink, perm=perm, ws=ws_p)
+                pbs.pbs_select(Qd, Kd, perm, w.blk, w.seg, w.mode, dt, w.band, w.n_sink, cap=cap,
+                               counts=counts, idx=idx, ws=ws_s)
+            pbs.pbs_attn_fwd(Qd, Kd, Vd, perm, counts, idx, w.blk, w.seg, out=O, lse=lse, gate_thr=thr)
             Oh.copy_(O, non_blocking=True)
 
         e2e_step()
@@ -363,7 +396,7 @@ def run_pbs(args):
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d, "blk": w.blk,
-                   "seg": w.seg, "selection": f"{w.mode} density={w.density} n_sink={w.n_sink}",
+                   "seg": w.seg, "selection": selection_label(w),
                    "per_gpu": "one full workload per GPU",
                    "l2": "inputs larger than L2 (Q alone is %.2f GB)" % (Q.numel() * 2 / 1e9)},
         "breakdown": {"permute_ms": ms_perm, "select_ms": ms_sel, "attn_ms": ms_attn,
