@@ -141,6 +141,31 @@ def test_gated_attention_workload_sampled():
         assert_close(torch.from_numpy(O_np[b, h, sl]), o_ref, what=str((b, h, i)))
 
 
+def test_gated_attention_64k_stored_thresholds():
+    """The 64K gating workload as the bench runs it: every earlier block
+    listed, the offline thresholds stored beside the tests, identity order.
+    Sampled query blocks (all with more than 64 causal tiles but block 0)
+    against the oracle; the kernel must gate most tiles."""
+    import os
+    w, Q, K, V = workload_inputs("gate_b1_64k")
+    thr = np.load(os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "gate_thr_gate_b1_64k.npy"))
+    perm = np.broadcast_to(np.arange(w.N, dtype=np.int32), (w.B, w.Hkv, w.N)).copy()
+    counts, lists = oracle.dense_lists(w.B, w.Hq, w.nb, w.blk, w.seg)
+    O, L, st = _run(w, Q, K, V, perm, counts, lists, gate=thr.astype(np.float64), stats=True)
+    n_causal = w.B * w.Hq * w.nb * (w.nb + 1) // 2
+    assert int(st[0]) == n_causal
+    # at most keep + ties + the own tile are kept per block with a finite threshold
+    assert int(st[1]) > n_causal // 2
+    blocks = [(0, 0, 0), (0, 0, 64), (0, 5, 65), (0, 17, 300), (0, 31, w.nb - 1), (0, 12, 449)]
+    ref = oracle.attn_blocks(Q, K, V, perm, lists, w.blk, w.seg, blocks, gate_thr=thr.astype(np.float64))
+    O_np = O.float().cpu().numpy().astype(np.float64)
+    L_np = L.cpu().numpy()
+    for (b, h, i), (o_ref, l_ref) in ref.items():
+        sl = slice(i * w.blk, (i + 1) * w.blk)
+        assert_close(torch.from_numpy(O_np[b, h, sl]), o_ref, what=str((b, h, i)))
+        assert np.max(np.abs(L_np[b, h, sl] - l_ref)) <= LSE_MAX_ABS
+
+
 def test_unvisited_tiles_are_never_read():
     """NaN in every K/V row outside one query block's key set must not reach
     that block's output (bit-identical to the clean run): rows of unlisted
