@@ -182,7 +182,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
       }
       for (int h = 0; h < 2; ++h) {
         mbar_init(&sh.bar_s[h], 1);
-        mbar_init(&sh.bar_p[h], 128);
+        mbar_init(&sh.bar_p[h], 4);             // one arrival per softmax warp
         mbar_init(&sh.bar_o[h], 1);
       }
       mbar_init(&sh.bar_fin, 1);
@@ -208,6 +208,25 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
     const __nv_bfloat16* vb = static_cast<const __nv_bfloat16*>(p.V.ptr) + b * p.V.sB + hk * p.V.sH;
     const int32_t* prow = p.perm + (static_cast<int64_t>(b) * p.K.H + hk) * N;
     constexpr int CH = D / 8;
+    // Tile gathers: thread pt always copies 16-byte chunk c of rows r0,
+    // r0 + RPP, r0 + 2 RPP, ... (RPP rows per pass of the 96 threads).  A
+    // tile's row indices are read from shared memory all at once before its
+    // copies are issued, so the copies go out back to back instead of each
+    // waiting on its own index load.
+    constexpr int RPP = kProducerThreads / CH, NIT = (BLK + RPP - 1) / RPP;
+    static_assert(kProducerThreads % CH == 0, "producer threads cover whole rows");
+    const int cc = pt % CH, r0 = pt / CH;
+    const uint32_t cc_off = static_cast<uint32_t>((cc / 8) * (BLK * 128));
+    auto gather_tile = [&](uint32_t dst, const __nv_bfloat16* base, int64_t sN, const int32_t* rows) {
+      int32_t x[NIT];
+#pragma unroll
+      for (int k = 0; k < NIT; ++k) x[k] = r0 + RPP * k < BLK ? rows[r0 + RPP * k] : 0;
+#pragma unroll
+      for (int k = 0; k < NIT; ++k) {
+        const int r = r0 + RPP * k;
+        if (r < BLK) cp_async16(dst + cc_off + sw128_offset(r, cc % 8), base + x[k] * sN + cc * 8);
+      }
+    };
     // Q tiles of both heads (rows >= BLK zero-filled when BLK < 128)
     for (int h = 0; h < (has1 ? 2 : 1); ++h) {
       const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(p.Q.ptr) + b * p.Q.sB + (h0 + h) * p.Q.sH;
@@ -264,11 +283,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
           rowbuf[st][r] = static_cast<int32_t>(x);
         }
         named_sync(1, kProducerThreads);
-        const uint32_t dk = sK + st * C::kKVBytes;
-        for (int id = pt; id < BLK * CH; id += kProducerThreads) {
-          const int r = id / CH, c = id % CH;
-          cp_async16(dk + (c / 8) * (BLK * 128) + sw128_offset(r, c % 8), kb + rowbuf[st][r] * p.K.sN + c * 8);
-        }
+        gather_tile(sK + st * C::kKVBytes, kb, p.K.sN, rowbuf[st]);
         cp_async_mbar_arrive(&sh.bar_k[st]);      // arrives when this thread's copies land
       }
       const int tv = gate ? t - 1 : t;            // tile whose V goes now
@@ -287,13 +302,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
           }
         }
         if (named_sync_or(1, kProducerThreads, !okv)) break;
-        if (keep) {
-          const uint32_t dv = sV + sv * C::kKVBytes;
-          for (int id = pt; id < BLK * CH; id += kProducerThreads) {
-            const int r = id / CH, c = id % CH;
-            cp_async16(dv + (c / 8) * (BLK * 128) + sw128_offset(r, c % 8), vb + rowbuf[sv][r] * p.V.sN + c * 8);
-          }
-        }
+        if (keep) gather_tile(sV + sv * C::kKVBytes, vb, p.V.sN, rowbuf[sv]);
         cp_async_mbar_arrive(&sh.bar_v[sv]);
       }
       if (t + 1 < T) fetch_rows(t + 1);
@@ -322,6 +331,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
       constexpr uint32_t idesc_qk = idesc_bf16(kM, BLK, false);
       constexpr uint32_t idesc_pv = idesc_bf16(kM, D, true);
       const int nh = has1 ? 2 : 1;
+      // All loop state lives in registers: per-head arrays are indexed only
+      // by the unrolled head loop's constant, per-stage values are separate
+      // scalars chosen by the stage bit.
       // Per head: next tile needing QK^T, tile whose PV is pending, QK count.
       int nq[2] = {T, T}, pend[2] = {-1, -1}, kh[2] = {0, 0};
       bool o_init[2] = {false, false};
@@ -330,22 +342,39 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
         while (t < T && !((tile_mask(t) >> h) & 1u)) ++t;
         return t;
       };
-      for (int h = 0; h < nh; ++h) nq[h] = next_tile(h, 0);
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+        if (h < nh) nq[h] = next_tile(h, 0);
       // Per ring stage: the tile it holds and how many heads still need it,
       // and how many of its fill phases have been observed.  A stage holds
       // tiles st, st+2, st+4, ... in turn; a tile's phase is tested only when
       // it is the next one due on its stage, since a parity test cannot tell
       // a phase two fills ahead from the current one.
-      int ktile[kStages] = {-1, -1}, kleft[kStages] = {0, 0}, kseen[kStages] = {0, 0};
-      int vtile[kStages] = {-1, -1}, vleft[kStages] = {0, 0}, vseen[kStages] = {0, 0};
-      auto landed = [&](uint64_t* bars, int* seen, int t) -> bool {
-        const int st = t & 1, due = st + 2 * seen[st];
+      int kt0 = -1, kt1 = -1, kl0 = 0, kl1 = 0, ks0 = 0, ks1 = 0;
+      int vt0 = -1, vt1 = -1, vl0 = 0, vl1 = 0, vs0 = 0, vs1 = 0;
+      auto landed = [&](uint64_t* bars, int& seen0, int& seen1, int t) -> bool {
+        const int st = t & 1;
+        const int seen = st ? seen1 : seen0;
+        const int due = st + 2 * seen;
         if (t < due) return true;                        // observed earlier, still held
         if (t > due) return false;                       // an earlier fill is not observed yet
-        if (!test(&bars[st], seen[st] & 1)) return false;
-        ++seen[st];
+        if (!test(&bars[st], seen & 1)) return false;
+        if (st) seen1 = seen + 1; else seen0 = seen + 1;
         if (leader) fence_proxy_async();                 // fill's cp.async writes -> tensor-core reads
         return true;
+      };
+      // One more head done with tile t on its stage; true when it was the
+      // last head that needed it (the stage may then be refilled).
+      auto release = [&](int& tile0, int& tile1, int& left0, int& left1, int t) -> bool {
+        const int st = t & 1;
+        int left = st ? left1 : left0;
+        if ((st ? tile1 : tile0) != t) {
+          if (st) tile1 = t; else tile0 = t;
+          left = __popc(tile_mask(t));
+        }
+        --left;
+        if (st) left1 = left; else left0 = left;
+        return left == 0;
       };
       uint32_t idle = 0;
       // Event-driven issue: whichever of PV_h (P ready, V landed) or QK_h
@@ -354,11 +383,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
       // S's columns) has been consumed before S is overwritten.
       while (ok) {
         bool pending = false, progress = false;
-        for (int h = 0; h < nh; ++h) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          if (h >= nh) break;
           if (pend[h] >= 0) {
             pending = true;
             const int t = pend[h], st = t & 1;
-            if (test(&sh.bar_p[h], (kh[h] - 1) & 1) && landed(sh.bar_v, vseen, t)) {
+            if (test(&sh.bar_p[h], (kh[h] - 1) & 1) && landed(sh.bar_v, vs0, vs1, t)) {
               tc_fence_after();
               int skip = 0;
               if (leader) skip = sh.skip[h][(kh[h] - 1) & 1];      // lane 0 acquired bar_p
@@ -375,11 +406,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
                 }
                 o_init[h] = true;
               }
-              if (vtile[st] != t) {
-                vtile[st] = t;
-                vleft[st] = __popc(tile_mask(t));
-              }
-              if (--vleft[st] == 0 && elect_one()) tc_commit(&sh.bar_vempty[st]);
+              if (release(vt0, vt1, vl0, vl1, t) && elect_one()) tc_commit(&sh.bar_vempty[st]);
               pend[h] = -1;
               progress = true;
             }
@@ -387,7 +414,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
           if (pend[h] < 0 && nq[h] < T) {
             pending = true;
             const int t = nq[h], st = t & 1;
-            if (landed(sh.bar_k, kseen, t)) {
+            if (landed(sh.bar_k, ks0, ks1, t)) {
               tc_fence_after();
               const uint32_t qbase = sQ0 + h * C::kQBytes;
               const uint32_t kbase = sK + st * C::kKVBytes;
@@ -403,11 +430,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
               }
               if (elect_one()) tc_commit(&sh.bar_s[h]);
               ++kh[h];
-              if (ktile[st] != t) {
-                ktile[st] = t;
-                kleft[st] = __popc(tile_mask(t));
-              }
-              if (--kleft[st] == 0 && elect_one()) tc_commit(&sh.bar_kempty[st]);
+              if (release(kt0, kt1, kl0, kl1, t) && elect_one()) tc_commit(&sh.bar_kempty[st]);
               pend[h] = t;
               nq[h] = next_tile(h, t + 1);
               progress = true;
@@ -428,8 +451,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
         }
       }
       if (leader) {
-        for (int h = 0; h < nh; ++h)
-          if (kh[h] > 0) tc_commit(&sh.bar_o[h]);
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+          if (h < nh && kh[h] > 0) tc_commit(&sh.bar_o[h]);
         tc_commit(&sh.bar_fin);
         // drain: every MMA of this CTA has completed before tensor memory is freed
         mbar_wait(&sh.bar_fin, 0, p.err);
@@ -480,13 +504,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
             cmax = fmaxf(cmax, v);
           }
         } else {
-          // Eight independent partial maxima (a single chain is latency bound).
+          // Eight independent 3-input max chains (a single chain is latency bound).
           float mm[8];
 #pragma unroll
-          for (int q = 0; q < 8; ++q) mm[q] = __uint_as_float(x[q]);
-#pragma unroll
-          for (int e = 8; e < 64; ++e) mm[e & 7] = fmaxf(mm[e & 7], __uint_as_float(x[e]));
-          cmax = fmaxf(fmaxf(fmaxf(mm[0], mm[1]), fmaxf(mm[2], mm[3])), fmaxf(fmaxf(mm[4], mm[5]), fmaxf(mm[6], mm[7])));
+          for (int q = 0; q < 8; ++q) {
+            mm[q] = fmax3(__uint_as_float(x[q]), __uint_as_float(x[8 + q]), __uint_as_float(x[16 + q]));
+            mm[q] = fmax3(mm[q], __uint_as_float(x[24 + q]), __uint_as_float(x[32 + q]));
+            mm[q] = fmax3(mm[q], __uint_as_float(x[40 + q]), __uint_as_float(x[48 + q]));
+            mm[q] = fmaxf(mm[q], __uint_as_float(x[56 + q]));
+          }
+          cmax = fmax3(fmax3(mm[0], mm[1], mm[2]), fmax3(mm[3], mm[4], mm[5]), fmaxf(mm[6], mm[7]));
         }
         rmax = fmaxf(rmax, cmax);
         const float cm = cmax * p.scale_log2;
@@ -520,17 +547,27 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
             u[e] = pack_bf16x2(a0, a1);
           }
         } else {
-          // Eight independent partial sums: one running sum would make the
-          // row's 64 additions a serial chain of FADD latencies.
-          float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+          // Pairs of columns in packed fp32x2 arithmetic (scale-and-shift and
+          // the row sums), four independent packed partial sums.
+          unsigned long long ps2[4] = {0ull, 0ull, 0ull, 0ull};   // +0.0f is all zero bits
+          const unsigned long long sc2 = f2_pack(p.scale_log2, p.scale_log2);
+          const unsigned long long nm2 = f2_pack(-m_use, -m_use);
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
-            const float a0 = ex2(fmaf(__uint_as_float(x[2 * e]), p.scale_log2, -m_use));
-            const float a1 = ex2(fmaf(__uint_as_float(x[2 * e + 1]), p.scale_log2, -m_use));
-            ps[e & 7] += a0 + a1;
-            u[e] = pack_bf16x2(a0, a1);
+            const unsigned long long y =
+                f2_fma(f2_pack(__uint_as_float(x[2 * e]), __uint_as_float(x[2 * e + 1])), sc2, nm2);
+            float y0, y1;
+            f2_unpack(y, y0, y1);
+            const float a0 = ex2(y0), a1 = ex2(y1);
+            ps2[e & 3] = f2_add(ps2[e & 3], f2_pack(a0, a1));
+            u[e] = cvt_bf16x2(a0, a1);
           }
-          psum += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+          float s0, s1, s2, s3, s4, s5, s6, s7;
+          f2_unpack(ps2[0], s0, s1);
+          f2_unpack(ps2[1], s2, s3);
+          f2_unpack(ps2[2], s4, s5);
+          f2_unpack(ps2[3], s6, s7);
+          psum += ((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7));
         }
         tmem_st32(tS + c * 32, u);
       }
@@ -549,7 +586,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
           tmem_st_wait();
           if (r == 0) sh.skip[h][k & 1] = 1;
           tc_fence_before();
-          mbar_arrive(&sh.bar_p[h]);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sh.bar_p[h]);     // one arrival per warp
           ++k;
           continue;
         }
@@ -577,7 +615,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
       tmem_st_wait();
       if (r == 0) sh.skip[h][k & 1] = 0;
       tc_fence_before();
-      mbar_arrive(&sh.bar_p[h]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh.bar_p[h]);         // one arrival per warp
       o_init = true;
       ++k;
     }
