@@ -199,15 +199,21 @@ def forced_blocks(i: int, inv_row: np.ndarray, blk: int, seg: int,
 def select(Q: np.ndarray, K: np.ndarray, perm: np.ndarray, blk: int, seg: int,
            mode: str, density: float = 1.0, tau: float = 1.0, band: int = 0,
            n_sink: int = 0, rows: Optional[Iterable[Tuple[int, int, int]]] = None,
-           trace: Optional[dict] = None):
-    """Per (b, hq, i) ascending lists of permuted key blocks to attend.
+           trace: Optional[dict] = None, list_order: str = "ascending"):
+    """Per (b, hq, i) lists of permuted key blocks to attend.
 
     Returns (counts [B,Hq,nb] int32, lists dict {(b,hq,i): int32 array}).
     With ``rows`` given, only those (b, hq, i) are computed (others count 0).
     mode "topk": budget from ``density``; mode "tau": cumulative mass.
     With ``trace`` (a dict), tau mode records per row the accumulated mass
     before the last added block and after it, so callers can check how far
-    each stopping decision is from tau."""
+    each stopping decision is from tau.
+    list_order "ascending": lists sorted by block id; "score": the forced
+    blocks first (ascending), then the other chosen blocks by descending
+    block score, ties to the lower block id -- the visiting order of S2O's
+    Pass 2, which processes candidates in descending estimated importance
+    ("S2O: Early Stopping for Sparse Attention via Online Permutation",
+    Technical Summary, 2. Early-Stopping Rule)."""
     B, Hq, N, d = Q.shape
     Hkv = K.shape[1]
     G = Hq // Hkv
@@ -272,7 +278,15 @@ def select(Q: np.ndarray, K: np.ndarray, perm: np.ndarray, blk: int, seg: int,
                     trace[(b, h, i)] = (before, cum)
         else:
             raise ValueError(mode)
-        arr = np.array(sorted(chosen), np.int32)
+        if list_order == "ascending":
+            arr = np.array(sorted(chosen), np.int32)
+        elif list_order == "score":
+            fset = set(int(x) for x in F)
+            lead = sorted(x for x in chosen if x in fset)
+            tail = sorted((x for x in chosen if x not in fset), key=lambda x: (-S[x], x))
+            arr = np.array(lead + tail, np.int32)
+        else:
+            raise ValueError(list_order)
         lists[(b, h, i)] = arr
         counts[b, h, i] = arr.size
     return counts, lists
@@ -371,6 +385,74 @@ def attn_blocks(Q, K, V, perm, lists: dict, blk: int, seg: int, blocks: Iterable
         listed = lists.get((b, h, i), np.zeros(0, np.int32))
         thr = None if gate_thr is None else float(gate_thr[b, h, i])
         out[(b, h, i)] = attn_block(Q, K, V, perm, listed, b, h, i, blk, seg, scale, thr)
+    return out
+
+
+def attn_early_stop_block(Q, K, V, perm, listed, b, hq, i, blk, seg, scale, stop_tau: float,
+                          trace: Optional[list] = None):
+    """S2O's two passes with the early-stopping rule, fp64, for the ``blk``
+    query rows of block i of (b, hq).  Returns (O, LSE, tiles of Pass 2 run).
+
+    "S2O: Early Stopping for Sparse Attention via Online Permutation",
+    Technical Summary, 3. Kernel Implementation and 2. Early-Stopping Rule:
+    Pass 1 runs dense causal attention over the block's own segment (natural
+    order) and leaves the online-softmax state (m, l, acc) per query row;
+    Pass 2 continues from that state over the listed permuted blocks in the
+    order given.  After each Pass-2 tile the marginal gain of every row is
+    dl / l, the tile's exponential mass over the accumulated mass (both in
+    the running-max frame, so the ratio does not depend on the frame); when
+    the largest gain over the block's rows is below ``stop_tau`` the
+    remaining listed blocks are skipped (the tile just run stays in).
+    ``trace``, if given, receives the largest gain of every tile run."""
+    Hq, Hkv = Q.shape[1], K.shape[1]
+    hk = hq // (Hq // Hkv)
+    q_pos = np.arange(i * blk, (i + 1) * blk)
+    q = Q[b, hq, i * blk:(i + 1) * blk].astype(F64)
+    # Pass 1: natural keys of the own segment up to the block's end, causal
+    s0 = segment_of_block(i, blk, seg) * seg
+    own = np.arange(s0, (i + 1) * blk, dtype=np.int64)
+    lg = (q @ K[b, hk, own].astype(F64).T) * scale
+    lg = np.where(own[None, :] <= q_pos[:, None], lg, -np.inf)
+    m = lg.max(axis=1)
+    e = np.exp(lg - m[:, None])
+    l = e.sum(axis=1)
+    acc = e @ V[b, hk, own].astype(F64)
+    # Pass 2: listed permuted blocks in the given order (all keys visible)
+    n_run = 0
+    for pb in listed:
+        pos = perm[b, hk, int(pb) * blk:(int(pb) + 1) * blk].astype(np.int64)
+        lg = (q @ K[b, hk, pos].astype(F64).T) * scale
+        m_new = np.maximum(m, lg.max(axis=1))
+        alpha = np.exp(m - m_new)
+        e = np.exp(lg - m_new[:, None])
+        dl = e.sum(axis=1)
+        l = l * alpha + dl
+        acc = acc * alpha[:, None] + e @ V[b, hk, pos].astype(F64)
+        m = m_new
+        n_run += 1
+        gain = float((dl / l).max())
+        if trace is not None:
+            trace.append(gain)
+        if gain < stop_tau:
+            break
+    return acc / l[:, None], m + np.log(l), n_run
+
+
+def attn_early_stop(Q, K, V, perm, lists: dict, blk: int, seg: int, stop_tau: float,
+                    blocks: Iterable[Tuple[int, int, int]], scale: Optional[float] = None,
+                    traces: Optional[dict] = None) -> dict:
+    """{(b, hq, i): (O [blk, d], LSE [blk], Pass-2 tiles run)} for the given
+    blocks; ``lists`` must hold each block's list in visiting order."""
+    d = Q.shape[3]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    out = {}
+    for (b, h, i) in blocks:
+        listed = lists.get((b, h, i), np.zeros(0, np.int32))
+        tr = [] if traces is not None else None
+        out[(b, h, i)] = attn_early_stop_block(Q, K, V, perm, listed, b, h, i, blk, seg, scale, stop_tau, tr)
+        if traces is not None:
+            traces[(b, h, i)] = tr
     return out
 
 

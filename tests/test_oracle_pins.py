@@ -422,3 +422,106 @@ def test_stripe_keys_cluster_in_leading_blocks():
     assert np.mean(rel < w.blk) >= 0.95
     # without the permutation the stripes sit wherever they were drawn
     assert np.mean(info["stripes"][0, 0] % w.seg < w.blk) < 0.5
+
+
+# ---------------------------------------------------------------------------
+# S2O visiting order and early stopping ("S2O: Early Stopping for Sparse
+# Attention via Online Permutation", Technical Summary 2 and 3)
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("mode,kw", [("topk", dict(density=0.4, n_sink=8)), ("tau", dict(tau=0.9)),
+                                     ("topk", dict(density=1.0))])
+def test_score_order_lists(mode, kw):
+    """Score order holds the same set as the ascending list; sink-forced
+    blocks lead in ascending order; the rest is non-increasing in the block
+    score (recomputed here as a sum of explicit logits), ties ascending."""
+    B, Hq, Hkv, N, d, blk, seg = 1, 4, 2, 128, 16, 8, 32
+    Q, K, V = _small(B, Hq, Hkv, N, d, seed=31)
+    n_sink = kw.get("n_sink", 0)
+    perm = oracle.permute(Q, K, blk, seg, n_sink)
+    c_a, l_a = oracle.select(Q, K, perm, blk, seg, mode, **kw)
+    c_s, l_s = oracle.select(Q, K, perm, blk, seg, mode, list_order="score", **kw)
+    assert np.array_equal(c_a, c_s)
+    G = Hq // Hkv
+    spb = seg // blk
+    checked = 0
+    for (b, h, i), arr in l_s.items():
+        assert sorted(arr.tolist()) == l_a[(b, h, i)].tolist()
+        if arr.size < 2:
+            continue
+        inv = oracle.inverse_permutation(perm[0, h // G])
+        s = i // spb
+        forced = {int(inv[pos]) // blk for pos in range(min(n_sink, s * seg))}
+        nf = sum(1 for x in arr.tolist() if x in forced)
+        assert set(arr[:nf].tolist()) == forced
+        assert arr[:nf].tolist() == sorted(arr[:nf].tolist())
+        S = [_tile_logit_sum(Q, K, perm, 0, h, i, int(pb), blk, G) for pb in arr[nf:]]
+        for (s1, a1), (s2, a2) in zip(zip(S, arr[nf:]), zip(S[1:], arr[nf + 1:])):
+            assert s1 > s2 or (s1 == s2 and a1 < a2), (h, i)
+        checked += 1
+    assert checked > 10
+
+
+def _es_case(seed=41):
+    B, Hq, Hkv, N, d, blk, seg = 1, 2, 1, 512, 16, 16, 128
+    Q, K, V = _small(B, Hq, Hkv, N, d, seed=seed, scale=2.0)
+    perm = oracle.permute(Q, K, blk, seg)
+    _, lists = oracle.select(Q, K, perm, blk, seg, "topk", density=1.0, list_order="score")
+    return blk, seg, d, Q, K, V, perm, lists
+
+
+def _explicit_gains(Q, K, perm, h, i, listed, blk, seg, scale):
+    """Per Pass-2 tile k: max over the block's rows of (exp mass of tile k) /
+    (exp mass of the own segment's visible keys and tiles 1..k), from
+    explicit exponentials of the logits (no running state)."""
+    rows = np.arange(i * blk, (i + 1) * blk)
+    q = Q[0, h, rows].astype(np.float64)
+    s0 = (i // (seg // blk)) * seg
+    own = np.arange(s0, (i + 1) * blk)
+    lo = (q @ K[0, 0, own].astype(np.float64).T) * scale
+    total = np.where(own[None, :] <= rows[:, None], np.exp(lo), 0.0).sum(axis=1)
+    gains = []
+    for pb in listed:
+        pos = perm[0, 0, int(pb) * blk:(int(pb) + 1) * blk]
+        et = np.exp((q @ K[0, 0, pos].astype(np.float64).T) * scale).sum(axis=1)
+        total = total + et
+        gains.append(float((et / total).max()))
+    return gains
+
+
+def test_early_stop_brute_force():
+    """The early-stopped result equals plain masked attention over the own
+    segment and the first k* listed blocks, where k* is the first tile whose
+    explicit mass ratio is below tau (all of them if none is)."""
+    blk, seg, d, Q, K, V, perm, lists = _es_case()
+    scale = 1.0 / math.sqrt(d)
+    n_mid = 0
+    for (b, h, i), listed in lists.items():
+        if listed.size < 3:
+            continue
+        gains = _explicit_gains(Q, K, perm, h, i, listed, blk, seg, scale)
+        for tau in (float(np.median(gains)), float(np.min(gains)) * 1.0001, float(np.max(gains)) * 0.999):
+            k_star = next((k + 1 for k, g in enumerate(gains) if g < tau), len(gains))
+            O, L, n = oracle.attn_early_stop_block(Q, K, V, perm, listed, b, h, i, blk, seg, scale, tau)
+            O_ref, L_ref = oracle.attn_block(Q, K, V, perm, listed[:k_star], b, h, i, blk, seg, scale)
+            assert n == k_star, (h, i, tau)
+            np.testing.assert_allclose(O, O_ref, rtol=0, atol=1e-12)
+            np.testing.assert_allclose(L, L_ref, rtol=0, atol=1e-12)
+            n_mid += 0 < k_star < len(gains)
+    assert n_mid > 5
+
+
+def test_early_stop_limits():
+    """tau = 0 never stops (plain sparse attention over every listed block);
+    tau > 1 stops right after the first listed block (a gain is at most 1)."""
+    blk, seg, d, Q, K, V, perm, lists = _es_case(seed=43)
+    scale = 1.0 / math.sqrt(d)
+    for (b, h, i), listed in lists.items():
+        O, L, n = oracle.attn_early_stop_block(Q, K, V, perm, listed, b, h, i, blk, seg, scale, 0.0)
+        O_ref, L_ref = oracle.attn_block(Q, K, V, perm, listed, b, h, i, blk, seg, scale)
+        assert n == len(listed)
+        np.testing.assert_allclose(O, O_ref, rtol=0, atol=1e-12)
+        O, L, n = oracle.attn_early_stop_block(Q, K, V, perm, listed, b, h, i, blk, seg, scale, 1.5)
+        O_ref, L_ref = oracle.attn_block(Q, K, V, perm, listed[:1], b, h, i, blk, seg, scale)
+        assert n == min(1, len(listed))
+        np.testing.assert_allclose(O, O_ref, rtol=0, atol=1e-12)
