@@ -64,6 +64,8 @@ def dense_causal_flops(w) -> float:
 def selection_label(w) -> str:
     if w.mode == "gate":
         return f"all earlier blocks, block-max gate calibrated to keep {w.gate_keep} tiles"
+    if w.stop_tau > 0:
+        return f"topk density={w.density} in descending block score, early stop at gain < {w.stop_tau}"
     sel = f"topk density={w.density}" if w.mode == "topk" else f"tau={w.tau}"
     return sel + (f" band={w.band}" if w.band else "") + (f" n_sink={w.n_sink}" if w.n_sink else "")
 
@@ -158,14 +160,18 @@ def oracle_baseline(w, Q, K, V, budget_s: float = 20.0, n_blocks: int = 48):
         perm[:, 0] = perm1[:, 0]
         t0 = time.perf_counter()
         counts, lists = oracle.select(Q, K, perm, w.blk, w.seg, w.mode, density=w.density, tau=w.tau,
-                                      band=w.band, n_sink=w.n_sink, rows=blocks)
+                                      band=w.band, n_sink=w.n_sink, rows=blocks,
+                                      list_order="score" if w.stop_tau > 0 else "ascending")
         t_sel = (time.perf_counter() - t0) * (w.B * w.Hq * w.nb) / len(blocks)
     t0 = time.perf_counter()
     done = []
     tiles_sample = 0
     spb = w.seg // w.blk
     for key in blocks:
-        oracle.attn_blocks(Q, K, V, perm, lists, w.blk, w.seg, [key], gate_thr=thr)
+        if w.stop_tau > 0:
+            oracle.attn_early_stop(Q, K, V, perm, lists, w.blk, w.seg, w.stop_tau, [key])
+        else:
+            oracle.attn_blocks(Q, K, V, perm, lists, w.blk, w.seg, [key], gate_thr=thr)
         i = key[2]
         tiles_sample += len(lists.get(key, ())) + (i - (i // spb) * spb + 1)
         done.append(key)
@@ -234,6 +240,7 @@ def run_pbs(args):
     # earlier block is listed and the thresholds (calibrated offline by the
     # oracle, stored beside the tests) decide per tile.
     gate = w.mode == "gate"
+    early = w.stop_tau > 0          # S2O early stopping: lists in visiting order
     thr = None
     if gate:
         thr_path = os.path.join(ROOT, "tests", "golden", f"gate_thr_{w.name}.npy")
@@ -256,10 +263,14 @@ def run_pbs(args):
             e[1].record(s)
         if not gate:
             pbs.pbs_select(Q, K, perm, w.blk, w.seg, w.mode, dt, w.band, w.n_sink, cap=cap, counts=counts,
-                           idx=idx, ws=ws_s)
+                           idx=idx, ws=ws_s, score_order=early)
         if record:
             e[2].record(s)
-        pbs.pbs_attn_fwd(Q, K, V, perm, counts, idx, w.blk, w.seg, out=O, lse=lse, stats=st, gate_thr=thr)
+        if early:
+            pbs.pbs_attn_fwd_early_stop(Q, K, V, perm, counts, idx, w.blk, w.seg, w.stop_tau, out=O, lse=lse,
+                                        stats=st)
+        else:
+            pbs.pbs_attn_fwd(Q, K, V, perm, counts, idx, w.blk, w.seg, out=O, lse=lse, stats=st, gate_thr=thr)
         if record:
             e[3].record(s)
             for k, x in zip(("p0", "p1", "s1", "a1"), e):
@@ -269,7 +280,9 @@ def run_pbs(args):
     step(st=stats)
     pbs.pbs_check_device()
     n_qk, n_gated = int(stats[0]), int(stats[1])
-    executed_flops = (n_qk - n_gated) * tile_flops(w) + n_gated * tile_flops(w) / 2
+    # gated tiles ran QK^T only; tiles left out by early stopping ran nothing
+    n_half = 0 if early else n_gated
+    executed_flops = (n_qk - n_half) * tile_flops(w) + n_half * tile_flops(w) / 2
     causal_tiles = w.B * w.Hq * w.nb * (w.nb + 1) // 2
 
     for _ in range(max(args.warmup, 0)):
@@ -343,8 +356,12 @@ def run_pbs(args):
             if not gate:
                 pbs.pbs_permute(Qd, Kd, w.blk, w.seg, w.n_sink, perm=perm, ws=ws_p)
                 pbs.pbs_select(Qd, Kd, perm, w.blk, w.seg, w.mode, dt, w.band, w.n_sink, cap=cap,
-                               counts=counts, idx=idx, ws=ws_s)
-            pbs.pbs_attn_fwd(Qd, Kd, Vd, perm, counts, idx, w.blk, w.seg, out=O, lse=lse, gate_thr=thr)
+                               counts=counts, idx=idx, ws=ws_s, score_order=early)
+            if early:
+                pbs.pbs_attn_fwd_early_stop(Qd, Kd, Vd, perm, counts, idx, w.blk, w.seg, w.stop_tau, out=O,
+                                            lse=lse)
+            else:
+                pbs.pbs_attn_fwd(Qd, Kd, Vd, perm, counts, idx, w.blk, w.seg, out=O, lse=lse, gate_thr=thr)
             Oh.copy_(O, non_blocking=True)
 
         e2e_step()
@@ -400,7 +417,8 @@ def run_pbs(args):
                    "per_gpu": "one full workload per GPU",
                    "l2": "inputs larger than L2 (Q alone is %.2f GB)" % (Q.numel() * 2 / 1e9)},
         "breakdown": {"permute_ms": ms_perm, "select_ms": ms_sel, "attn_ms": ms_attn,
-                      "executed_tiles": n_qk, "gated_tiles": n_gated, "causal_tiles": causal_tiles,
+                      "executed_tiles": n_qk, ("skipped_tiles" if early else "gated_tiles"): n_gated,
+                      "causal_tiles": causal_tiles,
                       "density": n_qk / causal_tiles, "executed_tflops": achieved,
                       "effective_tflops": value / world},
         "dense_same_kernel": dense,

@@ -20,6 +20,11 @@
  *                 Permutation", Technical Summary, 1. Online Permutation via
  *                 Index-Driven Loading and 3. Kernel Implementation;
  *                 "Block Sparse Flash Attention", Approach.
+ *   pbs_attn_fwd_early_stop
+ *                 the same two passes, the listed blocks visited in the order
+ *                 given, stopping once a tile's marginal attention mass falls
+ *                 below a fraction of the accumulated mass.  S2O page,
+ *                 2. Early-Stopping Rule.
  *
  * Conventions shared by every call
  * --------------------------------
@@ -77,6 +82,8 @@ typedef enum pbs_status {
 
 enum { PBS_OP_PERMUTE = 0, PBS_OP_SELECT = 1, PBS_OP_ATTN = 2 };
 enum { PBS_SELECT_TOPK = 0, PBS_SELECT_TAU = 1 };
+/* OR-ed into pbs_select's mode: write lists in visiting order (see there). */
+enum { PBS_SELECT_SCORE_ORDER = 0x10 };
 
 /* Bytes of workspace the given op needs for these shapes (0 if none).
  * Q and K may not be NULL; only their shapes are read.                     */
@@ -133,6 +140,12 @@ int pbs_select_capacity(int64_t N, int blk, int seg, int mode,
  *     mass (own segment included) is below tau.  tau >= 1 lists all.
  * counts: device int32 [B, Hq, N/blk]; idx: device int32
  * [B, Hq, N/blk, cap]; entries at and after counts[...] are unspecified.
+ * With mode | PBS_SELECT_SCORE_ORDER the same blocks are listed in visiting
+ * order instead of ascending: the forced blocks first (ascending), then the
+ * others by descending S, ties to the lower pb -- the descending estimated
+ * importance in which S2O's Pass 2 processes candidates ("S2O ...",
+ * Technical Summary, 2. Early-Stopping Rule); pbs_attn_fwd_early_stop
+ * consumes lists in this order.
  * Returns PBS_ERR_CAPACITY if cap < pbs_select_capacity(...).               */
 int pbs_select(const pbs_tensor* Q, const pbs_tensor* K, const int32_t* perm,
                int blk, int seg, int mode, double density_or_tau, int band,
@@ -158,6 +171,27 @@ int pbs_attn_fwd(const pbs_tensor* Q, const pbs_tensor* K, const pbs_tensor* V,
                  int cap, int blk, int seg, const float* gate_thr,
                  float softmax_scale, pbs_tensor* O, float* lse,
                  long long* stats, void* ws, size_t ws_bytes, void* stream);
+
+/* pbs_attn_fwd_early_stop: pbs_attn_fwd without gating, where Pass 2
+ * visits each block's listed permuted blocks in the order given (entries
+ * must be distinct; a repeated entry is dropped and sets the device error
+ * word) and stops early ("S2O ...", Technical Summary, 2. Early-Stopping
+ * Rule and 3. Kernel Implementation):
+ *   after each Pass-2 tile, every query row r of the block has a marginal
+ *   gain dl_r / l_r -- the tile's exponential mass over the row's mass
+ *   accumulated so far (own segment included), both in the running-max
+ *   frame; when the gains of all rows of the block are below stop_tau, the
+ *   remaining listed blocks are skipped (the tile just run stays in).
+ *   stop_tau = 0 never stops; stop_tau > 1 stops after the first listed
+ *   block.  Pass 1 (the own segment) always runs in full.
+ *   stop_tau: finite, >= 0.  Other arguments as for pbs_attn_fwd.
+ *   stats: NULL or device int64[2], incremented by (tiles whose QK^T was
+ *     computed, listed tiles the rule skipped); the caller zeroes it.
+ * The stop decisions are taken in fp32 on the kernel's running sums.       */
+int pbs_attn_fwd_early_stop(const pbs_tensor* Q, const pbs_tensor* K, const pbs_tensor* V,
+                            const int32_t* perm, const int32_t* counts, const int32_t* idx,
+                            int cap, int blk, int seg, float stop_tau, float softmax_scale,
+                            pbs_tensor* O, float* lse, long long* stats, void* stream);
 
 /* Synchronises `stream`, then returns and clears the sticky device error
  * word of the current device (PBS_OK if no device-side check failed).      */

@@ -20,10 +20,11 @@ LIB_PATH = os.path.join(_HERE, "libpbs.so")
 
 PBS_OP_PERMUTE, PBS_OP_SELECT, PBS_OP_ATTN = 0, 1, 2
 PBS_SELECT_TOPK, PBS_SELECT_TAU = 0, 1
+PBS_SELECT_SCORE_ORDER = 0x10
 STATUS = {0: "PBS_OK", -1: "PBS_ERR_INVALID_ARG", -2: "PBS_ERR_UNSUPPORTED", -3: "PBS_ERR_CAPACITY",
           -4: "PBS_ERR_CUDA", -5: "PBS_ERR_TIMEOUT", -6: "PBS_ERR_DEVICE_CHECK"}
 EXPORTS = ("pbs_workspace_size", "pbs_permute", "pbs_select_capacity", "pbs_select", "pbs_attn_fwd",
-           "pbs_check_device", "pbs_get_last_error", "pbs_version")
+           "pbs_attn_fwd_early_stop", "pbs_check_device", "pbs_get_last_error", "pbs_version")
 
 
 class PbsError(RuntimeError):
@@ -61,6 +62,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.pbs_select.restype = i32
     lib.pbs_attn_fwd.argtypes = [P, P, P, vp, vp, vp, i32, i32, i32, vp, ctypes.c_float, P, vp, vp, vp, sz, vp]
     lib.pbs_attn_fwd.restype = i32
+    lib.pbs_attn_fwd_early_stop.argtypes = [P, P, P, vp, vp, vp, i32, i32, i32, ctypes.c_float, ctypes.c_float,
+                                            P, vp, vp, vp]
+    lib.pbs_attn_fwd_early_stop.restype = i32
     lib.pbs_check_device.argtypes = [vp]
     lib.pbs_check_device.restype = i32
     lib.pbs_get_last_error.argtypes = []
@@ -148,13 +152,17 @@ def pbs_select(Q: torch.Tensor, K: torch.Tensor, perm: torch.Tensor, blk: int, s
                mode: str = "topk", density_or_tau: float = 1.0, band: int = 0, n_sink: int = 0,
                cap: Optional[int] = None, counts: Optional[torch.Tensor] = None,
                idx: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
-               stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
-    """(counts [B, Hq, nb] int32, idx [B, Hq, nb, cap] int32) block lists."""
+               stream=None, score_order: bool = False) -> Tuple[torch.Tensor, torch.Tensor]:
+    """(counts [B, Hq, nb] int32, idx [B, Hq, nb, cap] int32) block lists,
+    ascending, or in visiting order (forced blocks, then descending block
+    score) with ``score_order``."""
     lib = load()
     q, k = describe(Q), describe(K)
     B, Hq, N, _ = Q.shape
     nb = N // blk
     m = PBS_SELECT_TAU if mode == "tau" else PBS_SELECT_TOPK
+    if score_order:
+        m |= PBS_SELECT_SCORE_ORDER
     if cap is None:
         cap = max(1, select_capacity(N, blk, seg, mode, density_or_tau, band, n_sink))
     if counts is None:
@@ -193,6 +201,32 @@ def pbs_attn_fwd(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, perm: torch.
                             counts.data_ptr(), idx.data_ptr(), idx.shape[-1], blk, seg, _ptr(gate_thr),
                             float(softmax_scale), ctypes.byref(o), _ptr(lse), _ptr(stats), None, 0,
                             _stream(stream)))
+    return out, lse
+
+
+def pbs_attn_fwd_early_stop(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, perm: torch.Tensor,
+                            counts: torch.Tensor, idx: torch.Tensor, blk: int, seg: int, stop_tau: float,
+                            softmax_scale: Optional[float] = None, out: Optional[torch.Tensor] = None,
+                            lse: Optional[torch.Tensor] = None, want_lse: bool = True,
+                            stats: Optional[torch.Tensor] = None,
+                            stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """(O, LSE): S2O's two passes with the early-stopping rule; ``idx`` holds
+    each block's list in visiting order."""
+    lib = load()
+    B, Hq, N, D = Q.shape
+    if out is None:
+        out = torch.empty_like(Q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq, N), dtype=torch.float32, device=Q.device)
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(D)
+    if stats is not None and stats.dtype != torch.int64:
+        raise TypeError("stats must be int64")
+    q, k, v, o = describe(Q), describe(K), describe(V), describe(out)
+    _check(lib.pbs_attn_fwd_early_stop(ctypes.byref(q), ctypes.byref(k), ctypes.byref(v), perm.data_ptr(),
+                                       counts.data_ptr(), idx.data_ptr(), idx.shape[-1], blk, seg,
+                                       float(stop_tau), float(softmax_scale), ctypes.byref(o), _ptr(lse),
+                                       _ptr(stats), _stream(stream)))
     return out, lse
 
 

@@ -133,6 +133,53 @@ int api_validate_permute(const pbs_tensor* Qt, const pbs_tensor* Kt, int blk, in
 
 }  // namespace pbs
 
+namespace {
+int attn_common(const pbs_tensor* Qt, const pbs_tensor* Kt, const pbs_tensor* Vt,
+                const int32_t* perm, const int32_t* counts, const int32_t* idx, int cap, int blk,
+                int seg, const float* gate_thr, int early_stop, float stop_tau, float softmax_scale,
+                pbs_tensor* Ot, float* lse, long long* stats, void* stream) {
+  pbs::TensorDesc Q, K, V, O;
+  int rc;
+  if ((rc = check_tensor(Qt, "Q", &Q)) || (rc = check_tensor(Kt, "K", &K)) ||
+      (rc = check_tensor(Vt, "V", &V)) || (rc = check_tensor(Ot, "O", &O)))
+    return rc;
+  if ((rc = check_geometry(Q, K, blk, seg))) return rc;
+  if (V.B != K.B || V.H != K.H || V.N != K.N || V.D != K.D)
+    return fail(PBS_ERR_INVALID_ARG, "V shape differs from K");
+  if (O.B != Q.B || O.H != Q.H || O.N != Q.N || O.D != Q.D)
+    return fail(PBS_ERR_INVALID_ARG, "O shape differs from Q");
+  if (!perm || !counts || !idx) return fail(PBS_ERR_INVALID_ARG, "perm, counts or idx is null");
+  if (cap < 1) return fail(PBS_ERR_INVALID_ARG, "cap %d < 1", cap);
+  if (!(softmax_scale > 0.0f) || !std::isfinite(softmax_scale))
+    return fail(PBS_ERR_INVALID_ARG, "softmax_scale must be positive and finite");
+  int* err = device_error_word();
+  if (!err) return fail(PBS_ERR_CUDA, "cannot resolve the device error word");
+  pbs::AttnParams p;
+  p.Q = Q;
+  p.K = K;
+  p.V = V;
+  p.O = O;
+  p.perm = perm;
+  p.counts = counts;
+  p.idx = idx;
+  p.cap = cap;
+  p.blk = blk;
+  p.seg = seg;
+  p.nb = static_cast<int>(Q.N / blk);
+  p.G = static_cast<int>(Q.H / K.H);
+  p.gate_thr = gate_thr;
+  p.early_stop = early_stop;
+  p.stop_tau = stop_tau;
+  p.scale_log2 = softmax_scale * 1.4426950408889634f;
+  p.lse = lse;
+  p.stats = stats;
+  p.err = err;
+  cudaError_t e = pbs::launch_attn_fwd(p, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "attn_fwd launch");
+  return ok();
+}
+}  // namespace
+
 extern "C" {
 
 const char* pbs_version(void) { return "pbs 0.1 (sm_100a)"; }
@@ -179,6 +226,7 @@ int pbs_select_capacity(int64_t N, int blk, int seg, int mode, double density_or
                         int n_sink) {
   if (blk <= 0 || seg < blk || seg % blk || N <= 0 || N % blk)
     return fail(PBS_ERR_INVALID_ARG, "bad geometry for capacity");
+  mode &= ~PBS_SELECT_SCORE_ORDER;
   const int64_t nb = N / blk, spb = seg / blk;
   int64_t best = 0;
   const int64_t r = rho_permille(density_or_tau);
@@ -209,6 +257,8 @@ int pbs_select(const pbs_tensor* Qt, const pbs_tensor* Kt, const int32_t* perm, 
   if ((rc = check_tensor(Qt, "Q", &Q)) || (rc = check_tensor(Kt, "K", &K))) return rc;
   if ((rc = check_geometry(Q, K, blk, seg))) return rc;
   if (!perm || !counts || !idx) return fail(PBS_ERR_INVALID_ARG, "perm, counts or idx is null");
+  const int score_order = (mode & PBS_SELECT_SCORE_ORDER) ? 1 : 0;
+  mode &= ~PBS_SELECT_SCORE_ORDER;
   if (mode != PBS_SELECT_TOPK && mode != PBS_SELECT_TAU)
     return fail(PBS_ERR_INVALID_ARG, "mode %d unknown", mode);
   if (!(density_or_tau >= 0.0) || (mode == PBS_SELECT_TOPK && density_or_tau > 1.0))
@@ -243,6 +293,7 @@ int pbs_select(const pbs_tensor* Qt, const pbs_tensor* Kt, const int32_t* perm, 
   p.seg = seg;
   p.nb = static_cast<int>(nb);
   p.mode = mode;
+  p.score_order = score_order;
   p.band = band;
   p.n_sink = n_sink;
   p.cap = cap;
@@ -254,49 +305,25 @@ int pbs_select(const pbs_tensor* Qt, const pbs_tensor* Kt, const int32_t* perm, 
   return ok();
 }
 
+
 int pbs_attn_fwd(const pbs_tensor* Qt, const pbs_tensor* Kt, const pbs_tensor* Vt,
                  const int32_t* perm, const int32_t* counts, const int32_t* idx, int cap, int blk,
                  int seg, const float* gate_thr, float softmax_scale, pbs_tensor* Ot, float* lse,
                  long long* stats, void* ws, size_t ws_bytes, void* stream) {
   (void)ws;
   (void)ws_bytes;
-  pbs::TensorDesc Q, K, V, O;
-  int rc;
-  if ((rc = check_tensor(Qt, "Q", &Q)) || (rc = check_tensor(Kt, "K", &K)) ||
-      (rc = check_tensor(Vt, "V", &V)) || (rc = check_tensor(Ot, "O", &O)))
-    return rc;
-  if ((rc = check_geometry(Q, K, blk, seg))) return rc;
-  if (V.B != K.B || V.H != K.H || V.N != K.N || V.D != K.D)
-    return fail(PBS_ERR_INVALID_ARG, "V shape differs from K");
-  if (O.B != Q.B || O.H != Q.H || O.N != Q.N || O.D != Q.D)
-    return fail(PBS_ERR_INVALID_ARG, "O shape differs from Q");
-  if (!perm || !counts || !idx) return fail(PBS_ERR_INVALID_ARG, "perm, counts or idx is null");
-  if (cap < 1) return fail(PBS_ERR_INVALID_ARG, "cap %d < 1", cap);
-  if (!(softmax_scale > 0.0f) || !std::isfinite(softmax_scale))
-    return fail(PBS_ERR_INVALID_ARG, "softmax_scale must be positive and finite");
-  int* err = device_error_word();
-  if (!err) return fail(PBS_ERR_CUDA, "cannot resolve the device error word");
-  pbs::AttnParams p;
-  p.Q = Q;
-  p.K = K;
-  p.V = V;
-  p.O = O;
-  p.perm = perm;
-  p.counts = counts;
-  p.idx = idx;
-  p.cap = cap;
-  p.blk = blk;
-  p.seg = seg;
-  p.nb = static_cast<int>(Q.N / blk);
-  p.G = static_cast<int>(Q.H / K.H);
-  p.gate_thr = gate_thr;
-  p.scale_log2 = softmax_scale * 1.4426950408889634f;
-  p.lse = lse;
-  p.stats = stats;
-  p.err = err;
-  cudaError_t e = pbs::launch_attn_fwd(p, static_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) return cuda_fail(e, "attn_fwd launch");
-  return ok();
+  return attn_common(Qt, Kt, Vt, perm, counts, idx, cap, blk, seg, gate_thr, 0, 0.0f, softmax_scale,
+                     Ot, lse, stats, stream);
+}
+
+int pbs_attn_fwd_early_stop(const pbs_tensor* Qt, const pbs_tensor* Kt, const pbs_tensor* Vt,
+                            const int32_t* perm, const int32_t* counts, const int32_t* idx,
+                            int cap, int blk, int seg, float stop_tau, float softmax_scale,
+                            pbs_tensor* Ot, float* lse, long long* stats, void* stream) {
+  if (!(stop_tau >= 0.0f) || !std::isfinite(stop_tau))
+    return fail(PBS_ERR_INVALID_ARG, "stop_tau must be finite and >= 0");
+  return attn_common(Qt, Kt, Vt, perm, counts, idx, cap, blk, seg, nullptr, 1, stop_tau, softmax_scale,
+                     Ot, lse, stats, stream);
 }
 
 int pbs_check_device(void* stream) {

@@ -12,12 +12,18 @@
 // "Block Sparse Flash Attention", Approach: the exact tile maximum of QK^T
 // is compared with a per-(head, query block) threshold; below it the tile
 // adds nothing (no PV product, no softmax update).
+// S2O page, 2. Early-Stopping Rule (pbs_attn_fwd_early_stop): Pass 2 visits
+// each head's listed blocks in the order given and ends once every row's
+// marginal gain (the tile's exponential mass over the accumulated mass) is
+// below a threshold.
 //
 // sm_100a design.  One CTA per work item = (query block i, batch b, a pair
 // of query heads h0, h0+1 of the same GQA group).  The two heads share K/V,
 // so the CTA walks the UNION of their tile lists (the own segment's natural
 // blocks, then the listed permuted blocks in ascending order) and gathers
-// every K/V tile once for both heads.  Roles (384 threads):
+// every K/V tile once for both heads.  (With early stopping the two heads'
+// ordered lists are interleaved instead, each tile serving one head.)
+// Roles (384 threads):
 //   warp 0       tcgen05 MMA issuer (one thread) and tensor-memory owner;
 //   warps 1-3    producer: 16-byte cp.async row gathers of Q once and of the
 //                K and V tiles into a 2-stage ring of 128B-swizzled tiles;
@@ -77,9 +83,17 @@ struct Shared {
   int n_union;
   int skip[2][2];
   float red[2][4];
+  int vote[2][4];          // early stopping: per-warp "every row's gain is small"
+  int limit[2];            // early stopping: a head runs none of its tiles >= limit
+  int n_list[2];           // early stopping: listed tiles per head slot
 };
 
-template <int D, int BLK>
+// ES: S2O early stopping -- each head's listed blocks are visited in the
+// order given and its Pass 2 is cut once a tile's gain is small.  The two
+// heads' lists are interleaved (one tile of each in turn, every tile for one
+// head); tiles of a head that has stopped are not loaded and only passed
+// through the rings.
+template <int D, int BLK, bool ES>
 __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
   using C = Cfg<D, BLK>;
   extern __shared__ unsigned char smem_raw[];
@@ -138,7 +152,47 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
       bm[1][w] = 0u;
     }
     __syncwarp();
-    for (int h = 0; h < 2; ++h) {
+    int total = 0;
+    if (ES) {
+      // Each head's list in the order given (out-of-range and repeated
+      // entries dropped and flagged), compacted into the V ring, which is
+      // free until the producer starts; then interleaved: the k-th tiles of
+      // the two heads at 2k and 2k+1 while both lists last.
+      int32_t* scratch = reinterpret_cast<int32_t*>(smem + C::kV);
+      int nl[2] = {0, 0};
+      for (int h = 0; h < 2; ++h) {
+        const int32_t* list = p.idx + ((static_cast<int64_t>(b) * Hq + h0 + h) * p.nb + i) * p.cap;
+        for (int base = 0; base < cnt[h]; base += 32) {
+          const int e = base + lane;
+          bool keep = false;
+          int pb = 0;
+          if (e < cnt[h]) {
+            pb = list[e];
+            if (pb < 0 || pb >= ncand) {
+              set_error(p.err, kErrDeviceCheck);
+            } else if (atomicOr(&bm[h][pb >> 5], 1u << (pb & 31)) & (1u << (pb & 31))) {
+              set_error(p.err, kErrDeviceCheck);
+            } else {
+              keep = true;
+            }
+          }
+          const uint32_t km = __ballot_sync(0xffffffffu, keep);
+          if (keep) scratch[h * p.cap + nl[h] + __popc(km & ((1u << lane) - 1u))] = pb;
+          nl[h] += __popc(km);
+        }
+      }
+      __syncwarp();
+      const int m = min(nl[0], nl[1]);
+      for (int h = 0; h < 2; ++h)
+        for (int e = lane; e < nl[h]; e += 32)
+          sched[e < m ? 2 * e + h : m + e] = static_cast<uint32_t>(scratch[h * p.cap + e]) | ((1u << h) << 30);
+      total = nl[0] + nl[1];
+      if (lane == 0) {
+        sh.n_list[0] = nl[0];
+        sh.n_list[1] = nl[1];
+      }
+    }
+    for (int h = 0; h < 2 && !ES; ++h) {
       const int32_t* list = p.idx + ((static_cast<int64_t>(b) * Hq + h0 + h) * p.nb + i) * p.cap;
       for (int e = lane; e < cnt[h]; e += 32) {
         const int pb = list[e];
@@ -150,8 +204,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
       }
     }
     __syncwarp();
-    int total = 0;
-    for (int base = 0; base < words; base += 32) {
+    for (int base = 0; base < words && !ES; base += 32) {
       const int w = base + lane;
       const uint32_t m0 = w < words ? bm[0][w] : 0u, m1 = w < words ? bm[1][w] : 0u;
       uint32_t u = m0 | m1;
@@ -173,6 +226,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
     if (lane == 0) {
       sh.n_union = total;
       sh.abort = 0;
+      sh.limit[0] = 0x7fffffff;
+      sh.limit[1] = 0x7fffffff;
       mbar_init(&sh.bar_q, kProducerThreads);
       for (int st = 0; st < kStages; ++st) {
         mbar_init(&sh.bar_k[st], kProducerThreads);
@@ -198,8 +253,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
   const int T = n_diag + sh.n_union;
   const uint32_t both = has1 ? 3u : 1u;
   volatile int* abort_flag = &sh.abort;
+  volatile int* limit = sh.limit;
   // tile t: natural block i-t for t < n_diag, else sched[t - n_diag]
   auto tile_mask = [&](int t) -> uint32_t { return t < n_diag ? both : (sched[t - n_diag] >> 30); };
+  // Early stopping: does tile t still serve a head (t below that head's
+  // stop point)?  Heads that stopped have limit <= t.
+  auto live = [&](int t) -> bool {
+    const uint32_t m = tile_mask(t);
+    return ((m & 1u) && t < limit[0]) || ((m & 2u) && t < limit[1]);
+  };
+  // ... and is tile t, and every tile after it, past every head's stop point?
+  auto past_all = [&](int t) -> bool { return t >= limit[0] && (!has1 || t >= limit[1]); };
 
   if (warp >= 1 && warp <= 3) {
     // ============================================================ producer
@@ -253,6 +317,22 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
       }
     };
     if (T > 0) fetch_rows(0);
+    // Bounded wait for a ring slot.  With early stopping it also ends once
+    // the tile to be loaded is past every head's stop point: from there on
+    // nothing is run.
+    auto wait_slot = [&](uint64_t* bar, uint32_t parity, int t) -> bool {
+      if constexpr (!ES) {
+        return mbar_wait_or_abort(bar, parity, p.err, abort_flag);
+      } else {
+        for (uint32_t it = 0; it < kSpinLimit; ++it) {
+          if (mbar_try_wait(bar, parity)) return true;
+          if ((it & 15u) == 15u && (*abort_flag || past_all(t))) return false;
+        }
+        set_error(p.err, kErrTimeout);
+        *abort_flag = 1;
+        return false;
+      }
+    };
     // With gating, V of tile t-1 is issued after K of tile t, once every
     // head visiting tile t-1 has decided: a tile all of them dropped is not
     // loaded at all (its PVs are skipped too).
@@ -261,10 +341,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
     for (int t = 0; t <= T; ++t) {
       if (t < T) {
         const int st = t & 1;
-        const bool ok = t < kStages || mbar_wait_or_abort(&sh.bar_kempty[st], ((t >> 1) - 1) & 1, p.err, abort_flag);
+        const bool ok = t < kStages || wait_slot(&sh.bar_kempty[st], ((t >> 1) - 1) & 1, t);
         if (named_sync_or(1, kProducerThreads, !ok)) break;   // all producer threads leave together
         const bool nat = t < n_diag;
         const int id0 = nat ? i - t : static_cast<int>(sched[t - n_diag] & 0x3FFFFFFFu);
+        // a permuted block lies inside one segment (seg is a multiple of BLK)
+        const int64_t lo = static_cast<int64_t>((id0 * BLK) / p.seg) * p.seg;
 #pragma unroll
         for (int q = 0; q < RPT; ++q) {
           const int r = pt + q * kProducerThreads;
@@ -273,7 +355,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
           if (nat) {
             x = static_cast<int64_t>(id0) * BLK + r;
           } else {
-            const int64_t lo = ((static_cast<int64_t>(id0) * BLK + r) / p.seg) * p.seg;
             x = nxt[q];
             if (x < lo || x >= lo + p.seg || x >= N) {
               set_error(p.err, kErrDeviceCheck);
@@ -283,13 +364,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
           rowbuf[st][r] = static_cast<int32_t>(x);
         }
         named_sync(1, kProducerThreads);
-        gather_tile(sK + st * C::kKVBytes, kb, p.K.sN, rowbuf[st]);
+        if (!ES || live(t)) gather_tile(sK + st * C::kKVBytes, kb, p.K.sN, rowbuf[st]);
         cp_async_mbar_arrive(&sh.bar_k[st]);      // arrives when this thread's copies land
       }
       const int tv = gate ? t - 1 : t;            // tile whose V goes now
       if (tv >= 0 && tv < T) {
         const int sv = tv & 1;
-        bool okv = tv < kStages || mbar_wait_or_abort(&sh.bar_vempty[sv], ((tv >> 1) - 1) & 1, p.err, abort_flag);
+        bool okv = tv < kStages || wait_slot(&sh.bar_vempty[sv], ((tv >> 1) - 1) & 1, tv);
         bool keep = true;
         if (gate) {
           keep = false;
@@ -302,7 +383,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
           }
         }
         if (named_sync_or(1, kProducerThreads, !okv)) break;
-        if (keep) gather_tile(sV + sv * C::kKVBytes, vb, p.V.sN, rowbuf[sv]);
+        if (keep && (!ES || live(tv))) gather_tile(sV + sv * C::kKVBytes, vb, p.V.sN, rowbuf[sv]);
         cp_async_mbar_arrive(&sh.bar_v[sv]);
       }
       if (t + 1 < T) fetch_rows(t + 1);
@@ -337,6 +418,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
       // Per head: next tile needing QK^T, tile whose PV is pending, QK count.
       int nq[2] = {T, T}, pend[2] = {-1, -1}, kh[2] = {0, 0};
       bool o_init[2] = {false, false};
+      // Early stopping: head stopped; its next tile's K fill already passed on.
+      bool hstop[2] = {false, false}, kpassed[2] = {false, false};
       auto next_tile = [&](int h, int from) {
         int t = from;
         while (t < T && !((tile_mask(t) >> h) & 1u)) ++t;
@@ -383,9 +466,31 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
       // S's columns) has been consumed before S is overwritten.
       while (ok) {
         bool pending = false, progress = false;
+        const bool all_stopped = ES && hstop[0] && (nh < 2 || hstop[1]);
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           if (h >= nh) break;
+          if (ES && hstop[h]) {
+            // A stopped head runs nothing more, but each of its remaining
+            // tiles still occupies a ring slot in turn: pass the K and then
+            // the V fill on as they land (until every head has stopped).
+            if (nq[h] < T && !all_stopped) {
+              pending = true;
+              const int t = nq[h], st = t & 1;
+              if (!kpassed[h] && landed(sh.bar_k, ks0, ks1, t)) {
+                if (release(kt0, kt1, kl0, kl1, t) && elect_one()) tc_commit(&sh.bar_kempty[st]);
+                kpassed[h] = true;
+                progress = true;
+              }
+              if (kpassed[h] && landed(sh.bar_v, vs0, vs1, t)) {
+                if (release(vt0, vt1, vl0, vl1, t) && elect_one()) tc_commit(&sh.bar_vempty[st]);
+                kpassed[h] = false;
+                nq[h] = next_tile(h, t + 1);
+                progress = true;
+              }
+            }
+            continue;
+          }
           if (pend[h] >= 0) {
             pending = true;
             const int t = pend[h], st = t & 1;
@@ -409,9 +514,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
               if (release(vt0, vt1, vl0, vl1, t) && elect_one()) tc_commit(&sh.bar_vempty[st]);
               pend[h] = -1;
               progress = true;
+              if (ES) {
+                // lane 0 acquired bar_p, after which the stop point this
+                // tile's softmax pass may have set is visible
+                int lim = 0;
+                if (leader) lim = limit[h];
+                hstop[h] = __shfl_sync(0xffffffffu, lim, 0) <= t + 1;
+              }
             }
           }
-          if (pend[h] < 0 && nq[h] < T) {
+          if (pend[h] < 0 && nq[h] < T && !(ES && hstop[h])) {
             pending = true;
             const int t = nq[h], st = t & 1;
             if (landed(sh.bar_k, ks0, ks1, t)) {
@@ -482,15 +594,53 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
       if (!ok) break;
       tc_fence_after();
       ++n_qk;
+      // Block-max gate first: the tile's raw maximum over all rows decides
+      // before any exponential is taken, so a dropped tile costs one read of
+      // S and a reduction.  A dropped tile leaves m, l and O as they were;
+      // the diagonal tile (t == 0) is never gated.
+      if (p.gate_thr && t != 0) {
+        float rm = -INFINITY;
+#pragma unroll 1
+        for (int c = 0; c < BLK / 64; ++c) {
+          uint32_t x[64];
+          tmem_ld64(tS + c * 64, x);
+          float mm[8];
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            mm[q] = fmax3(__uint_as_float(x[q]), __uint_as_float(x[8 + q]), __uint_as_float(x[16 + q]));
+            mm[q] = fmax3(mm[q], __uint_as_float(x[24 + q]), __uint_as_float(x[32 + q]));
+            mm[q] = fmax3(mm[q], __uint_as_float(x[40 + q]), __uint_as_float(x[48 + q]));
+            mm[q] = fmaxf(mm[q], __uint_as_float(x[56 + q]));
+          }
+          rm = fmaxf(rm, fmax3(fmax3(mm[0], mm[1], mm[2]), fmax3(mm[3], mm[4], mm[5]), fmaxf(mm[6], mm[7])));
+        }
+        const float wm = warp_max(r < BLK ? rm : -INFINITY);
+        if (lane == 0) sh.red[h][warp & 3] = wm;
+        named_sync(2 + h, 128);
+        const float tmax = fmaxf(fmaxf(sh.red[h][0], sh.red[h][1]), fmaxf(sh.red[h][2], sh.red[h][3]));
+        named_sync(2 + h, 128);
+        const bool keep = !(tmax < thr);
+        if (r == 0) {
+          sh.gkeep[h][k & 1] = keep ? 1 : 0;
+          mbar_arrive(&sh.bar_g[h]);
+        }
+        if (!keep) {
+          ++n_gated;
+          if (r == 0) sh.skip[h][k & 1] = 1;
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sh.bar_p[h]);     // one arrival per warp
+          ++k;
+          continue;
+        }
+      }
       // One pass over S in 64-column chunks.  P = 2^(s*scale - m) is taken
       // against a running max m that starts at the row's max so far; when a
       // chunk's max exceeds m by more than 2^8, m moves up and the P columns
       // already written for this tile are rescaled in place (rare after the
-      // first tile).  So P stays below 2^8 and S is read once.  The tile's
-      // raw max decides the gate at the end; a gated tile leaves m, l and O
-      // as they were.
+      // first tile).  So P stays below 2^8 and S is read once here.
       const bool causal = t == 0;
-      float rmax = -INFINITY, psum = 0.f, m_t = m_run;
+      float psum = 0.f, m_t = m_run;
 #pragma unroll 1
       for (int c = 0; c < BLK / 64; ++c) {
         uint32_t x[64], u[32];
@@ -515,7 +665,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
           }
           cmax = fmax3(fmax3(mm[0], mm[1], mm[2]), fmax3(mm[3], mm[4], mm[5]), fmaxf(mm[6], mm[7]));
         }
-        rmax = fmaxf(rmax, cmax);
         const float cm = cmax * p.scale_log2;
         const bool up = cm > (m_t == -INFINITY ? -INFINITY : m_t + kRescaleSlack);
         if (__any_sync(0xffffffffu, up)) {
@@ -571,28 +720,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
         }
         tmem_st32(tS + c * 32, u);
       }
-      if (p.gate_thr && !causal) {
-        const float wm = warp_max(r < BLK ? rmax : -INFINITY);
-        if (lane == 0) sh.red[h][warp & 3] = wm;
-        named_sync(2 + h, 128);
-        const float tmax = fmaxf(fmaxf(sh.red[h][0], sh.red[h][1]), fmaxf(sh.red[h][2], sh.red[h][3]));
-        named_sync(2 + h, 128);
-        if (tmax < thr) {
-          ++n_gated;
-          if (r == 0) {
-            sh.gkeep[h][k & 1] = 0;
-            mbar_arrive(&sh.bar_g[h]);
-          }
-          tmem_st_wait();
-          if (r == 0) sh.skip[h][k & 1] = 1;
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&sh.bar_p[h]);     // one arrival per warp
-          ++k;
-          continue;
-        }
-      }
-      if (p.gate_thr && r == 0) {               // kept (the diagonal tile always is)
+      if (p.gate_thr && r == 0 && causal) {     // the diagonal tile is always kept
         sh.gkeep[h][k & 1] = 1;
         mbar_arrive(&sh.bar_g[h]);
       }
@@ -612,6 +740,23 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
       }
       l_run = l_run * alpha + psum;
       m_run = m_new;
+      // Early stopping (Pass 2 only): this tile's gain per row is psum / l,
+      // its exponential mass over the accumulated mass, both in the frame
+      // of m; when every row's gain is below stop_tau the later tiles are
+      // not run.  The stop point is published before P is, so the MMA
+      // thread sees it when it takes this tile's PV.
+      bool stop_now = false;
+      if (ES && t >= n_diag) {
+        const bool small = !(r < BLK) || psum < p.stop_tau * l_run;
+        const bool wsmall = __all_sync(0xffffffffu, small);
+        if (lane == 0) sh.vote[h][warp & 3] = wsmall ? 1 : 0;
+        named_sync(2 + h, 128);
+        stop_now = (sh.vote[h][0] & sh.vote[h][1] & sh.vote[h][2] & sh.vote[h][3]) != 0;
+        if (stop_now) {
+          if (r == 0) sh.limit[h] = t + 1;
+          n_gated += n_diag + sh.n_list[h] - (k + 1);   // listed tiles left out
+        }
+      }
       tmem_st_wait();
       if (r == 0) sh.skip[h][k & 1] = 0;
       tc_fence_before();
@@ -619,6 +764,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
       if (lane == 0) mbar_arrive(&sh.bar_p[h]);         // one arrival per warp
       o_init = true;
       ++k;
+      if (stop_now) break;
     }
     // ---- epilogue: O / l -> bf16, LSE
     if (active && ok && k > 0) {
@@ -662,22 +808,29 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
   }
 }
 
-template <int D, int BLK>
+template <int D, int BLK, bool ES>
 cudaError_t launch_typed(const AttnParams& p, cudaStream_t s) {
   using C = Cfg<D, BLK>;
   // schedule: at most min(candidates, 2 * cap) permuted tiles per item
-  const int max_union = std::min(p.nb, 2 * p.cap);
+  // (with early stopping both lists in full, compacted first in the V ring)
+  const int max_union = ES ? 2 * p.cap : std::min(p.nb, 2 * p.cap);
+  if (ES && 2 * p.cap * 4 > kStages * C::kKVBytes) return cudaErrorInvalidValue;
   int smem = 1024 + C::kEnd + 4 * max_union;
   smem = smem < C::kMinSmem ? C::kMinSmem : smem;
   if (smem + 4096 > 227 * 1024) return cudaErrorInvalidValue;   // + static shared memory
-  cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D, BLK>,
+  cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D, BLK, ES>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const int npair = (p.G + 1) / 2;
   const int64_t items = static_cast<int64_t>(p.nb) * p.Q.B * p.K.H * npair;
   if (items >= (1ll << 31)) return cudaErrorInvalidValue;
-  attn_fwd_kernel<D, BLK><<<static_cast<unsigned>(items), kThreads, smem, s>>>(p);
+  attn_fwd_kernel<D, BLK, ES><<<static_cast<unsigned>(items), kThreads, smem, s>>>(p);
   return cudaGetLastError();
+}
+
+template <int D, int BLK>
+cudaError_t launch_mode(const AttnParams& p, cudaStream_t s) {
+  return p.early_stop ? launch_typed<D, BLK, true>(p, s) : launch_typed<D, BLK, false>(p, s);
 }
 
 }  // namespace
@@ -685,10 +838,10 @@ cudaError_t launch_typed(const AttnParams& p, cudaStream_t s) {
 cudaError_t launch_attn_fwd(const AttnParams& p, cudaStream_t s) {
   const int D = static_cast<int>(p.Q.D);
   if (p.nb > 8192) return cudaErrorInvalidValue;
-  if (D == 128 && p.blk == 128) return launch_typed<128, 128>(p, s);
-  if (D == 128 && p.blk == 64) return launch_typed<128, 64>(p, s);
-  if (D == 64 && p.blk == 128) return launch_typed<64, 128>(p, s);
-  if (D == 64 && p.blk == 64) return launch_typed<64, 64>(p, s);
+  if (D == 128 && p.blk == 128) return launch_mode<128, 128>(p, s);
+  if (D == 128 && p.blk == 64) return launch_mode<128, 64>(p, s);
+  if (D == 64 && p.blk == 128) return launch_mode<64, 128>(p, s);
+  if (D == 64 && p.blk == 64) return launch_mode<64, 64>(p, s);
   return cudaErrorInvalidValue;
 }
 

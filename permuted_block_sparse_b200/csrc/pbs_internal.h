@@ -27,6 +27,7 @@ cudaError_t launch_pool_key_blocks(const TensorDesc& K, const int32_t* perm, int
                                    int32_t* inv, int* err, cudaStream_t s);
 struct SelectParams {
   int B, Hq, Hkv, D, blk, seg, nb, mode, band, n_sink, cap;
+  int score_order;        // lists in visiting order instead of ascending
   int64_t N;
   int64_t rho_permille;   // top-k density in per-mille
   double tau;
@@ -52,6 +53,8 @@ struct AttnParams {
   const int32_t* idx;
   int cap, blk, seg, nb, G;
   const float* gate_thr;
+  int early_stop;         // S2O early stopping: lists in visiting order, cut by stop_tau
+  float stop_tau;
   float scale_log2;       // softmax scale * log2(e)
   float* lse;
   long long* stats;

@@ -335,7 +335,8 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32) select_topk_kernel(
 // Cumulative-mass selection, one CTA per (query block, query head, batch):
 // the row's candidates are sorted by (forced first, descending score, lower
 // block id) and taken in that order while the accumulated softmax mass (fp64,
-// own segment included) is below tau.
+// own segment included) is below tau.  The same kernel serves top-k when the
+// lists are wanted in that visiting order (the first `want` sorted keys).
 __global__ void __launch_bounds__(kSelThreads) select_tau_kernel(
     SelectParams p, const float* __restrict__ S_all, const float* __restrict__ qbar,
     const float* __restrict__ kbar_nat, const int32_t* __restrict__ inv,
@@ -486,6 +487,21 @@ __global__ void __launch_bounds__(kSelThreads) select_tau_kernel(
     want = max(nf, sh_int[1]);
   }
 
+  if (p.score_order) {
+    // Visiting order: the chosen blocks are the first `want` of the sorted
+    // keys (forced first, then descending score, ties to the lower block).
+    if (want > p.cap) {
+      if (threadIdx.x == 0) {
+        set_error(err, kErrDeviceCheck);
+        counts[row] = 0;
+      }
+      return;
+    }
+    int32_t* out = idx + row * p.cap;
+    for (int t = threadIdx.x; t < want; t += blockDim.x) out[t] = static_cast<int32_t>(keys[t] & 0xffffffffu);
+    if (threadIdx.x == 0) counts[row] = want;
+    return;
+  }
   // Mark the chosen blocks and write them in ascending order.
   for (int t = threadIdx.x; t < n2; t += blockDim.x) flag[t] = 0;
   __syncthreads();
@@ -549,7 +565,7 @@ cudaError_t launch_select_blocks(const SelectParams& p, const float* qbar, const
   block_scores_kernel<<<g1, 256, 0, s>>>(p, qbar, kbar_perm, scores);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  if (p.mode == PBS_SELECT_TOPK) {
+  if (p.mode == PBS_SELECT_TOPK && !p.score_order) {
     const size_t smem = static_cast<size_t>(kWarpsPerCta) * (p.nb / 32 + 1) * 4;
     e = cudaFuncSetAttribute(select_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;

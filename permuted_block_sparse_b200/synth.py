@@ -55,6 +55,7 @@ class Workload:
     band: int = 0             # most recent keys always kept (0 = none)
     n_sink: int = 0           # leading sink keys always kept
     gate_keep: int = 0        # gating: calibrate thresholds to keep this many tiles
+    stop_tau: float = 0.0     # S2O early stopping threshold (0 = no early stopping)
     stripe_frac: float = 0.0
     c_lo: float = 4.0
     c_hi: float = 4.0
@@ -73,7 +74,7 @@ class Workload:
         return dataclasses.replace(self, **kw)
 
 
-# The five workloads.  Sizes, block/segment sizes, selection knobs and stripe
+# The benchmark workloads.  Sizes, block/segment sizes, selection knobs and stripe
 # recipes are the ones the benchmark plan states; the query offset 1.5 is the
 # single-head case's value, reused for the others, which leave it open.
 WORKLOADS = {
@@ -98,6 +99,13 @@ WORKLOADS = {
     "gate_b1_64k": Workload(
         "gate_b1_64k", B=1, Hq=32, Hkv=8, N=65536, d=128, blk=128, seg=128,
         mode="gate", gate_keep=64, stripe_frac=0.005, c_lo=3.0, c_hi=6.0),
+    # S2O early stopping: every candidate block listed in descending block
+    # score, Pass 2 cut once a tile adds less than 2 % of the accumulated
+    # mass.  The pages give no threshold; 2 % is an operating point at which
+    # late query blocks of these inputs run about a fifth of their candidates.
+    "s2o_32k_stop": Workload(
+        "s2o_32k_stop", B=1, Hq=32, Hkv=8, N=32768, d=128, blk=128, seg=2048,
+        mode="topk", density=1.0, stop_tau=0.02, stripe_frac=0.005, c_lo=3.0, c_hi=6.0),
 }
 
 

@@ -123,6 +123,25 @@ def test_attn_rejects_mismatched_output(lib):
     assert rc == -1
 
 
+def test_early_stop_and_score_order_argument_checks(lib):
+    q, k, v, o = _desc(H=2), _desc(H=1), _desc(H=1), _desc(H=2)
+    for tau in (-0.1, float("nan"), float("inf")):
+        rc = lib.pbs_attn_fwd_early_stop(ctypes.byref(q), ctypes.byref(k), ctypes.byref(v),
+                                         ctypes.c_void_p(0x2000), ctypes.c_void_p(0x3000),
+                                         ctypes.c_void_p(0x5000), 4, 128, 256, tau, 0.088, ctypes.byref(o),
+                                         None, None, None)
+        assert rc == -1 and b"stop_tau" in lib.pbs_get_last_error(), tau
+    # the visiting-order flag leaves the capacity unchanged; other flag bits are refused
+    assert (lib.pbs_select_capacity(32768, 128, 2048, 0x10 | 0, 0.3, 0, 0)
+            == lib.pbs_select_capacity(32768, 128, 2048, 0, 0.3, 0, 0))
+    q, k = _desc(H=2, N=1024), _desc(H=1, N=1024)
+    cap = pbs.select_capacity(1024, 128, 256, "topk", 0.5)
+    rc = lib.pbs_select(ctypes.byref(q), ctypes.byref(k), ctypes.c_void_p(0x2000), 128, 256, 0x20, 0.5, 0, 0,
+                        ctypes.c_void_p(0x3000), ctypes.c_void_p(0x5000), cap, ctypes.c_void_p(0x4000),
+                        1 << 30, None)
+    assert rc == -1
+
+
 def test_binding_refuses_cpu_tensors(lib):
     import torch
     x = torch.zeros(1, 1, 128, 64, dtype=torch.bfloat16)
