@@ -337,6 +337,36 @@ def run_pbs(args):
         dms = a.elapsed_time(b) / reps
         dense = {"ms": dms, "tflops": causal_tiles * tile_flops(w) / (dms * 1e-3) / 1e12,
                  "speedup_of_sparse_step": dms / ms_step}
+        # Attention coverage (outside the timed region): the share of each
+        # row's full causal softmax mass on its key set is exp(LSE over the
+        # key set - LSE over all causal keys).  The permuted selection of the
+        # timed step is compared with the same selection rule on the natural
+        # key order (identity permutation) at the same settings.
+        if not gate:
+            lse_all = torch.empty_like(lse)
+            pbs.pbs_attn_fwd(Q, K, V, ident, d_counts, d_idx, w.blk, w.blk, out=Od, lse=lse_all)
+            cov_perm = torch.exp(lse - lse_all).flatten()
+            c_nat = torch.empty_like(counts)
+            i_nat = torch.empty_like(idx)
+            pbs.pbs_select(Q, K, ident, w.blk, w.seg, w.mode, dt, w.band, w.n_sink, cap=cap, counts=c_nat,
+                           idx=i_nat, ws=ws_s, score_order=early)
+            lse_nat = torch.empty_like(lse)
+            if early:
+                pbs.pbs_attn_fwd_early_stop(Q, K, V, ident, c_nat, i_nat, w.blk, w.seg, w.stop_tau, out=Od,
+                                            lse=lse_nat)
+            else:
+                pbs.pbs_attn_fwd(Q, K, V, ident, c_nat, i_nat, w.blk, w.seg, out=Od, lse=lse_nat)
+            pbs.pbs_check_device()
+            cov_nat = torch.exp(lse_nat - lse_all).flatten()
+            q = torch.tensor([0.01, 0.5], device=dev)
+            sample = torch.randperm(cov_perm.numel(), device=dev)[:1 << 20]
+            pq = torch.quantile(cov_perm[sample], q).tolist()
+            nq = torch.quantile(cov_nat[sample], q).tolist()
+            dense["coverage"] = {"permuted": {"mean": cov_perm.mean().item(), "p01": pq[0], "median": pq[1]},
+                                 "natural": {"mean": cov_nat.mean().item(), "p01": nq[0], "median": nq[1]},
+                                 "what": "share of each query row's causal softmax mass on its key set, "
+                                         "permuted keys vs the same rule on natural key order"}
+            del lse_all, c_nat, i_nat, lse_nat
         del d_idx, Od
 
     # end to end through the C ABI with host buffers: H2D of Q, K, V from

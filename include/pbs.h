@@ -159,8 +159,8 @@ int pbs_select(const pbs_tensor* Q, const pbs_tensor* K, const int32_t* perm,
  *     map into its own segment); counts/idx as produced by pbs_select.
  *   gate_thr: NULL, or device fp32 [B, Hq, N/blk] in raw q.k units: a tile
  *     other than block i's own whose largest visible raw q.k is below
- *     gate_thr[b,hq,i] is skipped entirely (no V load, no PV, no softmax
- *     update).
+ *     gate_thr[b,hq,i] adds nothing (no PV product, no softmax update;
+ *     its V rows are still gathered, ahead of the decision).
  *   O: bf16 output, same shape as Q.  lse: NULL or device fp32 [B, Hq, N],
  *     natural-log normaliser of the scaled logits.
  *   stats: NULL or device int64[2], incremented by (tiles whose QK^T was

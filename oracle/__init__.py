@@ -5,7 +5,7 @@ and by the benchmark's CPU-baseline leg, never by the product path.
 """
 from .pbs_oracle import *  # noqa: F401,F403
 from .pbs_oracle import (attn, attn_block, attn_blocks, attn_early_stop, attn_early_stop_block,
-                         calibrate_thresholds, dense_lists,
+                         calibrate_thresholds, coverage_block, dense_lists,
                          diagonal_blocks, forced_blocks, inverse_permutation,
                          key_scores, key_tiles,
                          lists_to_array, n_candidates, natural_key_block_sums,

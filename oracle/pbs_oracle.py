@@ -456,6 +456,30 @@ def attn_early_stop(Q, K, V, perm, lists: dict, blk: int, seg: int, stop_tau: fl
     return out
 
 
+def coverage_block(Q, K, perm, listed, b, hq, i, blk, seg, scale) -> np.ndarray:
+    """Per query row of block i: the share of the row's full causal softmax
+    mass that falls on the block's key set (the own segment's causal keys
+    and the listed permuted blocks), fp64 from explicit exponentials.
+
+    This is the attention-coverage measure behind "Sparser Block-Sparse
+    Attention via Token Permutation", Key Results (fewer blocks for the same
+    coverage once keys are permuted)."""
+    Hq, Hkv = Q.shape[1], K.shape[1]
+    hk = hq // (Hq // Hkv)
+    q_pos = np.arange(i * blk, (i + 1) * blk)
+    q = Q[b, hq, i * blk:(i + 1) * blk].astype(F64)
+    keys = np.arange((i + 1) * blk)
+    lg = (q @ K[b, hk, keys].astype(F64).T) * scale
+    vis = keys[None, :] <= q_pos[:, None]
+    lg = np.where(vis, lg, -np.inf)
+    m = lg.max(axis=1, keepdims=True)
+    e = np.exp(lg - m)
+    inset = np.zeros(keys.size, bool)
+    for _, _, pos in key_tiles(i, listed, perm[b, hk], blk, seg):
+        inset[pos] = True
+    return (e * inset[None, :]).sum(axis=1) / e.sum(axis=1)
+
+
 # --------------------------------------------------------------------------
 # 6. gate calibration
 # --------------------------------------------------------------------------

@@ -76,8 +76,6 @@ struct Shared {
   uint64_t bar_q;
   uint64_t bar_k[kStages], bar_v[kStages], bar_kempty[kStages], bar_vempty[kStages];
   uint64_t bar_s[2], bar_p[2], bar_o[2], bar_fin;
-  uint64_t bar_g[2];       // gate decisions, one arrival per decided tile of a head
-  int gkeep[2][2];         // [head][decision parity]: tile kept by this head
   uint32_t tmem_base;
   int abort;
   int n_union;
@@ -241,8 +239,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
         mbar_init(&sh.bar_o[h], 1);
       }
       mbar_init(&sh.bar_fin, 1);
-      mbar_init(&sh.bar_g[0], 1);
-      mbar_init(&sh.bar_g[1], 1);
       fence_mbar_init();
     }
   }
@@ -333,13 +329,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
         return false;
       }
     };
-    // With gating, V of tile t-1 is issued after K of tile t, once every
-    // head visiting tile t-1 has decided: a tile all of them dropped is not
-    // loaded at all (its PVs are skipped too).
-    const bool gate = p.gate_thr != nullptr;
-    int gk[2] = {0, 0};
-    for (int t = 0; t <= T; ++t) {
-      if (t < T) {
+    // V of tile t is gathered right after its K, also under gating: the
+    // gate decides only after the tile's QK^T, and waiting for the decision
+    // would put the gather's latency in front of every kept tile's PV.
+    // (A dropped tile's V is gathered but never multiplied.)
+    for (int t = 0; t < T; ++t) {
+      {                                           // K of tile t
         const int st = t & 1;
         const bool ok = t < kStages || wait_slot(&sh.bar_kempty[st], ((t >> 1) - 1) & 1, t);
         if (named_sync_or(1, kProducerThreads, !ok)) break;   // all producer threads leave together
@@ -367,23 +362,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
         if (!ES || live(t)) gather_tile(sK + st * C::kKVBytes, kb, p.K.sN, rowbuf[st]);
         cp_async_mbar_arrive(&sh.bar_k[st]);      // arrives when this thread's copies land
       }
-      const int tv = gate ? t - 1 : t;            // tile whose V goes now
-      if (tv >= 0 && tv < T) {
-        const int sv = tv & 1;
-        bool okv = tv < kStages || wait_slot(&sh.bar_vempty[sv], ((tv >> 1) - 1) & 1, tv);
-        bool keep = true;
-        if (gate) {
-          keep = false;
-          const uint32_t mask = tile_mask(tv);
-          for (int h = 0; h < 2; ++h) {
-            if (!((mask >> h) & 1u)) continue;
-            okv = okv && mbar_wait_or_abort(&sh.bar_g[h], gk[h] & 1, p.err, abort_flag);
-            keep = keep || (okv && sh.gkeep[h][gk[h] & 1]);
-            ++gk[h];
-          }
-        }
+      {                                           // V of tile t
+        const int sv = t & 1;
+        const bool okv = t < kStages || wait_slot(&sh.bar_vempty[sv], ((t >> 1) - 1) & 1, t);
         if (named_sync_or(1, kProducerThreads, !okv)) break;
-        if (keep && (!ES || live(tv))) gather_tile(sV + sv * C::kKVBytes, vb, p.V.sN, rowbuf[sv]);
+        if (!ES || live(t)) gather_tile(sV + sv * C::kKVBytes, vb, p.V.sN, rowbuf[sv]);
         cp_async_mbar_arrive(&sh.bar_v[sv]);
       }
       if (t + 1 < T) fetch_rows(t + 1);
@@ -619,12 +602,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
         named_sync(2 + h, 128);
         const float tmax = fmaxf(fmaxf(sh.red[h][0], sh.red[h][1]), fmaxf(sh.red[h][2], sh.red[h][3]));
         named_sync(2 + h, 128);
-        const bool keep = !(tmax < thr);
-        if (r == 0) {
-          sh.gkeep[h][k & 1] = keep ? 1 : 0;
-          mbar_arrive(&sh.bar_g[h]);
-        }
-        if (!keep) {
+        if (tmax < thr) {
           ++n_gated;
           if (r == 0) sh.skip[h][k & 1] = 1;
           tc_fence_before();
@@ -719,10 +697,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
           psum += ((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7));
         }
         tmem_st32(tS + c * 32, u);
-      }
-      if (p.gate_thr && r == 0 && causal) {     // the diagonal tile is always kept
-        sh.gkeep[h][k & 1] = 1;
-        mbar_arrive(&sh.bar_g[h]);
       }
       const float m_new = m_t;
       const float alpha = ex2(m_run - m_new);

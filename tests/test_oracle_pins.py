@@ -525,3 +525,35 @@ def test_early_stop_limits():
         O_ref, L_ref = oracle.attn_block(Q, K, V, perm, listed[:1], b, h, i, blk, seg, scale)
         assert n == min(1, len(listed))
         np.testing.assert_allclose(O, O_ref, rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# attention coverage (PBS page, Key Results)
+# ---------------------------------------------------------------------------
+
+def test_coverage_definition():
+    """Coverage is 1 with every candidate listed; with a partial list it
+    equals exp(LSE over the key set - LSE over all causal keys), the two
+    LSEs taken from the (SDPA-pinned) attention oracle; it never decreases
+    as blocks are added."""
+    B, Hq, Hkv, N, d, blk, seg = 1, 2, 1, 512, 16, 16, 128
+    Q, K, V = _small(B, Hq, Hkv, N, d, seed=51, scale=2.0)
+    perm = oracle.permute(Q, K, blk, seg)
+    scale = 1.0 / math.sqrt(d)
+    _, full = oracle.select(Q, K, perm, blk, seg, "topk", density=1.0)
+    _, part = oracle.select(Q, K, perm, blk, seg, "topk", density=0.3, list_order="score")
+    checked = 0
+    for (b, h, i), listed in part.items():
+        c_full = oracle.coverage_block(Q, K, perm, full[(b, h, i)], b, h, i, blk, seg, scale)
+        np.testing.assert_allclose(c_full, 1.0, rtol=0, atol=1e-12)
+        c = oracle.coverage_block(Q, K, perm, listed, b, h, i, blk, seg, scale)
+        _, l_sel = oracle.attn_block(Q, K, V, perm, listed, b, h, i, blk, seg, scale)
+        _, l_all = oracle.attn_block(Q, K, V, perm, full[(b, h, i)], b, h, i, blk, seg, scale)
+        np.testing.assert_allclose(c, np.exp(l_sel - l_all), rtol=1e-12, atol=0)
+        prev = oracle.coverage_block(Q, K, perm, listed[:0], b, h, i, blk, seg, scale)
+        for k in range(1, len(listed) + 1):
+            cur = oracle.coverage_block(Q, K, perm, listed[:k], b, h, i, blk, seg, scale)
+            assert np.all(cur >= prev - 1e-15)
+            prev = cur
+        checked += len(listed) > 0
+    assert checked > 10
