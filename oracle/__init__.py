@@ -9,6 +9,7 @@ from .pbs_oracle import (attn, attn_block, attn_blocks, attn_early_stop, attn_ea
                          diagonal_blocks, forced_blocks, inverse_permutation,
                          key_scores, key_tiles,
                          lists_to_array, n_candidates, natural_key_block_sums,
-                         permute, permuted_key_block_sums, proxy_query,
+                         perm_for_block, permute, permute_segmented, permuted_key_block_sums,
+                         proxy_query, segment_queries,
                          query_block_sums, segment_of_block, select,
                          sort_segments, tile_maxima, topk_target)

@@ -142,6 +142,54 @@ def permute(Q: np.ndarray, K: np.ndarray, blk: int, seg: int, n_sink: int = 0) -
     return sort_segments(key_scores(qhat, K, n_sink), seg)
 
 
+def segment_queries(Q: np.ndarray, Hkv: int, seg: int) -> np.ndarray:
+    """qbar[b, hkv, s, :] = sum of every query row of segment s of every
+    query head in KV head hkv's group (fp64): the segment's representative
+    query.  Returns [B, Hkv, nseg, d]."""
+    B, Hq, N, d = Q.shape
+    G = Hq // Hkv
+    nseg = (N + seg - 1) // seg
+    out = np.zeros((B, Hkv, nseg, d), F64)
+    for b in range(B):
+        for h in range(Hkv):
+            for t in range(nseg):
+                rows = Q[b, h * G:(h + 1) * G, t * seg:min((t + 1) * seg, N), :].astype(F64)
+                out[b, h, t] = rows.reshape(-1, d).sum(axis=0)
+    return out
+
+
+def permute_segmented(Q: np.ndarray, K: np.ndarray, blk: int, seg: int, n_sink: int = 0) -> np.ndarray:
+    """One key permutation per query segment (S2O's historical KV permutation).
+
+    "S2O: Early Stopping for Sparse Attention via Online Permutation",
+    Technical Summary, 1. Online Permutation via Index-Driven Loading: the
+    historical keys are scored against a representative query of the
+    segment, and only prefix keys are considered.  For query segment s the
+    keys are scored against s's representative query (segment_queries; sinks
+    get +inf); each key segment before s is sorted by those scores
+    (descending, ties in ascending position); key segments from s on are not
+    s's history and keep their natural order.  Returns perm[b, hkv, s, p],
+    [B, Hkv, nseg, N] int32."""
+    B, Hkv, N, d = K.shape
+    qs = segment_queries(Q, Hkv, seg)
+    nseg = qs.shape[2]
+    out = np.empty((B, Hkv, nseg, N), np.int32)
+    for t in range(nseg):
+        sc = key_scores(qs[:, :, t], K, n_sink)
+        srt = sort_segments(sc, seg)
+        out[:, :, t] = np.arange(N, dtype=np.int32)
+        out[:, :, t, :t * seg] = srt[:, :, :t * seg]
+    return out
+
+
+def perm_for_block(perm: np.ndarray, b: int, hk: int, i: int, blk: int, seg: int) -> np.ndarray:
+    """The key permutation query block i reads: the KV head's ([B, Hkv, N]),
+    or its query segment's ([B, Hkv, nseg, N], permute_segmented)."""
+    if perm.ndim == 3:
+        return perm[b, hk]
+    return perm[b, hk, segment_of_block(i, blk, seg)]
+
+
 # --------------------------------------------------------------------------
 # 3-4. block selection
 # --------------------------------------------------------------------------
@@ -221,21 +269,21 @@ def select(Q: np.ndarray, K: np.ndarray, perm: np.ndarray, blk: int, seg: int,
     if rows is None:
         rows = [(b, h, i) for b in range(B) for h in range(Hq) for i in range(nb)]
     rows = list(rows)
-    need_q = sorted({(b, h) for b, h, _ in rows})
     counts = np.zeros((B, Hq, nb), np.int32)
     lists = {}
     kbar_p = {}
     kbar_n = {}
     inv = {}
-    for (b, h) in need_q:
-        hk = h // G
-        if (b, hk) not in kbar_p:
-            kbar_p[(b, hk)] = permuted_key_block_sums(K[b:b + 1, hk:hk + 1], perm[b:b + 1, hk:hk + 1], blk)[0, 0]
-            kbar_n[(b, hk)] = natural_key_block_sums(K[b:b + 1, hk:hk + 1], blk)[0, 0]
-            inv[(b, hk)] = inverse_permutation(perm[b, hk])
     qbar_cache = {}
     for (b, h, i) in rows:
         hk = h // G
+        pkey = (b, hk) if perm.ndim == 3 else (b, hk, segment_of_block(i, blk, seg))
+        if pkey not in kbar_p:
+            prow = perm_for_block(perm, b, hk, i, blk, seg)
+            kbar_p[pkey] = permuted_key_block_sums(K[b:b + 1, hk:hk + 1], prow[None, None], blk)[0, 0]
+            inv[pkey] = inverse_permutation(prow)
+        if (b, hk) not in kbar_n:
+            kbar_n[(b, hk)] = natural_key_block_sums(K[b:b + 1, hk:hk + 1], blk)[0, 0]
         if (b, h) not in qbar_cache:
             qbar_cache[(b, h)] = query_block_sums(Q[b:b + 1, h:h + 1], blk)[0, 0]
         qb = qbar_cache[(b, h)][i]
@@ -245,8 +293,8 @@ def select(Q: np.ndarray, K: np.ndarray, perm: np.ndarray, blk: int, seg: int,
         if ncand == 0:
             lists[(b, h, i)] = np.zeros(0, np.int32)
             continue
-        S = kbar_p[(b, hk)][:ncand] @ qb                      # exact on lattice inputs
-        F = forced_blocks(i, inv[(b, hk)], blk, seg, band, n_sink)
+        S = kbar_p[pkey][:ncand] @ qb                         # exact on lattice inputs
+        F = forced_blocks(i, inv[pkey], blk, seg, band, n_sink)
         rest = np.setdiff1d(np.arange(ncand, dtype=np.int64), np.array(F, np.int64))
         # descending score, ties to the lower block id
         order = rest[np.lexsort((rest, -S[rest]))] if rest.size else rest
@@ -331,7 +379,7 @@ def attn_block(Q, K, V, perm, listed, b, hq, i, blk, seg, scale,
     q_pos = np.arange(i * blk, (i + 1) * blk)
     q = Q[b, hq, i * blk:(i + 1) * blk].astype(F64)
     keys, kmask = [], []
-    for kind, tid, pos in key_tiles(i, listed, perm[b, hk], blk, seg):
+    for kind, tid, pos in key_tiles(i, listed, perm_for_block(perm, b, hk, i, blk, seg), blk, seg):
         visible = pos[None, :] <= q_pos[:, None]
         if gate_thr is not None and not (kind == "diag" and tid == i):
             raw = q @ K[b, hk, pos].astype(F64).T
@@ -419,8 +467,9 @@ def attn_early_stop_block(Q, K, V, perm, listed, b, hq, i, blk, seg, scale, stop
     acc = e @ V[b, hk, own].astype(F64)
     # Pass 2: listed permuted blocks in the given order (all keys visible)
     n_run = 0
+    prow = perm_for_block(perm, b, hk, i, blk, seg)
     for pb in listed:
-        pos = perm[b, hk, int(pb) * blk:(int(pb) + 1) * blk].astype(np.int64)
+        pos = prow[int(pb) * blk:(int(pb) + 1) * blk].astype(np.int64)
         lg = (q @ K[b, hk, pos].astype(F64).T) * scale
         m_new = np.maximum(m, lg.max(axis=1))
         alpha = np.exp(m - m_new)
@@ -475,7 +524,7 @@ def coverage_block(Q, K, perm, listed, b, hq, i, blk, seg, scale) -> np.ndarray:
     m = lg.max(axis=1, keepdims=True)
     e = np.exp(lg - m)
     inset = np.zeros(keys.size, bool)
-    for _, _, pos in key_tiles(i, listed, perm[b, hk], blk, seg):
+    for _, _, pos in key_tiles(i, listed, perm_for_block(perm, b, hk, i, blk, seg), blk, seg):
         inset[pos] = True
     return (e * inset[None, :]).sum(axis=1) / e.sum(axis=1)
 

@@ -557,3 +557,100 @@ def test_coverage_definition():
             prev = cur
         checked += len(listed) > 0
     assert checked > 10
+
+
+# ---------------------------------------------------------------------------
+# per-query-segment key permutation (S2O, Technical Summary 1: historical
+# KV permutation against a representative query of each segment)
+# ---------------------------------------------------------------------------
+
+def test_segment_queries_closed_form():
+    """The representative query of segment s is the plain sum of its rows
+    over the group's heads: checked on inputs whose rows encode their
+    position, head and dimension."""
+    B, Hq, Hkv, N, d, seg = 1, 4, 2, 64, 8, 16
+    Q = np.zeros((B, Hq, N, d), np.float32)
+    for h in range(Hq):
+        for n in range(N):
+            Q[0, h, n] = (h + 1) * 0.125 + (n % seg) * 0.5 + np.arange(d) * 0.25 + (n // seg) * 4
+    qs = oracle.segment_queries(Q, Hkv, seg)
+    G = Hq // Hkv
+    for hk in range(Hkv):
+        for s in range(N // seg):
+            # closed form: sum over heads g and rows r of the formula above
+            heads = sum((hk * G + g + 1) * 0.125 for g in range(G)) * seg
+            rows = G * sum(r * 0.5 for r in range(seg))
+            want = heads + rows + G * seg * (np.arange(d) * 0.25 + s * 4)
+            np.testing.assert_allclose(qs[0, hk, s], want, rtol=0, atol=1e-9)
+
+
+@pytest.mark.parametrize("seed", [0, 1])
+def test_permute_segmented_brute_force(seed):
+    """Per query segment s: every key segment before s is the unique stable
+    descending order of its keys' scores against s's representative query
+    (brute-force enumeration); key segments from s on keep natural order."""
+    B, Hq, Hkv, N, d, blk, seg = 1, 2, 1, 32, 4, 2, 8
+    Q = synth.random_lattice((B, Hq, N, d), seed, 1.0)
+    K = synth.random_lattice((B, Hkv, N, d), seed + 5, 1.0)
+    K[0, 0, 3] = K[0, 0, 5]                          # a tie inside key segment 0
+    perm = oracle.permute_segmented(Q, K, blk, seg)
+    for s in range(N // seg):
+        qs = Q[0, :, s * seg:(s + 1) * seg].astype(np.float64).reshape(-1, d).sum(axis=0)
+        for j in range(N // seg):
+            got = perm[0, 0, s, j * seg:(j + 1) * seg]
+            if j >= s:
+                assert got.tolist() == list(range(j * seg, (j + 1) * seg))
+                continue
+            sc = [float(K[0, 0, j * seg + x].astype(np.float64) @ qs) for x in range(seg)]
+            ref = _brute_force_segment_order(sc)
+            assert got.tolist() == [j * seg + x for x in ref], (s, j)
+
+
+def test_segmented_permutation_reduces_to_shared_one():
+    """When every segment has the same representative query, each query
+    segment's permutation of its prefix equals the shared permutation
+    sorted by that query."""
+    B, Hq, Hkv, N, d, blk, seg = 1, 2, 1, 64, 8, 8, 16
+    Q = np.zeros((B, Hq, N, d), np.float32)
+    base = synth.random_lattice((B, Hq, seg, d), 3, 1.0)
+    for s in range(N // seg):
+        Q[:, :, s * seg:(s + 1) * seg] = base
+    K = synth.random_lattice((B, Hkv, N, d), 4, 1.0)
+    perm = oracle.permute_segmented(Q, K, blk, seg)
+    qs = oracle.segment_queries(Q, Hkv, seg)[:, :, 0]
+    shared = oracle.sort_segments(oracle.key_scores(qs, K), seg)
+    for s in range(N // seg):
+        assert np.array_equal(perm[0, 0, s, :s * seg], shared[0, 0, :s * seg])
+
+
+@pytest.mark.parametrize("mode,kw", [("topk", dict(density=0.3)), ("tau", dict(tau=0.9)),
+                                     ("topk", dict(density=0.2, band=20, n_sink=5))])
+def test_segmented_sparse_attention_equals_masked_sdpa(mode, kw):
+    """With one permutation per query segment, every block's key set (built
+    position by position from its segment's permutation) gives the same O
+    as torch fp64 SDPA under that mask; stacking one shared permutation for
+    every segment reproduces the shared-permutation selection exactly."""
+    B, Hq, Hkv, N, d, blk, seg = 1, 4, 2, 128, 16, 8, 32
+    Q, K, V = _small(B, Hq, Hkv, N, d, seed=9, scale=2.0)
+    n_sink = kw.get("n_sink", 0)
+    perm4 = oracle.permute_segmented(Q, K, blk, seg, n_sink)
+    counts, lists = oracle.select(Q, K, perm4, blk, seg, mode, **kw)
+    O, L = oracle.attn(Q, K, V, perm4, lists, blk, seg)
+    G = Hq // Hkv
+    for h in range(Hq):
+        mask = np.zeros((N, N), bool)
+        for q in range(N):
+            i = q // blk
+            s = i * blk // seg
+            mask[q, s * seg:q + 1] = True
+            for pb in lists[(0, h, i)]:
+                mask[q, perm4[0, h // G, s, pb * blk:(pb + 1) * blk]] = True
+        assert not np.any(np.triu(mask, 1))
+        ref = _sdpa(Q[0, h], K[0, h // G], V[0, h // G], mask=mask)
+        assert np.max(np.abs(O[0, h] - ref)) < 1e-12
+    perm3 = oracle.permute(Q, K, blk, seg, n_sink)
+    stacked = np.repeat(perm3[:, :, None, :], N // seg, axis=2)
+    c3, l3 = oracle.select(Q, K, perm3, blk, seg, mode, **kw)
+    c4, l4 = oracle.select(Q, K, stacked, blk, seg, mode, **kw)
+    assert np.array_equal(c3, c4)
+    assert all(np.array_equal(l3[k], l4[k]) for k in l3)
