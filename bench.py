@@ -65,7 +65,8 @@ def selection_label(w) -> str:
     if w.mode == "gate":
         return f"all earlier blocks, block-max gate calibrated to keep {w.gate_keep} tiles"
     if w.stop_tau > 0:
-        return f"topk density={w.density} in descending block score, early stop at gain < {w.stop_tau}"
+        return (f"topk density={w.density} in descending block score, early stop at gain < {w.stop_tau}"
+                + (", one key permutation per query segment" if w.perm_per_segment else ""))
     sel = f"topk density={w.density}" if w.mode == "topk" else f"tau={w.tau}"
     return sel + (f" band={w.band}" if w.band else "") + (f" n_sink={w.n_sink}" if w.n_sink else "")
 
@@ -154,9 +155,13 @@ def oracle_baseline(w, Q, K, V, budget_s: float = 20.0, n_blocks: int = 48):
         thr = np.load(os.path.join(ROOT, "tests", "golden", f"gate_thr_{w.name}.npy")).astype(np.float64)
     else:
         t0 = time.perf_counter()
-        perm1 = oracle.permute(Q[:, :w.G], K[:, :1], w.blk, w.seg, w.n_sink)
+        if w.perm_per_segment:
+            perm1 = oracle.permute_segmented(Q[:, :w.G], K[:, :1], w.blk, w.seg, w.n_sink)
+            perm = np.zeros((w.B, w.Hkv) + perm1.shape[2:], np.int32)
+        else:
+            perm1 = oracle.permute(Q[:, :w.G], K[:, :1], w.blk, w.seg, w.n_sink)
+            perm = np.zeros((w.B, w.Hkv, w.N), np.int32)
         t_perm = (time.perf_counter() - t0) * w.B * w.Hkv
-        perm = np.zeros((w.B, w.Hkv, w.N), np.int32)
         perm[:, 0] = perm1[:, 0]
         t0 = time.perf_counter()
         counts, lists = oracle.select(Q, K, perm, w.blk, w.seg, w.mode, density=w.density, tau=w.tau,
@@ -227,13 +232,18 @@ def run_pbs(args):
     s = torch.cuda.current_stream()
     dt = w.tau if w.mode == "tau" else w.density
     cap = max(1, pbs.select_capacity(w.N, w.blk, w.seg, w.mode, dt, w.band, w.n_sink))
-    perm = torch.empty((w.B, w.Hkv, w.N), dtype=torch.int32, device=dev)
+    segperm = w.perm_per_segment       # one key permutation per query segment
+    nseg = (w.N + w.seg - 1) // w.seg
+    perm = torch.empty((w.B, w.Hkv, nseg, w.N) if segperm else (w.B, w.Hkv, w.N), dtype=torch.int32, device=dev)
     counts = torch.empty((w.B, w.Hq, w.nb), dtype=torch.int32, device=dev)
     idx = torch.empty((w.B, w.Hq, w.nb, cap), dtype=torch.int32, device=dev)
     O = torch.empty_like(Q)
     lse = torch.empty((w.B, w.Hq, w.N), dtype=torch.float32, device=dev)
-    ws_p = torch.empty(pbs.workspace_size(pbs.PBS_OP_PERMUTE, Q, K, w.blk, w.seg) + 256, dtype=torch.uint8, device=dev)
-    ws_s = torch.empty(pbs.workspace_size(pbs.PBS_OP_SELECT, Q, K, w.blk, w.seg) + 256, dtype=torch.uint8, device=dev)
+    op_p = pbs.PBS_OP_PERMUTE_SEGMENTED if segperm else pbs.PBS_OP_PERMUTE
+    op_s = pbs.PBS_OP_SELECT_SEGMENTED if segperm else pbs.PBS_OP_SELECT
+    ws_p = torch.empty(pbs.workspace_size(op_p, Q, K, w.blk, w.seg) + 256, dtype=torch.uint8, device=dev)
+    ws_s = torch.empty(pbs.workspace_size(op_s, Q, K, w.blk, w.seg) + 256, dtype=torch.uint8, device=dev)
+    permute = pbs.pbs_permute_segmented if segperm else pbs.pbs_permute
     stats = torch.zeros(2, dtype=torch.int64, device=dev)
     launches_per_step = 6   # 2 permute + 3 select + 1 attention kernels
     # Block-max gating workloads: no permutation or selection step; every
@@ -258,7 +268,7 @@ def run_pbs(args):
         if record:
             e[0].record(s)
         if not gate:
-            pbs.pbs_permute(Q, K, w.blk, w.seg, w.n_sink, perm=perm, ws=ws_p)
+            permute(Q, K, w.blk, w.seg, w.n_sink, perm=perm, ws=ws_p)
         if record:
             e[1].record(s)
         if not gate:
@@ -384,7 +394,7 @@ def run_pbs(args):
             Kd.copy_(Kh, non_blocking=True)
             Vd.copy_(Vh, non_blocking=True)
             if not gate:
-                pbs.pbs_permute(Qd, Kd, w.blk, w.seg, w.n_sink, perm=perm, ws=ws_p)
+                permute(Qd, Kd, w.blk, w.seg, w.n_sink, perm=perm, ws=ws_p)
                 pbs.pbs_select(Qd, Kd, perm, w.blk, w.seg, w.mode, dt, w.band, w.n_sink, cap=cap,
                                counts=counts, idx=idx, ws=ws_s, score_order=early)
             if early:

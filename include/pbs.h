@@ -80,10 +80,14 @@ typedef enum pbs_status {
   PBS_ERR_DEVICE_CHECK = -6   /* device: an index failed its bounds check   */
 } pbs_status;
 
-enum { PBS_OP_PERMUTE = 0, PBS_OP_SELECT = 1, PBS_OP_ATTN = 2 };
+enum { PBS_OP_PERMUTE = 0, PBS_OP_SELECT = 1, PBS_OP_ATTN = 2, PBS_OP_PERMUTE_SEGMENTED = 3,
+       PBS_OP_SELECT_SEGMENTED = 4 };
 enum { PBS_SELECT_TOPK = 0, PBS_SELECT_TAU = 1 };
-/* OR-ed into pbs_select's mode: write lists in visiting order (see there). */
-enum { PBS_SELECT_SCORE_ORDER = 0x10 };
+/* OR-ed into pbs_select's mode: write lists in visiting order, and/or read
+ * one permutation per query segment (see there). */
+enum { PBS_SELECT_SCORE_ORDER = 0x10, PBS_SELECT_PERM_PER_SEGMENT = 0x20 };
+/* pbs_attn_fwd_ex flags. */
+enum { PBS_ATTN_EARLY_STOP = 1, PBS_ATTN_PERM_PER_SEGMENT = 2 };
 
 /* Bytes of workspace the given op needs for these shapes (0 if none).
  * Q and K may not be NULL; only their shapes are read.                     */
@@ -119,6 +123,25 @@ int pbs_permute(const pbs_tensor* Q, const pbs_tensor* K, int blk, int seg,
 int pbs_permute_noalloc(const pbs_tensor* Q, const pbs_tensor* K, int blk, int seg,
                         int n_sink, int32_t* perm, void* stream);
 
+/* pbs_permute_segmented: one key permutation per query segment,
+ * perm[b, hkv, s, p] = original key position at logical position p as read
+ * by query segment s ("S2O ...", Technical Summary, 1. Online Permutation
+ * via Index-Driven Loading: historical keys are scored against a
+ * representative query of the segment, prefix keys only).
+ *   1. qbar_s[b,hkv] = sum of every query row of segment s of every query
+ *      head of KV head hkv's group (fp64);
+ *   2. score s_j = qbar_s . K[b,hkv,j] (fp64); positions j < n_sink get +inf;
+ *   3. each key segment t < s is sorted by descending score, equal scores by
+ *      ascending position; key segments t >= s keep their natural order.
+ * perm: device int32 [B, Hkv, nseg, N] with nseg = ceil(N / seg).
+ * ws: pbs_workspace_size(PBS_OP_PERMUTE_SEGMENTED, ...) bytes.
+ * Select with mode | PBS_SELECT_PERM_PER_SEGMENT and attend with
+ * PBS_ATTN_PERM_PER_SEGMENT to use it; each query block then reads its
+ * segment's permutation.  Fp64 keeps the order exact on inputs whose values
+ * are multiples of 1/8 (any bf16 input sorts by its fp64-rounded scores). */
+int pbs_permute_segmented(const pbs_tensor* Q, const pbs_tensor* K, int blk, int seg, int n_sink,
+                          int32_t* perm, void* ws, size_t ws_bytes, void* stream);
+
 /* Upper bound on the list length pbs_select can produce for these settings
  * (host-only arithmetic).  Pass at least this as `cap`.                    */
 int pbs_select_capacity(int64_t N, int blk, int seg, int mode,
@@ -140,6 +163,10 @@ int pbs_select_capacity(int64_t N, int blk, int seg, int mode,
  *     mass (own segment included) is below tau.  tau >= 1 lists all.
  * counts: device int32 [B, Hq, N/blk]; idx: device int32
  * [B, Hq, N/blk, cap]; entries at and after counts[...] are unspecified.
+ * With mode | PBS_SELECT_PERM_PER_SEGMENT, perm is [B, Hkv, nseg, N] from
+ * pbs_permute_segmented and block i pools and scores the keys of its own
+ * segment's permutation; ws then needs pbs_workspace_size(
+ * PBS_OP_SELECT_SEGMENTED, ...) bytes.
  * With mode | PBS_SELECT_SCORE_ORDER the same blocks are listed in visiting
  * order instead of ascending: the forced blocks first (ascending), then the
  * others by descending S, ties to the lower pb -- the descending estimated
@@ -192,6 +219,17 @@ int pbs_attn_fwd_early_stop(const pbs_tensor* Q, const pbs_tensor* K, const pbs_
                             const int32_t* perm, const int32_t* counts, const int32_t* idx,
                             int cap, int blk, int seg, float stop_tau, float softmax_scale,
                             pbs_tensor* O, float* lse, long long* stats, void* stream);
+
+/* pbs_attn_fwd_ex: pbs_attn_fwd and pbs_attn_fwd_early_stop in one call.
+ *   flags: PBS_ATTN_EARLY_STOP -- lists in visiting order, stop_tau as for
+ *            pbs_attn_fwd_early_stop (gate_thr must then be NULL);
+ *          PBS_ATTN_PERM_PER_SEGMENT -- perm is [B, Hkv, nseg, N] from
+ *            pbs_permute_segmented and each query block reads its segment's.
+ *   Other arguments as for pbs_attn_fwd; unknown flags are rejected.       */
+int pbs_attn_fwd_ex(const pbs_tensor* Q, const pbs_tensor* K, const pbs_tensor* V, const int32_t* perm,
+                    const int32_t* counts, const int32_t* idx, int cap, int blk, int seg, unsigned flags,
+                    const float* gate_thr, float stop_tau, float softmax_scale, pbs_tensor* O, float* lse,
+                    long long* stats, void* stream);
 
 /* Synchronises `stream`, then returns and clears the sticky device error
  * word of the current device (PBS_OK if no device-side check failed).      */

@@ -18,13 +18,15 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libpbs.so")
 
-PBS_OP_PERMUTE, PBS_OP_SELECT, PBS_OP_ATTN = 0, 1, 2
+PBS_OP_PERMUTE, PBS_OP_SELECT, PBS_OP_ATTN, PBS_OP_PERMUTE_SEGMENTED, PBS_OP_SELECT_SEGMENTED = 0, 1, 2, 3, 4
 PBS_SELECT_TOPK, PBS_SELECT_TAU = 0, 1
-PBS_SELECT_SCORE_ORDER = 0x10
+PBS_SELECT_SCORE_ORDER, PBS_SELECT_PERM_PER_SEGMENT = 0x10, 0x20
+PBS_ATTN_EARLY_STOP, PBS_ATTN_PERM_PER_SEGMENT = 1, 2
 STATUS = {0: "PBS_OK", -1: "PBS_ERR_INVALID_ARG", -2: "PBS_ERR_UNSUPPORTED", -3: "PBS_ERR_CAPACITY",
           -4: "PBS_ERR_CUDA", -5: "PBS_ERR_TIMEOUT", -6: "PBS_ERR_DEVICE_CHECK"}
-EXPORTS = ("pbs_workspace_size", "pbs_permute", "pbs_select_capacity", "pbs_select", "pbs_attn_fwd",
-           "pbs_attn_fwd_early_stop", "pbs_check_device", "pbs_get_last_error", "pbs_version")
+EXPORTS = ("pbs_workspace_size", "pbs_permute", "pbs_permute_segmented", "pbs_select_capacity", "pbs_select",
+           "pbs_attn_fwd", "pbs_attn_fwd_early_stop", "pbs_attn_fwd_ex", "pbs_check_device",
+           "pbs_get_last_error", "pbs_version")
 
 
 class PbsError(RuntimeError):
@@ -56,6 +58,11 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.pbs_workspace_size.restype = sz
     lib.pbs_permute.argtypes = [P, P, i32, i32, i32, vp, vp, sz, vp]
     lib.pbs_permute.restype = i32
+    lib.pbs_permute_segmented.argtypes = [P, P, i32, i32, i32, vp, vp, sz, vp]
+    lib.pbs_permute_segmented.restype = i32
+    lib.pbs_attn_fwd_ex.argtypes = [P, P, P, vp, vp, vp, i32, i32, i32, ctypes.c_uint, vp, ctypes.c_float,
+                                    ctypes.c_float, P, vp, vp, vp]
+    lib.pbs_attn_fwd_ex.restype = i32
     lib.pbs_select_capacity.argtypes = [i64, i32, i32, i32, dbl, i32, i32]
     lib.pbs_select_capacity.restype = i32
     lib.pbs_select.argtypes = [P, P, vp, i32, i32, i32, dbl, i32, i32, vp, vp, i32, vp, sz, vp]
@@ -148,6 +155,26 @@ def pbs_permute(Q: torch.Tensor, K: torch.Tensor, blk: int, seg: int, n_sink: in
     return perm
 
 
+def pbs_permute_segmented(Q: torch.Tensor, K: torch.Tensor, blk: int, seg: int, n_sink: int = 0,
+                          perm: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
+                          stream=None) -> torch.Tensor:
+    """perm [B, Hkv, nseg, N] int32: one permutation per query segment (its
+    history's key segments sorted by the segment's pooled query)."""
+    lib = load()
+    q, k = describe(Q), describe(K)
+    B, Hkv, N, _ = K.shape
+    nseg = (N + seg - 1) // seg
+    if perm is None:
+        perm = torch.empty((B, Hkv, nseg, N), dtype=torch.int32, device=K.device)
+    if ws is None:
+        ws = _workspace(lib.pbs_workspace_size(PBS_OP_PERMUTE_SEGMENTED, ctypes.byref(q), ctypes.byref(k), blk, seg),
+                        K.device)
+    wp, wn = _aligned(ws)
+    _check(lib.pbs_permute_segmented(ctypes.byref(q), ctypes.byref(k), blk, seg, n_sink, perm.data_ptr(), wp, wn,
+                                     _stream(stream)))
+    return perm
+
+
 def pbs_select(Q: torch.Tensor, K: torch.Tensor, perm: torch.Tensor, blk: int, seg: int,
                mode: str = "topk", density_or_tau: float = 1.0, band: int = 0, n_sink: int = 0,
                cap: Optional[int] = None, counts: Optional[torch.Tensor] = None,
@@ -163,6 +190,10 @@ def pbs_select(Q: torch.Tensor, K: torch.Tensor, perm: torch.Tensor, blk: int, s
     m = PBS_SELECT_TAU if mode == "tau" else PBS_SELECT_TOPK
     if score_order:
         m |= PBS_SELECT_SCORE_ORDER
+    op = PBS_OP_SELECT
+    if perm.dim() == 4:                      # one permutation per query segment
+        m |= PBS_SELECT_PERM_PER_SEGMENT
+        op = PBS_OP_SELECT_SEGMENTED
     if cap is None:
         cap = max(1, select_capacity(N, blk, seg, mode, density_or_tau, band, n_sink))
     if counts is None:
@@ -170,7 +201,7 @@ def pbs_select(Q: torch.Tensor, K: torch.Tensor, perm: torch.Tensor, blk: int, s
     if idx is None:
         idx = torch.empty((B, Hq, nb, cap), dtype=torch.int32, device=Q.device)
     if ws is None:
-        ws = _workspace(lib.pbs_workspace_size(PBS_OP_SELECT, ctypes.byref(q), ctypes.byref(k), blk, seg), Q.device)
+        ws = _workspace(lib.pbs_workspace_size(op, ctypes.byref(q), ctypes.byref(k), blk, seg), Q.device)
     wp, wn = _aligned(ws)
     _check(lib.pbs_select(ctypes.byref(q), ctypes.byref(k), perm.data_ptr(), blk, seg, m, float(density_or_tau),
                           band, n_sink, counts.data_ptr(), idx.data_ptr(), cap, wp, wn, _stream(stream)))
@@ -197,6 +228,12 @@ def pbs_attn_fwd(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, perm: torch.
     if stats is not None and stats.dtype != torch.int64:
         raise TypeError("stats must be int64")
     q, k, v, o = describe(Q), describe(K), describe(V), describe(out)
+    if perm.dim() == 4:                      # one permutation per query segment
+        _check(lib.pbs_attn_fwd_ex(ctypes.byref(q), ctypes.byref(k), ctypes.byref(v), perm.data_ptr(),
+                                   counts.data_ptr(), idx.data_ptr(), idx.shape[-1], blk, seg,
+                                   PBS_ATTN_PERM_PER_SEGMENT, _ptr(gate_thr), 0.0, float(softmax_scale),
+                                   ctypes.byref(o), _ptr(lse), _ptr(stats), _stream(stream)))
+        return out, lse
     _check(lib.pbs_attn_fwd(ctypes.byref(q), ctypes.byref(k), ctypes.byref(v), perm.data_ptr(),
                             counts.data_ptr(), idx.data_ptr(), idx.shape[-1], blk, seg, _ptr(gate_thr),
                             float(softmax_scale), ctypes.byref(o), _ptr(lse), _ptr(stats), None, 0,
@@ -223,6 +260,13 @@ def pbs_attn_fwd_early_stop(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, p
     if stats is not None and stats.dtype != torch.int64:
         raise TypeError("stats must be int64")
     q, k, v, o = describe(Q), describe(K), describe(V), describe(out)
+    if perm.dim() == 4:                      # one permutation per query segment
+        _check(lib.pbs_attn_fwd_ex(ctypes.byref(q), ctypes.byref(k), ctypes.byref(v), perm.data_ptr(),
+                                   counts.data_ptr(), idx.data_ptr(), idx.shape[-1], blk, seg,
+                                   PBS_ATTN_EARLY_STOP | PBS_ATTN_PERM_PER_SEGMENT, None, float(stop_tau),
+                                   float(softmax_scale), ctypes.byref(o), _ptr(lse), _ptr(stats),
+                                   _stream(stream)))
+        return out, lse
     _check(lib.pbs_attn_fwd_early_stop(ctypes.byref(q), ctypes.byref(k), ctypes.byref(v), perm.data_ptr(),
                                        counts.data_ptr(), idx.data_ptr(), idx.shape[-1], blk, seg,
                                        float(stop_tau), float(softmax_scale), ctypes.byref(o), _ptr(lse),

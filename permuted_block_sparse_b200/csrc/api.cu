@@ -89,14 +89,16 @@ struct SelectWs {
   size_t qbar, kperm, knat, inv, scores, total;
 };
 
-SelectWs select_ws(const pbs::TensorDesc& Q, const pbs::TensorDesc& K, int blk) {
+// perm_nseg permutations per KV head (1, or one per query segment).
+SelectWs select_ws(const pbs::TensorDesc& Q, const pbs::TensorDesc& K, int blk, int64_t perm_nseg = 1) {
   const size_t nb = static_cast<size_t>(Q.N / blk);
+  const size_t np = static_cast<size_t>(perm_nseg);
   SelectWs w;
   w.qbar = 0;
   w.kperm = w.qbar + align256(static_cast<size_t>(Q.B * Q.H) * nb * Q.D * 4);
-  w.knat = w.kperm + align256(static_cast<size_t>(K.B * K.H) * nb * K.D * 4);
+  w.knat = w.kperm + align256(static_cast<size_t>(K.B * K.H) * np * nb * K.D * 4);
   w.inv = w.knat + align256(static_cast<size_t>(K.B * K.H) * nb * K.D * 4);
-  w.scores = w.inv + align256(static_cast<size_t>(K.B * K.H) * K.N * 4);
+  w.scores = w.inv + align256(static_cast<size_t>(K.B * K.H) * np * K.N * 4);
   w.total = w.scores + align256(static_cast<size_t>(Q.B * Q.H) * nb * nb * 4);
   return w;
 }
@@ -136,8 +138,8 @@ int api_validate_permute(const pbs_tensor* Qt, const pbs_tensor* Kt, int blk, in
 namespace {
 int attn_common(const pbs_tensor* Qt, const pbs_tensor* Kt, const pbs_tensor* Vt,
                 const int32_t* perm, const int32_t* counts, const int32_t* idx, int cap, int blk,
-                int seg, const float* gate_thr, int early_stop, float stop_tau, float softmax_scale,
-                pbs_tensor* Ot, float* lse, long long* stats, void* stream) {
+                int seg, const float* gate_thr, int early_stop, float stop_tau, int per_segment,
+                float softmax_scale, pbs_tensor* Ot, float* lse, long long* stats, void* stream) {
   pbs::TensorDesc Q, K, V, O;
   int rc;
   if ((rc = check_tensor(Qt, "Q", &Q)) || (rc = check_tensor(Kt, "K", &K)) ||
@@ -170,6 +172,7 @@ int attn_common(const pbs_tensor* Qt, const pbs_tensor* Kt, const pbs_tensor* Vt
   p.gate_thr = gate_thr;
   p.early_stop = early_stop;
   p.stop_tau = stop_tau;
+  p.perm_nseg = per_segment ? static_cast<int>((Q.N + seg - 1) / seg) : 1;
   p.scale_log2 = softmax_scale * 1.4426950408889634f;
   p.lse = lse;
   p.stats = stats;
@@ -187,18 +190,36 @@ const char* pbs_version(void) { return "pbs 0.1 (sm_100a)"; }
 const char* pbs_get_last_error(void) { return g_last_error.c_str(); }
 
 size_t pbs_workspace_size(int op, const pbs_tensor* Qt, const pbs_tensor* Kt, int blk, int seg) {
-  (void)seg;
   pbs::TensorDesc Q, K;
   if (check_tensor(Qt, "Q", &Q) || check_tensor(Kt, "K", &K)) return 0;
   if (blk != 64 && blk != 128) return 0;
+  const int64_t nseg = seg > 0 ? (K.N + seg - 1) / seg : 0;
   switch (op) {
     case PBS_OP_PERMUTE:
       return align256(static_cast<size_t>(K.B * K.H * K.D) * 4);
     case PBS_OP_SELECT:
       return select_ws(Q, K, blk).total;
+    case PBS_OP_PERMUTE_SEGMENTED:
+      return nseg > 0 ? align256(static_cast<size_t>(K.B * K.H * nseg * K.D) * 8) : 0;
+    case PBS_OP_SELECT_SEGMENTED:
+      return nseg > 0 ? select_ws(Q, K, blk, nseg).total : 0;
     default:
       return 0;
   }
+}
+
+int pbs_permute_segmented(const pbs_tensor* Qt, const pbs_tensor* Kt, int blk, int seg, int n_sink,
+                          int32_t* perm, void* ws, size_t ws_bytes, void* stream) {
+  pbs::TensorDesc Q, K;
+  int rc;
+  if ((rc = pbs::api_validate_permute(Qt, Kt, blk, seg, n_sink, perm, &Q, &K))) return rc;
+  const int64_t nseg = (K.N + seg - 1) / seg;
+  if (nseg > 65535 || K.B * K.H > 65535) return fail(PBS_ERR_UNSUPPORTED, "too many segments or heads");
+  if ((rc = check_ws(ws, ws_bytes, align256(static_cast<size_t>(K.B * K.H * nseg * K.D) * 8)))) return rc;
+  cudaError_t e = pbs::launch_permute_segmented(Q, K, seg, n_sink, static_cast<double*>(ws), perm,
+                                                static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "permute_segmented launch");
+  return ok();
 }
 
 int pbs_permute(const pbs_tensor* Qt, const pbs_tensor* Kt, int blk, int seg, int n_sink,
@@ -226,7 +247,7 @@ int pbs_select_capacity(int64_t N, int blk, int seg, int mode, double density_or
                         int n_sink) {
   if (blk <= 0 || seg < blk || seg % blk || N <= 0 || N % blk)
     return fail(PBS_ERR_INVALID_ARG, "bad geometry for capacity");
-  mode &= ~PBS_SELECT_SCORE_ORDER;
+  mode &= ~(PBS_SELECT_SCORE_ORDER | PBS_SELECT_PERM_PER_SEGMENT);
   const int64_t nb = N / blk, spb = seg / blk;
   int64_t best = 0;
   const int64_t r = rho_permille(density_or_tau);
@@ -258,7 +279,8 @@ int pbs_select(const pbs_tensor* Qt, const pbs_tensor* Kt, const int32_t* perm, 
   if ((rc = check_geometry(Q, K, blk, seg))) return rc;
   if (!perm || !counts || !idx) return fail(PBS_ERR_INVALID_ARG, "perm, counts or idx is null");
   const int score_order = (mode & PBS_SELECT_SCORE_ORDER) ? 1 : 0;
-  mode &= ~PBS_SELECT_SCORE_ORDER;
+  const int per_segment = (mode & PBS_SELECT_PERM_PER_SEGMENT) ? 1 : 0;
+  mode &= ~(PBS_SELECT_SCORE_ORDER | PBS_SELECT_PERM_PER_SEGMENT);
   if (mode != PBS_SELECT_TOPK && mode != PBS_SELECT_TAU)
     return fail(PBS_ERR_INVALID_ARG, "mode %d unknown", mode);
   if (!(density_or_tau >= 0.0) || (mode == PBS_SELECT_TOPK && density_or_tau > 1.0))
@@ -269,7 +291,8 @@ int pbs_select(const pbs_tensor* Qt, const pbs_tensor* Kt, const int32_t* perm, 
   const int need_cap = pbs_select_capacity(Q.N, blk, seg, mode, density_or_tau, band, n_sink);
   if (cap < need_cap || cap < 1)
     return fail(PBS_ERR_CAPACITY, "cap %d < required %d", cap, std::max(need_cap, 1));
-  const SelectWs w = select_ws(Q, K, blk);
+  const int64_t perm_nseg = per_segment ? (Q.N + seg - 1) / seg : 1;
+  const SelectWs w = select_ws(Q, K, blk, perm_nseg);
   if ((rc = check_ws(ws, ws_bytes, w.total))) return rc;
   int* err = device_error_word();
   if (!err) return fail(PBS_ERR_CUDA, "cannot resolve the device error word");
@@ -282,7 +305,8 @@ int pbs_select(const pbs_tensor* Qt, const pbs_tensor* Kt, const int32_t* perm, 
   float* scores = reinterpret_cast<float*>(base + w.scores);
   cudaError_t e = pbs::launch_pool_query_blocks(Q, blk, qbar, s);
   if (e != cudaSuccess) return cuda_fail(e, "pool_query_blocks launch");
-  e = pbs::launch_pool_key_blocks(K, perm, blk, seg, mode == PBS_SELECT_TAU, kperm, knat, inv, err, s);
+  e = pbs::launch_pool_key_blocks(K, perm, static_cast<int>(perm_nseg), blk, seg, mode == PBS_SELECT_TAU, kperm,
+                                  knat, inv, err, s);
   if (e != cudaSuccess) return cuda_fail(e, "pool_key_blocks launch");
   pbs::SelectParams p;
   p.B = static_cast<int>(Q.B);
@@ -294,6 +318,7 @@ int pbs_select(const pbs_tensor* Qt, const pbs_tensor* Kt, const int32_t* perm, 
   p.nb = static_cast<int>(nb);
   p.mode = mode;
   p.score_order = score_order;
+  p.perm_nseg = static_cast<int>(perm_nseg);
   p.band = band;
   p.n_sink = n_sink;
   p.cap = cap;
@@ -312,7 +337,7 @@ int pbs_attn_fwd(const pbs_tensor* Qt, const pbs_tensor* Kt, const pbs_tensor* V
                  long long* stats, void* ws, size_t ws_bytes, void* stream) {
   (void)ws;
   (void)ws_bytes;
-  return attn_common(Qt, Kt, Vt, perm, counts, idx, cap, blk, seg, gate_thr, 0, 0.0f, softmax_scale,
+  return attn_common(Qt, Kt, Vt, perm, counts, idx, cap, blk, seg, gate_thr, 0, 0.0f, 0, softmax_scale,
                      Ot, lse, stats, stream);
 }
 
@@ -322,8 +347,24 @@ int pbs_attn_fwd_early_stop(const pbs_tensor* Qt, const pbs_tensor* Kt, const pb
                             pbs_tensor* Ot, float* lse, long long* stats, void* stream) {
   if (!(stop_tau >= 0.0f) || !std::isfinite(stop_tau))
     return fail(PBS_ERR_INVALID_ARG, "stop_tau must be finite and >= 0");
-  return attn_common(Qt, Kt, Vt, perm, counts, idx, cap, blk, seg, nullptr, 1, stop_tau, softmax_scale,
+  return attn_common(Qt, Kt, Vt, perm, counts, idx, cap, blk, seg, nullptr, 1, stop_tau, 0, softmax_scale,
                      Ot, lse, stats, stream);
+}
+
+int pbs_attn_fwd_ex(const pbs_tensor* Qt, const pbs_tensor* Kt, const pbs_tensor* Vt, const int32_t* perm,
+                    const int32_t* counts, const int32_t* idx, int cap, int blk, int seg, unsigned flags,
+                    const float* gate_thr, float stop_tau, float softmax_scale, pbs_tensor* Ot, float* lse,
+                    long long* stats, void* stream) {
+  if (flags & ~static_cast<unsigned>(PBS_ATTN_EARLY_STOP | PBS_ATTN_PERM_PER_SEGMENT))
+    return fail(PBS_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
+  const int early = (flags & PBS_ATTN_EARLY_STOP) ? 1 : 0;
+  if (early) {
+    if (gate_thr) return fail(PBS_ERR_UNSUPPORTED, "early stopping with a gate is not supported");
+    if (!(stop_tau >= 0.0f) || !std::isfinite(stop_tau))
+      return fail(PBS_ERR_INVALID_ARG, "stop_tau must be finite and >= 0");
+  }
+  return attn_common(Qt, Kt, Vt, perm, counts, idx, cap, blk, seg, gate_thr, early, early ? stop_tau : 0.0f,
+                     (flags & PBS_ATTN_PERM_PER_SEGMENT) ? 1 : 0, softmax_scale, Ot, lse, stats, stream);
 }
 
 int pbs_check_device(void* stream) {

@@ -266,7 +266,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
     const int pt = tid - 32;
     const __nv_bfloat16* kb = static_cast<const __nv_bfloat16*>(p.K.ptr) + b * p.K.sB + hk * p.K.sH;
     const __nv_bfloat16* vb = static_cast<const __nv_bfloat16*>(p.V.ptr) + b * p.V.sB + hk * p.V.sH;
-    const int32_t* prow = p.perm + (static_cast<int64_t>(b) * p.K.H + hk) * N;
+    // the key permutation this query block reads: its KV head's, or with one
+    // permutation per query segment, its segment's
+    const int32_t* prow =
+        p.perm + ((static_cast<int64_t>(b) * p.K.H + hk) * p.perm_nseg + (p.perm_nseg > 1 ? s : 0)) * N;
     constexpr int CH = D / 8;
     // Tile gathers: thread pt always copies 16-byte chunk c of rows r0,
     // r0 + RPP, r0 + 2 RPP, ... (RPP rows per pass of the 96 threads).  A

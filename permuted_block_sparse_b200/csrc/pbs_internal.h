@@ -22,12 +22,15 @@ cudaError_t launch_score_sort(const TensorDesc& K, int seg, int n_sink, const fl
 
 // pbs_select launchers ----------------------------------------------------
 cudaError_t launch_pool_query_blocks(const TensorDesc& Q, int blk, float* qbar, cudaStream_t s);
-cudaError_t launch_pool_key_blocks(const TensorDesc& K, const int32_t* perm, int blk, int seg,
-                                   bool natural, float* kbar_perm, float* kbar_nat,
+cudaError_t launch_pool_key_blocks(const TensorDesc& K, const int32_t* perm, int perm_nseg, int blk,
+                                   int seg, bool natural, float* kbar_perm, float* kbar_nat,
                                    int32_t* inv, int* err, cudaStream_t s);
+cudaError_t launch_permute_segmented(const TensorDesc& Q, const TensorDesc& K, int seg, int n_sink,
+                                     double* qs, int32_t* perm, cudaStream_t s);
 struct SelectParams {
   int B, Hq, Hkv, D, blk, seg, nb, mode, band, n_sink, cap;
   int score_order;        // lists in visiting order instead of ascending
+  int perm_nseg;          // 1: one permutation per KV head; else one per query segment
   int64_t N;
   int64_t rho_permille;   // top-k density in per-mille
   double tau;
@@ -54,6 +57,7 @@ struct AttnParams {
   int cap, blk, seg, nb, G;
   const float* gate_thr;
   int early_stop;         // S2O early stopping: lists in visiting order, cut by stop_tau
+  int perm_nseg;          // 1: one permutation per KV head; else one per query segment
   float stop_tau;
   float scale_log2;       // softmax scale * log2(e)
   float* lse;

@@ -55,10 +55,14 @@ __global__ void __launch_bounds__(256) pool_query_blocks_kernel(
 // optionally Kbar_nat = sum of rows pb*blk+r; and the inverse permutation
 // inv[perm[p]] = p.  A perm entry outside its segment sets the error word
 // and is skipped.
+// perm, inv and kbar_perm rows of consecutive (b, h) are perm_stride elements
+// (inv likewise) and kbar_stride blocks apart: one permutation per KV head,
+// or one per (KV head, query segment) launched segment by segment.
 __global__ void __launch_bounds__(256) pool_key_blocks_kernel(
     const __nv_bfloat16* __restrict__ K, int64_t sB, int64_t sH, int64_t sN, int64_t N, int D,
-    int blk, int seg, const int32_t* __restrict__ perm, int natural, float* __restrict__ kbar_perm,
-    float* __restrict__ kbar_nat, int32_t* __restrict__ inv, int* err) {
+    int blk, int seg, const int32_t* __restrict__ perm, int64_t perm_stride, int natural,
+    float* __restrict__ kbar_perm, int64_t kbar_stride, float* __restrict__ kbar_nat,
+    int32_t* __restrict__ inv, int* err) {
   const int pb = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int nb = gridDim.x, H = gridDim.y;
   __shared__ int32_t rows[256];
@@ -66,8 +70,8 @@ __global__ void __launch_bounds__(256) pool_key_blocks_kernel(
   const int64_t p0 = static_cast<int64_t>(pb) * blk;
   const int64_t seg_lo = (p0 / seg) * seg;
   const int64_t seg_hi = min(seg_lo + seg, N);
-  const int32_t* prow = perm + (static_cast<int64_t>(b) * H + h) * N;
-  int32_t* irow = inv + (static_cast<int64_t>(b) * H + h) * N;
+  const int32_t* prow = perm + (static_cast<int64_t>(b) * H + h) * perm_stride;
+  int32_t* irow = inv + (static_cast<int64_t>(b) * H + h) * perm_stride;
   for (int r = threadIdx.x; r < blk; r += blockDim.x) {
     int32_t x = prow[p0 + r];
     if (x < seg_lo || x >= seg_hi) {
@@ -99,14 +103,54 @@ __global__ void __launch_bounds__(256) pool_key_blocks_kernel(
 #pragma unroll
     for (int e = 0; e < 8; ++e) red[threadIdx.x * 8 + e] = acc[e];
     __syncthreads();
-    float* out = pass == 0 ? kbar_perm : kbar_nat;
+    float* out = pass == 0 ? kbar_perm + ((static_cast<int64_t>(b) * H + h) * kbar_stride + pb) * D
+                           : kbar_nat + ((static_cast<int64_t>(b) * H + h) * nb + pb) * D;
     for (int c = threadIdx.x; c < D; c += blockDim.x) {
       const int ch = c / 8, e = c % 8;
       float t = 0.f;
       for (int l = 0; l < lanes; ++l) t += red[(l * nchunk + ch) * 8 + e];
-      out[((static_cast<int64_t>(b) * H + h) * nb + pb) * D + c] = t;
+      out[c] = t;
     }
     __syncthreads();
+  }
+}
+
+// Block scores with one permutation per query segment: S[row, pb] =
+// Qbar[row] . Kbar[s(row), pb] for the row's candidates pb < ncand.  One warp
+// per (b, hq, i) row; each lane takes candidates lane, lane + 32, ... and
+// reads that block's pooled key row as float4s against the row's pooled
+// query held in shared memory.  Exact in fp32 on lattice inputs (every
+// partial sum is a multiple of 2^-6 below 2^18), like the tiled kernel.
+constexpr int kSegScoreWarps = 8;
+__global__ void __launch_bounds__(kSegScoreWarps * 32) block_scores_seg_kernel(
+    SelectParams p, const float* __restrict__ qbar, const float* __restrict__ kbar4,
+    float* __restrict__ scores) {
+  __shared__ __align__(16) float qs[kSegScoreWarps][128];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * kSegScoreWarps + warp;
+  if (row >= static_cast<int64_t>(p.B) * p.Hq * p.nb) return;
+  const int i = static_cast<int>(row % p.nb);
+  const int h = static_cast<int>((row / p.nb) % p.Hq);
+  const int b = static_cast<int>(row / (static_cast<int64_t>(p.nb) * p.Hq));
+  const int hk = h / (p.Hq / p.Hkv);
+  const int spb = p.seg / p.blk;
+  const int s = i / spb, ncand = s * spb;
+  if (ncand == 0) return;
+  for (int c = lane; c < p.D; c += 32) qs[warp][c] = qbar[row * p.D + c];
+  __syncwarp();
+  const float* kb = kbar4 + ((static_cast<int64_t>(b) * p.Hkv + hk) * p.perm_nseg + s) * p.nb * p.D;
+  float* out = scores + row * p.nb;
+  for (int pb = lane; pb < ncand; pb += 32) {
+    const float4* kr = reinterpret_cast<const float4*>(kb + static_cast<int64_t>(pb) * p.D);
+    float acc = 0.f;
+    for (int c = 0; c < p.D / 4; ++c) {
+      const float4 k4 = kr[c];
+      acc = fmaf(qs[warp][4 * c], k4.x, acc);
+      acc = fmaf(qs[warp][4 * c + 1], k4.y, acc);
+      acc = fmaf(qs[warp][4 * c + 2], k4.z, acc);
+      acc = fmaf(qs[warp][4 * c + 3], k4.w, acc);
+    }
+    out[pb] = acc;
   }
 }
 
@@ -251,7 +295,8 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32) select_topk_kernel(
     return;
   }
   const float* S = S_all + row * p.nb;
-  forced_bitmap(p, inv + (static_cast<int64_t>(b) * p.Hkv + hk) * p.N, i, ncand, fbits, lane);
+  forced_bitmap(p, inv + ((static_cast<int64_t>(b) * p.Hkv + hk) * p.perm_nseg + (p.perm_nseg > 1 ? s : 0)) * p.N,
+                i, ncand, fbits, lane);
   const int words = (ncand + 31) >> 5;
   int nf = 0;
   for (int w = lane; w < words; w += 32) nf += __popc(fbits[w]);
@@ -375,7 +420,7 @@ __global__ void __launch_bounds__(kSelThreads) select_tau_kernel(
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   // Forced blocks: sinks and the recent-key band that fall before the own segment.
   const int64_t s_start = static_cast<int64_t>(s) * p.seg;
-  const int32_t* irow = inv + (static_cast<int64_t>(b) * p.Hkv + hk) * p.N;
+  const int32_t* irow = inv + ((static_cast<int64_t>(b) * p.Hkv + hk) * p.perm_nseg + (p.perm_nseg > 1 ? s : 0)) * p.N;
   const int64_t sink_hi = min(static_cast<int64_t>(p.n_sink), s_start);
   for (int64_t pos = threadIdx.x; pos < sink_hi; pos += blockDim.x) {
     const int32_t lp = irow[pos];
@@ -547,23 +592,37 @@ cudaError_t launch_pool_query_blocks(const TensorDesc& Q, int blk, float* qbar, 
   return cudaGetLastError();
 }
 
-cudaError_t launch_pool_key_blocks(const TensorDesc& K, const int32_t* perm, int blk, int seg,
-                                   bool natural, float* kbar_perm, float* kbar_nat, int32_t* inv,
+cudaError_t launch_pool_key_blocks(const TensorDesc& K, const int32_t* perm, int perm_nseg, int blk,
+                                   int seg, bool natural, float* kbar_perm, float* kbar_nat, int32_t* inv,
                                    int* err, cudaStream_t s) {
   dim3 grid(static_cast<unsigned>(K.N / blk), static_cast<unsigned>(K.H), static_cast<unsigned>(K.B));
-  pool_key_blocks_kernel<<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(K.ptr), K.sB,
-                                               K.sH, K.sN, K.N, static_cast<int>(K.D), blk, seg,
-                                               perm, natural ? 1 : 0, kbar_perm, kbar_nat, inv, err);
-  return cudaGetLastError();
+  const int64_t nb = K.N / blk;
+  for (int q = 0; q < perm_nseg; ++q) {      // one launch per query segment's permutation
+    pool_key_blocks_kernel<<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(K.ptr), K.sB, K.sH, K.sN,
+                                                 K.N, static_cast<int>(K.D), blk, seg, perm + q * K.N,
+                                                 perm_nseg * K.N, (natural && q == 0) ? 1 : 0,
+                                                 kbar_perm + q * nb * K.D, perm_nseg * nb, kbar_nat,
+                                                 inv + q * K.N, err);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 cudaError_t launch_select_blocks(const SelectParams& p, const float* qbar, const float* kbar_perm,
                                  const float* kbar_nat, const int32_t* inv, float* scores, int32_t* counts,
                                  int32_t* idx, int* err, cudaStream_t s) {
-  const int tiles = (p.nb + kTile - 1) / kTile;
-  dim3 g1(static_cast<unsigned>(tiles), static_cast<unsigned>(tiles), static_cast<unsigned>(p.B * p.Hq));
-  block_scores_kernel<<<g1, 256, 0, s>>>(p, qbar, kbar_perm, scores);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e;
+  if (p.perm_nseg > 1) {
+    const int64_t rows = static_cast<int64_t>(p.B) * p.Hq * p.nb;
+    block_scores_seg_kernel<<<static_cast<unsigned>((rows + kSegScoreWarps - 1) / kSegScoreWarps),
+                              kSegScoreWarps * 32, 0, s>>>(p, qbar, kbar_perm, scores);
+  } else {
+    const int tiles = (p.nb + kTile - 1) / kTile;
+    dim3 g1(static_cast<unsigned>(tiles), static_cast<unsigned>(tiles), static_cast<unsigned>(p.B * p.Hq));
+    block_scores_kernel<<<g1, 256, 0, s>>>(p, qbar, kbar_perm, scores);
+  }
+  e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (p.mode == PBS_SELECT_TOPK && !p.score_order) {
     const size_t smem = static_cast<size_t>(kWarpsPerCta) * (p.nb / 32 + 1) * 4;

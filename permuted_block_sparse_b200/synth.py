@@ -56,6 +56,7 @@ class Workload:
     n_sink: int = 0           # leading sink keys always kept
     gate_keep: int = 0        # gating: calibrate thresholds to keep this many tiles
     stop_tau: float = 0.0     # S2O early stopping threshold (0 = no early stopping)
+    perm_per_segment: bool = False   # one key permutation per query segment
     stripe_frac: float = 0.0
     c_lo: float = 4.0
     c_hi: float = 4.0
@@ -106,6 +107,12 @@ WORKLOADS = {
     "s2o_32k_stop": Workload(
         "s2o_32k_stop", B=1, Hq=32, Hkv=8, N=32768, d=128, blk=128, seg=2048,
         mode="topk", density=1.0, stop_tau=0.02, stripe_frac=0.005, c_lo=3.0, c_hi=6.0),
+    # The same with S2O's per-segment key permutation: each query segment's
+    # history sorted by that segment's pooled query.
+    "s2o_32k_segperm": Workload(
+        "s2o_32k_segperm", B=1, Hq=32, Hkv=8, N=32768, d=128, blk=128, seg=2048,
+        mode="topk", density=1.0, stop_tau=0.02, perm_per_segment=True, stripe_frac=0.005, c_lo=3.0,
+        c_hi=6.0),
 }
 
 

@@ -136,9 +136,34 @@ def test_early_stop_and_score_order_argument_checks(lib):
             == lib.pbs_select_capacity(32768, 128, 2048, 0, 0.3, 0, 0))
     q, k = _desc(H=2, N=1024), _desc(H=1, N=1024)
     cap = pbs.select_capacity(1024, 128, 256, "topk", 0.5)
-    rc = lib.pbs_select(ctypes.byref(q), ctypes.byref(k), ctypes.c_void_p(0x2000), 128, 256, 0x20, 0.5, 0, 0,
+    rc = lib.pbs_select(ctypes.byref(q), ctypes.byref(k), ctypes.c_void_p(0x2000), 128, 256, 0x40, 0.5, 0, 0,
                         ctypes.c_void_p(0x3000), ctypes.c_void_p(0x5000), cap, ctypes.c_void_p(0x4000),
                         1 << 30, None)
+    assert rc == -1
+
+
+def test_segmented_permutation_host_checks(lib):
+    q, k, v, o = _desc(H=2), _desc(H=1), _desc(H=1), _desc(H=2)
+    # general entry point: unknown flags, and a gate together with early stopping
+    rc = lib.pbs_attn_fwd_ex(ctypes.byref(q), ctypes.byref(k), ctypes.byref(v), ctypes.c_void_p(0x2000),
+                             ctypes.c_void_p(0x3000), ctypes.c_void_p(0x5000), 4, 128, 256, 8, None, 0.0, 0.088,
+                             ctypes.byref(o), None, None, None)
+    assert rc == -1 and b"flags" in lib.pbs_get_last_error()
+    rc = lib.pbs_attn_fwd_ex(ctypes.byref(q), ctypes.byref(k), ctypes.byref(v), ctypes.c_void_p(0x2000),
+                             ctypes.c_void_p(0x3000), ctypes.c_void_p(0x5000), 4, 128, 256, 1,
+                             ctypes.c_void_p(0x6000), 0.1, 0.088, ctypes.byref(o), None, None, None)
+    assert rc == -2
+    # workspaces: fp64 pooled query per (b, KV head, segment); select holds one
+    # pooled-key matrix and one inverse permutation per query segment
+    Q, K = _desc(B=1, H=32, N=32768), _desc(B=1, H=8, N=32768)
+    nseg, nb = 32768 // 2048, 32768 // 128
+    assert lib.pbs_workspace_size(3, ctypes.byref(Q), ctypes.byref(K), 128, 2048) == 8 * nseg * 128 * 8
+    expect = (32 * nb * 128 * 4 + 8 * nseg * nb * 128 * 4 + 8 * nb * 128 * 4 + 8 * nseg * 32768 * 4
+              + 32 * nb * nb * 4)
+    assert lib.pbs_workspace_size(4, ctypes.byref(Q), ctypes.byref(K), 128, 2048) == expect
+    # a null permutation is refused before anything runs
+    rc = lib.pbs_permute_segmented(ctypes.byref(Q), ctypes.byref(K), 128, 2048, 0, None,
+                                   ctypes.c_void_p(0x4000), 1 << 30, None)
     assert rc == -1
 
 
