@@ -10,6 +10,7 @@ from .pbs_oracle import (attn, attn_block, attn_blocks, attn_early_stop, attn_ea
                          key_scores, key_tiles,
                          lists_to_array, n_candidates, natural_key_block_sums,
                          perm_for_block, permute, permute_segmented, permuted_key_block_sums,
-                         proxy_query, segment_queries,
+                         proxy_query, segment_queries, select_sample, sample_pattern_scores,
+                         sample_trunk_rows, cumulative_cut,
                          query_block_sums, segment_of_block, select,
                          sort_segments, tile_maxima, topk_target)

@@ -340,6 +340,109 @@ def select(Q: np.ndarray, K: np.ndarray, perm: np.ndarray, blk: int, seg: int,
     return counts, lists
 
 
+def sample_trunk_rows(N: int, blk: int, seg: int) -> np.ndarray:
+    """SampleAttention's sampled queries: one trunk per segment, its last
+    query block (the rows that see the segment's whole history)."""
+    rows = []
+    for lo in range(0, N, seg):
+        hi = min(lo + seg, N)
+        rows.extend(range(hi - blk, hi))
+    return np.array(rows, np.int64)
+
+
+def sample_pattern_scores(Q, K, b: int, hq: int, blk: int, seg: int, scale: float):
+    """Stage 1 ("SampleAttention", Technical Deep Dive, 1. Trunk Sampling):
+    the softmax probabilities of the sampled rows over every key they see
+    (fp64), summed per key column and per slash offset q - k.  Returns
+    (col [N], slash [N])."""
+    Hq, Hkv = Q.shape[1], K.shape[1]
+    hk = hq // (Hq // Hkv)
+    N = Q.shape[2]
+    col = np.zeros(N, F64)
+    sl = np.zeros(N, F64)
+    Kf = K[b, hk].astype(F64)
+    for q in sample_trunk_rows(N, blk, seg):
+        lg = (Kf[:q + 1] @ Q[b, hq, q].astype(F64)) * scale
+        e = np.exp(lg - lg.max())
+        p = e / e.sum()
+        col[:q + 1] += p
+        sl[:q + 1] += p[::-1]                    # offset q - k for k = q .. 0
+    return col, sl
+
+
+def cumulative_cut(score: np.ndarray, alpha: float) -> np.ndarray:
+    """Stage 2 decoupled filtering for one pattern family: the entries in
+    descending score (ties to the lower index) up to and including the one
+    at which the accumulated score first reaches alpha of the total; alpha
+    >= 1 keeps every entry with a positive score.  Boolean mask."""
+    keep = np.zeros(score.size, bool)
+    order = np.lexsort((np.arange(score.size), -score))
+    total = score.sum()
+    if alpha >= 1.0:
+        keep[score > 0] = True
+        return keep
+    acc = 0.0
+    for x in order:
+        if acc >= alpha * total:
+            break
+        keep[x] = True
+        acc += score[x]
+    return keep
+
+
+def select_sample(Q, K, blk: int, seg: int, alpha: float,
+                  rows: Optional[Iterable[Tuple[int, int, int]]] = None, trace: Optional[dict] = None):
+    """A SampleAttention-style selector over natural key blocks ("SampleAttention",
+    Technical Deep Dive, Stage 1 Trunk Sampling and Stage 2 Score-Based
+    Filtering).  Per (b, hq): Stage 1 scores (sample_pattern_scores); kept
+    key columns and kept slash offsets by decoupled cumulative cuts at alpha
+    of each family's total (the CIA target for both); query block i lists
+    every earlier-segment key block that holds a kept column or a key q - d
+    of one of its queries q and a kept offset d.  Lists ascending, natural
+    key order (attend with the identity permutation).  ``trace`` receives,
+    per (b, hq), the accumulated score before and after each family's last
+    kept entry and alpha times the total, for margin checks."""
+    B, Hq, N, d = Q.shape
+    nb = N // blk
+    scale = 1.0 / math.sqrt(d)
+    if rows is None:
+        rows = [(b, h, i) for b in range(B) for h in range(Hq) for i in range(nb)]
+    rows = list(rows)
+    counts = np.zeros((B, Hq, nb), np.int32)
+    lists = {}
+    kept = {}
+    for (b, h, i) in rows:
+        if (b, h) not in kept:
+            col, sl = sample_pattern_scores(Q, K, b, h, blk, seg, scale)
+            kc, ks = cumulative_cut(col, alpha), cumulative_cut(sl, alpha)
+            kept[(b, h)] = (kc, ks)
+            if trace is not None:
+                tr = []
+                for sc, kp in ((col, kc), (sl, ks)):
+                    order = np.lexsort((np.arange(sc.size), -sc))
+                    n = int(kp.sum())
+                    before = sc[order[:n - 1]].sum() if n > 0 else 0.0
+                    tr.append((before, sc[order[:n]].sum(), alpha * sc.sum()))
+                trace[(b, h)] = tr
+        kc, ks = kept[(b, h)]
+        ncand = n_candidates(i, blk, seg)
+        chosen = set()
+        for j in range(ncand):
+            if kc[j * blk:(j + 1) * blk].any():
+                chosen.add(j)
+        q0 = i * blk
+        for dlt in np.nonzero(ks)[0]:
+            lo, hi = q0 - int(dlt), q0 + blk - 1 - int(dlt)
+            if hi < 0:
+                continue
+            for j in range(max(lo, 0) // blk, min(hi // blk, ncand - 1) + 1):
+                chosen.add(j)
+        arr = np.array(sorted(chosen), np.int32)
+        lists[(b, h, i)] = arr
+        counts[b, h, i] = arr.size
+    return counts, lists
+
+
 def lists_to_array(counts: np.ndarray, lists: dict, cap: int) -> np.ndarray:
     """Pack lists into idx[B,Hq,nb,cap] (unused entries -1)."""
     B, H, nb = counts.shape

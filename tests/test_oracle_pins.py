@@ -654,3 +654,73 @@ def test_segmented_sparse_attention_equals_masked_sdpa(mode, kw):
     c4, l4 = oracle.select(Q, K, stacked, blk, seg, mode, **kw)
     assert np.array_equal(c3, c4)
     assert all(np.array_equal(l3[k], l4[k]) for k in l3)
+
+
+# ---------------------------------------------------------------------------
+# SampleAttention-style selector ("SampleAttention", Technical Deep Dive,
+# Stage 1 Trunk Sampling and Stage 2 Score-Based Filtering)
+# ---------------------------------------------------------------------------
+
+def test_sample_pattern_scores_explicit():
+    """Column and slash scores equal sums over an explicit torch fp64 softmax
+    of the sampled rows (the last block of every segment)."""
+    B, Hq, Hkv, N, d, blk, seg = 1, 2, 1, 96, 8, 8, 32
+    Q, K, V = _small(B, Hq, Hkv, N, d, seed=61, scale=2.0)
+    scale = 1.0 / math.sqrt(d)
+    rows = oracle.sample_trunk_rows(N, blk, seg)
+    assert rows.tolist() == [r for s in range(N // seg) for r in range(s * seg + seg - blk, (s + 1) * seg)]
+    for h in range(Hq):
+        col, sl = oracle.sample_pattern_scores(Q, K, 0, h, blk, seg, scale)
+        lg = torch.from_numpy(Q[0, h].astype(np.float64)) @ torch.from_numpy(K[0, 0].astype(np.float64)).T * scale
+        mask = torch.tril(torch.ones(N, N, dtype=torch.bool))
+        P = torch.softmax(lg.masked_fill(~mask, float("-inf")), dim=1).numpy()
+        want_col = P[rows].sum(axis=0)
+        want_sl = np.zeros(N)
+        for q in rows:
+            for k in range(q + 1):
+                want_sl[q - k] += P[q, k]
+        np.testing.assert_allclose(col, want_col, rtol=1e-12, atol=1e-15)
+        np.testing.assert_allclose(sl, want_sl, rtol=1e-12, atol=1e-15)
+
+
+@pytest.mark.parametrize("alpha", [0.3, 0.6, 0.9, 0.99])
+def test_cumulative_cut_is_smallest_set(alpha):
+    rng = np.random.default_rng(5)
+    for _ in range(20):
+        sc = rng.random(9) ** 3
+        keep = oracle.cumulative_cut(sc, alpha)
+        goal = alpha * sc.sum()
+        assert sc[keep].sum() >= goal
+        best = None
+        for size in range(0, 10):
+            if any(sum(sc[list(c)]) >= goal for c in itertools.combinations(range(9), size)):
+                best = size
+                break
+        assert keep.sum() == best
+        # the kept entries are the highest scores
+        assert sc[keep].min() >= sc[~keep].max() if (~keep).any() else True
+    assert oracle.cumulative_cut(np.array([0.5, 0.0, 0.2]), 1.0).tolist() == [True, False, True]
+
+
+@pytest.mark.parametrize("alpha", [0.5, 0.9, 1.0])
+def test_select_sample_matches_position_mask(alpha):
+    """Block lists equal the blocks touched by the position-level pattern
+    mask kept_column[k] or kept_slash[q - k], restricted to earlier
+    segments; alpha = 1 lists every candidate."""
+    B, Hq, Hkv, N, d, blk, seg = 1, 2, 1, 128, 16, 8, 32
+    Q, K, V = _small(B, Hq, Hkv, N, d, seed=62, scale=2.0)
+    scale = 1.0 / math.sqrt(d)
+    counts, lists = oracle.select_sample(Q, K, blk, seg, alpha)
+    for h in range(Hq):
+        col, sl = oracle.sample_pattern_scores(Q, K, 0, h, blk, seg, scale)
+        kc, ks = oracle.cumulative_cut(col, alpha), oracle.cumulative_cut(sl, alpha)
+        for i in range(N // blk):
+            ncand = oracle.n_candidates(i, blk, seg)
+            want = set()
+            for q in range(i * blk, (i + 1) * blk):
+                for k in range(ncand * blk):
+                    if k <= q and (kc[k] or ks[q - k]):
+                        want.add(k // blk)
+            assert lists[(0, h, i)].tolist() == sorted(want), (h, i)
+            if alpha >= 1.0:
+                assert lists[(0, h, i)].tolist() == list(range(ncand))
