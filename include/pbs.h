@@ -81,8 +81,8 @@ typedef enum pbs_status {
 } pbs_status;
 
 enum { PBS_OP_PERMUTE = 0, PBS_OP_SELECT = 1, PBS_OP_ATTN = 2, PBS_OP_PERMUTE_SEGMENTED = 3,
-       PBS_OP_SELECT_SEGMENTED = 4 };
-enum { PBS_SELECT_TOPK = 0, PBS_SELECT_TAU = 1 };
+       PBS_OP_SELECT_SEGMENTED = 4, PBS_OP_SELECT_SAMPLE = 5 };
+enum { PBS_SELECT_TOPK = 0, PBS_SELECT_TAU = 1, PBS_SELECT_SAMPLE = 2 };
 /* OR-ed into pbs_select's mode: write lists in visiting order, and/or read
  * one permutation per query segment (see there). */
 enum { PBS_SELECT_SCORE_ORDER = 0x10, PBS_SELECT_PERM_PER_SEGMENT = 0x20 };
@@ -163,6 +163,22 @@ int pbs_select_capacity(int64_t N, int blk, int seg, int mode,
  *     mass (own segment included) is below tau.  tau >= 1 lists all.
  * counts: device int32 [B, Hq, N/blk]; idx: device int32
  * [B, Hq, N/blk, cap]; entries at and after counts[...] are unspecified.
+ *   mode PBS_SELECT_SAMPLE: a SampleAttention-style selector over natural
+ *     key blocks ("SampleAttention", Technical Deep Dive, Stage 1 Trunk
+ *     Sampling and Stage 2 Score-Based Filtering).  The sampled queries are
+ *     the last block of every segment; their softmax probabilities (scale
+ *     1/sqrt(D)) are summed per key column and per slash offset q - k; each
+ *     family keeps its highest entries up to the one at which the
+ *     accumulated score reaches density_or_tau (the CIA target, > 0) of its
+ *     total, ties to the lower index; block i lists every earlier-segment
+ *     block holding a kept column, or a key q - d for one of its queries q
+ *     and a kept offset d.  perm is not read (may be NULL): the lists index
+ *     natural key blocks, to be attended with the identity permutation.
+ *     band, n_sink and the flags do not apply.  ws: pbs_workspace_size(
+ *     PBS_OP_SELECT_SAMPLE, ...) bytes.  The probabilities are fp32, summed
+ *     in fp64, so a column or slash whose accumulated score lies within
+ *     about 1e-6 of the cut may be decided differently from an fp64
+ *     reference.
  * With mode | PBS_SELECT_PERM_PER_SEGMENT, perm is [B, Hkv, nseg, N] from
  * pbs_permute_segmented and block i pools and scores the keys of its own
  * segment's permutation; ws then needs pbs_workspace_size(

@@ -400,8 +400,9 @@ def select_sample(Q, K, blk: int, seg: int, alpha: float,
     every earlier-segment key block that holds a kept column or a key q - d
     of one of its queries q and a kept offset d.  Lists ascending, natural
     key order (attend with the identity permutation).  ``trace`` receives,
-    per (b, hq), the accumulated score before and after each family's last
-    kept entry and alpha times the total, for margin checks."""
+    per (b, hq) and family, the accumulated score before and after the last
+    kept entry, alpha times the total, and the scores of the last kept and
+    the first dropped entry, for margin checks."""
     B, Hq, N, d = Q.shape
     nb = N // blk
     scale = 1.0 / math.sqrt(d)
@@ -422,7 +423,9 @@ def select_sample(Q, K, blk: int, seg: int, alpha: float,
                     order = np.lexsort((np.arange(sc.size), -sc))
                     n = int(kp.sum())
                     before = sc[order[:n - 1]].sum() if n > 0 else 0.0
-                    tr.append((before, sc[order[:n]].sum(), alpha * sc.sum()))
+                    last = sc[order[n - 1]] if n > 0 else np.inf
+                    nxt = sc[order[n]] if n < sc.size else -np.inf
+                    tr.append((before, sc[order[:n]].sum(), alpha * sc.sum(), last, nxt))
                 trace[(b, h)] = tr
         kc, ks = kept[(b, h)]
         ncand = n_candidates(i, blk, seg)

@@ -19,7 +19,9 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libpbs.so")
 
 PBS_OP_PERMUTE, PBS_OP_SELECT, PBS_OP_ATTN, PBS_OP_PERMUTE_SEGMENTED, PBS_OP_SELECT_SEGMENTED = 0, 1, 2, 3, 4
-PBS_SELECT_TOPK, PBS_SELECT_TAU = 0, 1
+PBS_OP_SELECT_SAMPLE = 5
+PBS_SELECT_TOPK, PBS_SELECT_TAU, PBS_SELECT_SAMPLE = 0, 1, 2
+_MODES = {"topk": PBS_SELECT_TOPK, "tau": PBS_SELECT_TAU, "sample": PBS_SELECT_SAMPLE}
 PBS_SELECT_SCORE_ORDER, PBS_SELECT_PERM_PER_SEGMENT = 0x10, 0x20
 PBS_ATTN_EARLY_STOP, PBS_ATTN_PERM_PER_SEGMENT = 1, 2
 STATUS = {0: "PBS_OK", -1: "PBS_ERR_INVALID_ARG", -2: "PBS_ERR_UNSUPPORTED", -3: "PBS_ERR_CAPACITY",
@@ -132,7 +134,7 @@ def workspace_size(op: int, Q: torch.Tensor, K: torch.Tensor, blk: int, seg: int
 
 def select_capacity(N: int, blk: int, seg: int, mode: str, density_or_tau: float,
                     band: int = 0, n_sink: int = 0) -> int:
-    m = PBS_SELECT_TAU if mode == "tau" else PBS_SELECT_TOPK
+    m = _MODES.get(mode, PBS_SELECT_TOPK)
     rc = load().pbs_select_capacity(N, blk, seg, m, float(density_or_tau), band, n_sink)
     _check(min(rc, 0))
     return rc
@@ -187,11 +189,11 @@ def pbs_select(Q: torch.Tensor, K: torch.Tensor, perm: torch.Tensor, blk: int, s
     q, k = describe(Q), describe(K)
     B, Hq, N, _ = Q.shape
     nb = N // blk
-    m = PBS_SELECT_TAU if mode == "tau" else PBS_SELECT_TOPK
+    m = _MODES.get(mode, PBS_SELECT_TOPK)
     if score_order:
         m |= PBS_SELECT_SCORE_ORDER
-    op = PBS_OP_SELECT
-    if perm.dim() == 4:                      # one permutation per query segment
+    op = PBS_OP_SELECT_SAMPLE if mode == "sample" else PBS_OP_SELECT
+    if perm is not None and perm.dim() == 4:   # one permutation per query segment
         m |= PBS_SELECT_PERM_PER_SEGMENT
         op = PBS_OP_SELECT_SEGMENTED
     if cap is None:
@@ -203,7 +205,7 @@ def pbs_select(Q: torch.Tensor, K: torch.Tensor, perm: torch.Tensor, blk: int, s
     if ws is None:
         ws = _workspace(lib.pbs_workspace_size(op, ctypes.byref(q), ctypes.byref(k), blk, seg), Q.device)
     wp, wn = _aligned(ws)
-    _check(lib.pbs_select(ctypes.byref(q), ctypes.byref(k), perm.data_ptr(), blk, seg, m, float(density_or_tau),
+    _check(lib.pbs_select(ctypes.byref(q), ctypes.byref(k), _ptr(perm), blk, seg, m, float(density_or_tau),
                           band, n_sink, counts.data_ptr(), idx.data_ptr(), cap, wp, wn, _stream(stream)))
     return counts, idx
 

@@ -103,6 +103,22 @@ SelectWs select_ws(const pbs::TensorDesc& Q, const pbs::TensorDesc& K, int blk, 
   return w;
 }
 
+// The sample selector's workspace: column and slash scores (fp64) and the
+// two kept-entry bitmaps per (b, hq), in the SelectWs slots qbar, kperm,
+// knat and inv.
+SelectWs sample_ws(const pbs::TensorDesc& Q) {
+  const size_t rows = static_cast<size_t>(Q.B * Q.H);
+  const size_t words = static_cast<size_t>((Q.N + 31) / 32);
+  SelectWs w;
+  w.qbar = 0;
+  w.kperm = w.qbar + align256(rows * Q.N * 8);
+  w.knat = w.kperm + align256(rows * Q.N * 8);
+  w.inv = w.knat + align256(rows * words * 4);
+  w.scores = w.inv + align256(rows * words * 4);
+  w.total = w.scores;
+  return w;
+}
+
 int check_ws(void* ws, size_t ws_bytes, size_t need) {
   if (need == 0) return PBS_OK;
   if (!ws) return fail(PBS_ERR_INVALID_ARG, "workspace is null but %zu bytes are needed", need);
@@ -203,6 +219,8 @@ size_t pbs_workspace_size(int op, const pbs_tensor* Qt, const pbs_tensor* Kt, in
       return nseg > 0 ? align256(static_cast<size_t>(K.B * K.H * nseg * K.D) * 8) : 0;
     case PBS_OP_SELECT_SEGMENTED:
       return nseg > 0 ? select_ws(Q, K, blk, nseg).total : 0;
+    case PBS_OP_SELECT_SAMPLE:
+      return sample_ws(Q).total;
     default:
       return 0;
   }
@@ -255,7 +273,7 @@ int pbs_select_capacity(int64_t N, int blk, int seg, int mode, double density_or
     const int64_t s = i / spb, ncand = s * spb;
     if (ncand == 0) continue;
     int64_t need;
-    if (mode == PBS_SELECT_TAU) {
+    if (mode == PBS_SELECT_TAU || mode == PBS_SELECT_SAMPLE) {
       need = ncand;
     } else {
       const int64_t Di = i - s * spb + 1;
@@ -277,12 +295,17 @@ int pbs_select(const pbs_tensor* Qt, const pbs_tensor* Kt, const int32_t* perm, 
   int rc;
   if ((rc = check_tensor(Qt, "Q", &Q)) || (rc = check_tensor(Kt, "K", &K))) return rc;
   if ((rc = check_geometry(Q, K, blk, seg))) return rc;
-  if (!perm || !counts || !idx) return fail(PBS_ERR_INVALID_ARG, "perm, counts or idx is null");
+  if (!counts || !idx) return fail(PBS_ERR_INVALID_ARG, "counts or idx is null");
+  if (!perm && (mode & 0xF) != PBS_SELECT_SAMPLE) return fail(PBS_ERR_INVALID_ARG, "perm is null");
   const int score_order = (mode & PBS_SELECT_SCORE_ORDER) ? 1 : 0;
   const int per_segment = (mode & PBS_SELECT_PERM_PER_SEGMENT) ? 1 : 0;
   mode &= ~(PBS_SELECT_SCORE_ORDER | PBS_SELECT_PERM_PER_SEGMENT);
-  if (mode != PBS_SELECT_TOPK && mode != PBS_SELECT_TAU)
+  if (mode != PBS_SELECT_TOPK && mode != PBS_SELECT_TAU && mode != PBS_SELECT_SAMPLE)
     return fail(PBS_ERR_INVALID_ARG, "mode %d unknown", mode);
+  if (mode == PBS_SELECT_SAMPLE && (score_order || per_segment))
+    return fail(PBS_ERR_UNSUPPORTED, "the sample selector lists natural blocks in ascending order only");
+  if (mode == PBS_SELECT_SAMPLE && !(density_or_tau > 0.0))
+    return fail(PBS_ERR_INVALID_ARG, "CIA target %g must be positive", density_or_tau);
   if (!(density_or_tau >= 0.0) || (mode == PBS_SELECT_TOPK && density_or_tau > 1.0))
     return fail(PBS_ERR_INVALID_ARG, "density/tau %g out of range", density_or_tau);
   if (band < 0 || n_sink < 0) return fail(PBS_ERR_INVALID_ARG, "band/n_sink negative");
@@ -292,7 +315,7 @@ int pbs_select(const pbs_tensor* Qt, const pbs_tensor* Kt, const int32_t* perm, 
   if (cap < need_cap || cap < 1)
     return fail(PBS_ERR_CAPACITY, "cap %d < required %d", cap, std::max(need_cap, 1));
   const int64_t perm_nseg = per_segment ? (Q.N + seg - 1) / seg : 1;
-  const SelectWs w = select_ws(Q, K, blk, perm_nseg);
+  const SelectWs w = mode == PBS_SELECT_SAMPLE ? sample_ws(Q) : select_ws(Q, K, blk, perm_nseg);
   if ((rc = check_ws(ws, ws_bytes, w.total))) return rc;
   int* err = device_error_word();
   if (!err) return fail(PBS_ERR_CUDA, "cannot resolve the device error word");
@@ -303,6 +326,32 @@ int pbs_select(const pbs_tensor* Qt, const pbs_tensor* Kt, const int32_t* perm, 
   float* knat = reinterpret_cast<float*>(base + w.knat);
   int32_t* inv = reinterpret_cast<int32_t*>(base + w.inv);
   float* scores = reinterpret_cast<float*>(base + w.scores);
+  if (mode == PBS_SELECT_SAMPLE) {
+    pbs::SelectParams p;
+    p.B = static_cast<int>(Q.B);
+    p.Hq = static_cast<int>(Q.H);
+    p.Hkv = static_cast<int>(K.H);
+    p.D = static_cast<int>(Q.D);
+    p.blk = blk;
+    p.seg = seg;
+    p.nb = static_cast<int>(nb);
+    p.mode = mode;
+    p.score_order = 0;
+    p.perm_nseg = 1;
+    p.band = 0;
+    p.n_sink = 0;
+    p.cap = cap;
+    p.N = Q.N;
+    p.rho_permille = 0;
+    p.tau = density_or_tau;
+    const float scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(Q.D)));
+    cudaError_t e = pbs::launch_select_sample(p, Q, K, scale_log2, reinterpret_cast<double*>(base + w.qbar),
+                                              reinterpret_cast<double*>(base + w.kperm),
+                                              reinterpret_cast<uint32_t*>(base + w.knat),
+                                              reinterpret_cast<uint32_t*>(base + w.inv), counts, idx, err, s);
+    if (e != cudaSuccess) return cuda_fail(e, "select_sample launch");
+    return ok();
+  }
   cudaError_t e = pbs::launch_pool_query_blocks(Q, blk, qbar, s);
   if (e != cudaSuccess) return cuda_fail(e, "pool_query_blocks launch");
   e = pbs::launch_pool_key_blocks(K, perm, static_cast<int>(perm_nseg), blk, seg, mode == PBS_SELECT_TAU, kperm,

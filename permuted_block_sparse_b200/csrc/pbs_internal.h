@@ -35,6 +35,9 @@ struct SelectParams {
   int64_t rho_permille;   // top-k density in per-mille
   double tau;
 };
+cudaError_t launch_select_sample(const SelectParams& p, const TensorDesc& Q, const TensorDesc& K,
+                                 float scale_log2, double* col, double* sl, uint32_t* keep_col,
+                                 uint32_t* keep_sl, int32_t* counts, int32_t* idx, int* err, cudaStream_t s);
 cudaError_t launch_select_blocks(const SelectParams& p, const float* qbar, const float* kbar_perm,
                                  const float* kbar_nat, const int32_t* inv, float* scores, int32_t* counts,
                                  int32_t* idx, int* err, cudaStream_t s);
