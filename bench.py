@@ -62,6 +62,9 @@ def dense_causal_flops(w) -> float:
 
 
 def selection_label(w) -> str:
+    if w.mode == "sample":
+        return (f"SampleAttention-style: trunks = last block of each segment, CIA target alpha={w.tau} "
+                f"on key columns and slashes, natural key order")
     if w.mode == "gate":
         return f"all earlier blocks, block-max gate calibrated to keep {w.gate_keep} tiles"
     if w.stop_tau > 0:
@@ -153,6 +156,14 @@ def oracle_baseline(w, Q, K, V, budget_s: float = 20.0, n_blocks: int = 48):
         perm = np.broadcast_to(np.arange(w.N, dtype=np.int32), (w.B, w.Hkv, w.N)).copy()
         lists = {key: np.arange(key[2], dtype=np.int32) for key in blocks}
         thr = np.load(os.path.join(ROOT, "tests", "golden", f"gate_thr_{w.name}.npy")).astype(np.float64)
+    elif w.mode == "sample":
+        # no permutation: identity order; the selector of one query head
+        # (its trunk scores dominate), scaled by B*Hq
+        t_perm = 0.0
+        perm = np.broadcast_to(np.arange(w.N, dtype=np.int32), (w.B, w.Hkv, w.N)).copy()
+        t0 = time.perf_counter()
+        _, lists = oracle.select_sample(Q, K, w.blk, w.seg, w.tau, rows=[(0, 0, i) for i in range(w.nb)])
+        t_sel = (time.perf_counter() - t0) * w.B * w.Hq
     else:
         t0 = time.perf_counter()
         if w.perm_per_segment:
@@ -198,7 +209,9 @@ def oracle_baseline(w, Q, K, V, budget_s: float = 20.0, n_blocks: int = 48):
         "cores": cores,
         "kind": "oracle",
         "sample": (f"fp64 numpy oracle: "
-                   + ("" if w.mode == "gate" else f"permutation of 1 of {w.B * w.Hkv} KV heads, selection + ")
+                   + ("" if w.mode == "gate" else
+                      f"selection of 1 of {w.B * w.Hq} query heads + " if w.mode == "sample" else
+                      f"permutation of 1 of {w.B * w.Hkv} KV heads, selection + ")
                    + f"attention of {len(done)} query blocks of head 0 spread over N={w.N}; scaled to all "
                    f"{n_rows} query blocks; est. full run {total:.0f} s"),
         "est_total_s": total,
@@ -230,7 +243,7 @@ def run_pbs(args):
     K = torch.from_numpy(Kn).to(torch.bfloat16).to(dev)
     V = torch.from_numpy(Vn).to(torch.bfloat16).to(dev)
     s = torch.cuda.current_stream()
-    dt = w.tau if w.mode == "tau" else w.density
+    dt = w.tau if w.mode in ("tau", "sample") else w.density
     cap = max(1, pbs.select_capacity(w.N, w.blk, w.seg, w.mode, dt, w.band, w.n_sink))
     segperm = w.perm_per_segment       # one key permutation per query segment
     nseg = (w.N + w.seg - 1) // w.seg
@@ -240,7 +253,9 @@ def run_pbs(args):
     O = torch.empty_like(Q)
     lse = torch.empty((w.B, w.Hq, w.N), dtype=torch.float32, device=dev)
     op_p = pbs.PBS_OP_PERMUTE_SEGMENTED if segperm else pbs.PBS_OP_PERMUTE
-    op_s = pbs.PBS_OP_SELECT_SEGMENTED if segperm else pbs.PBS_OP_SELECT
+    sample = w.mode == "sample"     # SampleAttention-style selection, natural key order
+    op_s = (pbs.PBS_OP_SELECT_SEGMENTED if segperm else
+            pbs.PBS_OP_SELECT_SAMPLE if sample else pbs.PBS_OP_SELECT)
     ws_p = torch.empty(pbs.workspace_size(op_p, Q, K, w.blk, w.seg) + 256, dtype=torch.uint8, device=dev)
     ws_s = torch.empty(pbs.workspace_size(op_s, Q, K, w.blk, w.seg) + 256, dtype=torch.uint8, device=dev)
     permute = pbs.pbs_permute_segmented if segperm else pbs.pbs_permute
@@ -260,6 +275,9 @@ def run_pbs(args):
         cap = max(w.nb - 1, 1)
         idx = torch.arange(cap, dtype=torch.int32, device=dev).expand(w.B, w.Hq, w.nb, cap).contiguous()
         launches_per_step = 1
+    if sample:
+        perm.copy_(torch.arange(w.N, dtype=torch.int32, device=dev).expand(w.B, w.Hkv, w.N))
+        launches_per_step = 4   # 3 select + 1 attention kernels
 
     ev = {k: [] for k in ("p0", "p1", "s1", "a1")}
 
@@ -267,13 +285,13 @@ def run_pbs(args):
         e = [torch.cuda.Event(enable_timing=True) for _ in range(4)] if record else None
         if record:
             e[0].record(s)
-        if not gate:
+        if not gate and not sample:
             permute(Q, K, w.blk, w.seg, w.n_sink, perm=perm, ws=ws_p)
         if record:
             e[1].record(s)
         if not gate:
-            pbs.pbs_select(Q, K, perm, w.blk, w.seg, w.mode, dt, w.band, w.n_sink, cap=cap, counts=counts,
-                           idx=idx, ws=ws_s, score_order=early)
+            pbs.pbs_select(Q, K, None if sample else perm, w.blk, w.seg, w.mode, dt, w.band, w.n_sink, cap=cap,
+                           counts=counts, idx=idx, ws=ws_s, score_order=early)
         if record:
             e[2].record(s)
         if early:
@@ -356,27 +374,34 @@ def run_pbs(args):
             lse_all = torch.empty_like(lse)
             pbs.pbs_attn_fwd(Q, K, V, ident, d_counts, d_idx, w.blk, w.blk, out=Od, lse=lse_all)
             cov_perm = torch.exp(lse - lse_all).flatten()
-            c_nat = torch.empty_like(counts)
-            i_nat = torch.empty_like(idx)
-            pbs.pbs_select(Q, K, ident, w.blk, w.seg, w.mode, dt, w.band, w.n_sink, cap=cap, counts=c_nat,
-                           idx=i_nat, ws=ws_s, score_order=early)
-            lse_nat = torch.empty_like(lse)
-            if early:
-                pbs.pbs_attn_fwd_early_stop(Q, K, V, ident, c_nat, i_nat, w.blk, w.seg, w.stop_tau, out=Od,
-                                            lse=lse_nat)
-            else:
-                pbs.pbs_attn_fwd(Q, K, V, ident, c_nat, i_nat, w.blk, w.seg, out=Od, lse=lse_nat)
-            pbs.pbs_check_device()
-            cov_nat = torch.exp(lse_nat - lse_all).flatten()
             q = torch.tensor([0.01, 0.5], device=dev)
-            sample = torch.randperm(cov_perm.numel(), device=dev)[:1 << 20]
-            pq = torch.quantile(cov_perm[sample], q).tolist()
-            nq = torch.quantile(cov_nat[sample], q).tolist()
-            dense["coverage"] = {"permuted": {"mean": cov_perm.mean().item(), "p01": pq[0], "median": pq[1]},
-                                 "natural": {"mean": cov_nat.mean().item(), "p01": nq[0], "median": nq[1]},
-                                 "what": "share of each query row's causal softmax mass on its key set, "
-                                         "permuted keys vs the same rule on natural key order"}
-            del lse_all, c_nat, i_nat, lse_nat
+            pick = torch.randperm(cov_perm.numel(), device=dev)[:1 << 20]
+            pq = torch.quantile(cov_perm[pick], q).tolist()
+            if sample:
+                # the sample selector already works on the natural key order
+                dense["coverage"] = {"selected": {"mean": cov_perm.mean().item(), "p01": pq[0],
+                                                  "median": pq[1]},
+                                     "what": "share of each query row's causal softmax mass on its key set"}
+            else:
+                c_nat = torch.empty_like(counts)
+                i_nat = torch.empty_like(idx)
+                pbs.pbs_select(Q, K, ident, w.blk, w.seg, w.mode, dt, w.band, w.n_sink, cap=cap, counts=c_nat,
+                               idx=i_nat, ws=ws_s, score_order=early)
+                lse_nat = torch.empty_like(lse)
+                if early:
+                    pbs.pbs_attn_fwd_early_stop(Q, K, V, ident, c_nat, i_nat, w.blk, w.seg, w.stop_tau, out=Od,
+                                                lse=lse_nat)
+                else:
+                    pbs.pbs_attn_fwd(Q, K, V, ident, c_nat, i_nat, w.blk, w.seg, out=Od, lse=lse_nat)
+                pbs.pbs_check_device()
+                cov_nat = torch.exp(lse_nat - lse_all).flatten()
+                nq = torch.quantile(cov_nat[pick], q).tolist()
+                dense["coverage"] = {"permuted": {"mean": cov_perm.mean().item(), "p01": pq[0], "median": pq[1]},
+                                     "natural": {"mean": cov_nat.mean().item(), "p01": nq[0], "median": nq[1]},
+                                     "what": "share of each query row's causal softmax mass on its key set, "
+                                             "permuted keys vs the same rule on natural key order"}
+                del c_nat, i_nat, lse_nat
+            del lse_all
         del d_idx, Od
 
     # end to end through the C ABI with host buffers: H2D of Q, K, V from
@@ -394,9 +419,10 @@ def run_pbs(args):
             Kd.copy_(Kh, non_blocking=True)
             Vd.copy_(Vh, non_blocking=True)
             if not gate:
-                permute(Qd, Kd, w.blk, w.seg, w.n_sink, perm=perm, ws=ws_p)
-                pbs.pbs_select(Qd, Kd, perm, w.blk, w.seg, w.mode, dt, w.band, w.n_sink, cap=cap,
-                               counts=counts, idx=idx, ws=ws_s, score_order=early)
+                if not sample:
+                    permute(Qd, Kd, w.blk, w.seg, w.n_sink, perm=perm, ws=ws_p)
+                pbs.pbs_select(Qd, Kd, None if sample else perm, w.blk, w.seg, w.mode, dt, w.band, w.n_sink,
+                               cap=cap, counts=counts, idx=idx, ws=ws_s, score_order=early)
             if early:
                 pbs.pbs_attn_fwd_early_stop(Qd, Kd, Vd, perm, counts, idx, w.blk, w.seg, w.stop_tau, out=O,
                                             lse=lse)

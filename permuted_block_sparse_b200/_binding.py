@@ -189,7 +189,9 @@ def pbs_select(Q: torch.Tensor, K: torch.Tensor, perm: torch.Tensor, blk: int, s
     q, k = describe(Q), describe(K)
     B, Hq, N, _ = Q.shape
     nb = N // blk
-    m = _MODES.get(mode, PBS_SELECT_TOPK)
+    if mode not in _MODES:
+        raise ValueError(f"unknown selection mode {mode!r}; expected one of {sorted(_MODES)}")
+    m = _MODES[mode]
     if score_order:
         m |= PBS_SELECT_SCORE_ORDER
     op = PBS_OP_SELECT_SAMPLE if mode == "sample" else PBS_OP_SELECT

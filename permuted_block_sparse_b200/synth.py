@@ -17,6 +17,12 @@ activations are not available, so a planted-stripe model stands in for them:
     without replacement, get K += c * u_h, with c fixed or drawn per stripe
     key from U[c_lo, c_hi];
   * every query of the heads in that KV head's group gets Q += q_off * u_h;
+  * optionally (``local_amp`` > 0) a planted local window, the slash
+    pattern that "SampleAttention" (Background; Key Findings 5) names beside
+    column stripes: the same deterministic positional vector -- ``local_pairs``
+    (cos, sin) pairs of geometric periods from ``local_pmin`` to
+    ``local_pmax`` with amplitude ``local_amp``, in the last dims -- is added
+    to every query and key at that position, so q.k rises near the diagonal;
   * finally every value is rounded to a multiple of 1/8 and clipped to
     +-31.875, so it is exact in bfloat16 ("lattice" values).  On lattice
     inputs every pooled sum and block score of the method is exactly
@@ -49,13 +55,17 @@ class Workload:
     d: int
     blk: int
     seg: int
-    mode: str                 # "topk", "tau" or "gate"
+    mode: str                 # "topk", "tau", "gate" or "sample"
     density: float = 1.0      # top-k density rho
-    tau: float = 1.0          # cumulative-mass target
+    tau: float = 1.0          # cumulative-mass target (the CIA target alpha for "sample")
     band: int = 0             # most recent keys always kept (0 = none)
     n_sink: int = 0           # leading sink keys always kept
     gate_keep: int = 0        # gating: calibrate thresholds to keep this many tiles
     stop_tau: float = 0.0     # S2O early stopping threshold (0 = no early stopping)
+    local_amp: float = 0.0    # planted local window: amplitude of the positional pairs (0 = none)
+    local_pairs: int = 16     # number of (cos, sin) pairs, in the last 2*local_pairs dims
+    local_pmin: float = 32.0  # shortest and longest period of the pairs, in positions
+    local_pmax: float = 32768.0
     perm_per_segment: bool = False   # one key permutation per query segment
     stripe_frac: float = 0.0
     c_lo: float = 4.0
@@ -113,6 +123,15 @@ WORKLOADS = {
         "s2o_32k_segperm", B=1, Hq=32, Hkv=8, N=32768, d=128, blk=128, seg=2048,
         mode="topk", density=1.0, stop_tau=0.02, perm_per_segment=True, stripe_frac=0.005, c_lo=3.0,
         c_hi=6.0),
+    # SampleAttention-style selection on inputs with both of the patterns that
+    # page names: a planted local window (slash) and strong column stripes.
+    # CIA target 0.95 for both families.  Amplitude and stripe strength are
+    # set so that the selection keeps about a quarter of the causal tiles
+    # and about 99 % of a row's softmax mass on average, near the highly
+    # sparse attention that page reports for real models.
+    "sample_32k_local": Workload(
+        "sample_32k_local", B=1, Hq=32, Hkv=8, N=32768, d=128, blk=128, seg=2048,
+        mode="sample", tau=0.95, stripe_frac=0.005, c_lo=8.0, c_hi=12.0, q_off=3.0, local_amp=3.5),
 }
 
 
@@ -156,6 +175,18 @@ def make_inputs(w: Workload, seed: Optional[int] = None) -> Tuple[np.ndarray, np
             dirs[b, h] = u
             stripes[b, h] = pos
             offsets[b, h] = c
+    if w.local_amp > 0:
+        # same positional pairs on queries and keys: q.k gains
+        # amp^2 * sum_f cos(omega_f (n - k)), largest on the diagonal
+        per = np.geomspace(w.local_pmin, w.local_pmax, w.local_pairs)
+        om = 2.0 * np.pi / per
+        ang = np.arange(N, dtype=np.float64)[:, None] * om[None, :]
+        P = np.zeros((N, d), np.float32)
+        c0 = d - 2 * w.local_pairs
+        P[:, c0::2] = (w.local_amp * np.cos(ang)).astype(np.float32)
+        P[:, c0 + 1::2] = (w.local_amp * np.sin(ang)).astype(np.float32)
+        Q += P
+        K += P
     Q = lattice(Q)
     K = lattice(K)
     V = lattice(V)

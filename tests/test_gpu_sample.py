@@ -77,3 +77,43 @@ def test_sample_lists_match_oracle(shape, alpha):
 def test_sample_lists_8k_workload(alpha):
     w, Q, K, V = workload_inputs("gqa_8k_band")
     _compare(w, Q, K, alpha, min_heads=(w.B * w.Hq) // 2)
+
+
+def test_sample_32k_workload_sampled():
+    """The benchmark's 32K SampleAttention workload in the launch
+    configuration the benchmark times: the selector over all heads, then
+    attention over its lists.  Two query heads' lists are compared with the
+    oracle's (bit-exact where their cuts have room), and six query blocks of
+    each head with the oracle's attention over the GPU's own lists."""
+    w, Q, K, V = workload_inputs("sample_32k_local")
+    Qd, Kd, Vd = dev(Q), dev(K), dev(V)
+    cap = pbs.select_capacity(w.N, w.blk, w.seg, "sample", w.tau)
+    c_d, i_d = pbs.pbs_select(Qd, Kd, None, w.blk, w.seg, "sample", w.tau, cap=cap)
+    ident = torch.arange(w.N, dtype=torch.int32, device="cuda").expand(w.B, w.Hkv, w.N).contiguous()
+    O, L = pbs.pbs_attn_fwd(Qd, Kd, Vd, ident, c_d, i_d, w.blk, w.seg)
+    pbs.pbs_check_device()
+    c_g, i_g = c_d.cpu().numpy(), i_d.cpu().numpy()
+    # the selection is sparse on these inputs
+    spb = w.seg // w.blk
+    cand = sum(oracle.n_candidates(i, w.blk, w.seg) for i in range(w.nb)) * w.B * w.Hq
+    assert 0 < c_g.sum() < 0.5 * cand
+    ident_np = np.broadcast_to(np.arange(w.N, dtype=np.int32), (w.B, w.Hkv, w.N)).copy()
+    compared = 0
+    for h in (0, 21):
+        trace = {}
+        _, lists = oracle.select_sample(Q, K, w.blk, w.seg, w.tau, rows=[(0, h, i) for i in range(w.nb)],
+                                        trace=trace)
+        if _clear(trace[(0, h)], w.tau):
+            compared += 1
+            for i in range(w.nb):
+                arr = lists[(0, h, i)]
+                assert int(c_g[0, h, i]) == arr.size, (h, i)
+                assert i_g[0, h, i, :arr.size].tolist() == arr.tolist(), (h, i)
+        blocks = [(0, h, int(i)) for i in np.linspace(spb, w.nb - 1, 6).round()]
+        gl = {key: i_g[key][:c_g[key]].copy() for key in blocks}
+        ref = oracle.attn_blocks(Q, K, V, ident_np, gl, w.blk, w.seg, blocks)
+        for (b, hh, i), (o_ref, l_ref) in ref.items():
+            r = slice(i * w.blk, (i + 1) * w.blk)
+            assert_close(O[b, hh, r], o_ref, what=f"head {hh} block {i}")
+            assert np.nanmax(np.abs(L[b, hh, r].cpu().numpy() - l_ref)) <= LSE_MAX_ABS
+    assert compared >= 1
