@@ -24,66 +24,235 @@ namespace {
 
 constexpr int kSampleWarps = 8;
 
-// Stage 1.  One warp per (sampled row, hq, b); lanes own keys.  The raw q.k
-// of bf16 inputs is accumulated in fp32; the probabilities are
-// 2^(x - m) / l with x the scaled logit in log2 units.
-__global__ void __launch_bounds__(kSampleWarps * 32) sample_scores_kernel(
+// Stage 1 on the tensor cores.  One CTA of 256 threads per (trunk s, hq, b),
+// heaviest trunks first.  The trunk's rows (the last blk queries of segment
+// s, zero rows up to 128) stay in shared memory; the keys 0 .. seg_end - 1
+// stream through in tiles of 128, and S = Q_trunk K_tile^T is computed by
+// tcgen05.mma into one of two tensor-memory buffers while the previous tile
+// is processed and the next one is copied in.  Warp w reads tensor-memory
+// lanes 32 (w mod 4) .. +31 (trunk rows) and columns 64 (w / 4) .. +63, so
+// each row has two threads, one per column half.
+//   Pass 1 (tiles 0 .. T-1): per row and half the running maximum m of
+//     x = S * log2(e) / sqrt(d) over the causal keys, kept rounded up to an
+//     integer so that every rescale of the running sum l = sum 2^(x - m)
+//     (fp64) is an exact power of two; the halves are merged at the end.
+//   Pass 2 (the same tiles again): p = 2^(x - m) (fp32) is written to a
+//     skewed 128 x 128 fp32 tile in shared memory -- element (t, c) at
+//     column (c - t) mod 128 -- so that thread c (< 128) reads key column c
+//     and thread 128 + u reads the two diagonals t - c = -u and 128 - u,
+//     both without bank conflicts.  Each reduction weighs row t by 1 / l_t
+//     in fp64 and adds its total to the key's column score or the offset's
+//     slash score.
+// The logits q.k of bf16 inputs are accumulated in fp32 by the tensor core.
+template <int D>
+struct SampleCfg {
+  static constexpr int kHalfBytes = 128 * 128;               // 128 rows x 64 bf16
+  static constexpr int kTileBytes = (D / 64) * kHalfBytes;   // Q or K tile
+  static constexpr int kQ = 0;
+  static constexpr int kK = kQ + kTileBytes;
+  static constexpr int kP = kK + 2 * kTileBytes;
+  static constexpr int kW = kP + 128 * 128 * 4;
+  static constexpr int kMl = kW + 128 * 8;                     // per-half (m, l) at the end of pass 1
+  static constexpr int kBar = kMl + 2 * 128 * 16;
+  static constexpr int kSlot = kBar + 2 * 8;
+  static constexpr int kBytes = kSlot + 16;
+  static constexpr int kSmem = kBytes + 1024;                // alignment slack
+};
+constexpr int kScoreThreads = 256;
+
+template <int D>
+__global__ void __launch_bounds__(kScoreThreads, 1) sample_scores_kernel(
     const __nv_bfloat16* __restrict__ Q, int64_t qsB, int64_t qsH, int64_t qsN,
-    const __nv_bfloat16* __restrict__ K, int64_t ksB, int64_t ksH, int64_t ksN, int64_t N, int D, int G,
-    int blk, int seg, float scale_log2, double* __restrict__ col, double* __restrict__ sl) {
-  __shared__ float qs[kSampleWarps][128];
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int rrow = blockIdx.x * kSampleWarps + warp;            // sampled row index
+    const __nv_bfloat16* __restrict__ K, int64_t ksB, int64_t ksH, int64_t ksN, int64_t N, int B, int Hq,
+    int G, int blk, int seg, float scale_log2, double* __restrict__ col, double* __restrict__ sl,
+    int* __restrict__ err) {
+  using C = SampleCfg<D>;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                         ~static_cast<uintptr_t>(1023));
+  float* sP = reinterpret_cast<float*>(smem + C::kP);
+  double* sW = reinterpret_cast<double*>(smem + C::kW);
+  float* sM = reinterpret_cast<float*>(smem + C::kMl);                   // [2][128]
+  double* sL = reinterpret_cast<double*>(smem + C::kMl + 2 * 128 * 4);   // [2][128]
+  uint64_t* bar_s = reinterpret_cast<uint64_t*>(smem + C::kBar);
+  uint32_t* slot = reinterpret_cast<uint32_t*>(smem + C::kSlot);
+  const uint32_t sQ = smem_u32(smem + C::kQ), sK = smem_u32(smem + C::kK);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int t = (warp & 3) * 32 + lane;                        // trunk row of this thread
+  const int hc = warp >> 2;                                    // column half
   const int nseg = static_cast<int>((N + seg - 1) / seg);
-  if (rrow >= nseg * blk) return;
-  const int hq = blockIdx.y, b = blockIdx.z, Hq = gridDim.y;
-  const int s = rrow / blk;
+  const int BH = B * Hq;
+  const int s = nseg - 1 - static_cast<int>(blockIdx.x / BH);
+  const int bh = static_cast<int>(blockIdx.x % BH);
+  const int b = bh / Hq, hq = bh % Hq;
   const int64_t seg_end = min(static_cast<int64_t>(s + 1) * seg, N);
-  const int64_t q = seg_end - blk + (rrow % blk);
-  const __nv_bfloat16* qrow = Q + b * qsB + hq * qsH + q * qsN;
-  for (int c = lane; c < D; c += 32) qs[warp][c] = __bfloat162float(qrow[c]);
-  __syncwarp();
+  const int64_t qbase = seg_end - blk;
+  const int T = static_cast<int>((seg_end + 127) / 128);
+  constexpr int CH = D / 8;                                    // 16-byte chunks per row
+
+  const __nv_bfloat16* qb = Q + b * qsB + hq * qsH;
   const __nv_bfloat16* kb = K + b * ksB + (hq / G) * ksH;
-  auto logit = [&](int64_t k) -> float {
-    const uint4* kr = reinterpret_cast<const uint4*>(kb + k * ksN);
-    float acc = 0.f;
-    for (int c = 0; c < D / 8; ++c) {
-      const uint4 v = kr[c];
-      const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v);
+  auto load_k = [&](int j, int buf) {
+    const int64_t k0 = static_cast<int64_t>(j) * 128;
+    const uint32_t dst = sK + buf * C::kTileBytes;
+    for (int id = tid; id < 128 * CH; id += kScoreThreads) {
+      const int r = id / CH, c = id % CH;
+      const bool valid = k0 + r < seg_end;
+      cp_async16_zfill(dst + (c / 8) * C::kHalfBytes + sw128_offset(r, c % 8),
+                       valid ? kb + (k0 + r) * ksN + c * 8 : kb, valid);
+    }
+    cp_async_commit();
+  };
+
+  if (warp == 0) {
+    tmem_alloc(slot, 256);
+    tmem_relinquish();
+  }
+  if (tid == 0) {
+    mbar_init(&bar_s[0], 1);
+    mbar_init(&bar_s[1], 1);
+    fence_mbar_init();
+  }
+  for (int id = tid; id < 128 * CH; id += kScoreThreads) {
+    const int r = id / CH, c = id % CH;
+    const bool valid = r < blk;
+    cp_async16_zfill(sQ + (c / 8) * C::kHalfBytes + sw128_offset(r, c % 8),
+                     valid ? qb + (qbase + r) * qsN + c * 8 : qb, valid);
+  }
+  load_k(0, 0);
+  load_k(1 % T, 1);
+  cp_async_wait_all();
+  fence_proxy_async();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *slot;
+  const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+  constexpr uint32_t idesc = idesc_bf16(128, 128, false);
+
+  const int64_t q_t = qbase + t;
+  const bool row_ok = t < blk;
+  float m = -INFINITY;                                         // integer-valued running maximum
+  double l = 0.0;
+  uint32_t phase[2] = {0u, 0u};
+  bool failed = false;
+
+  for (int it = 0; it <= 2 * T; ++it) {
+    if (it < 2 * T && warp == 0) {
+      const int buf = it & 1;
+      tc_fence_after();
+      const uint64_t a0 = sdesc_sw128(sQ, 16, 1024);
+      const uint64_t b0 = sdesc_sw128(sK + buf * C::kTileBytes, 16, 1024);
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 f = __bfloat1622float2(p[e]);
-        acc = fmaf(f.x, qs[warp][c * 8 + 2 * e], acc);
-        acc = fmaf(f.y, qs[warp][c * 8 + 2 * e + 1], acc);
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = (kk / 4) * C::kHalfBytes + (kk % 4) * 32;
+        if (elect_one()) mma_ss(tmem + buf * 128, sdesc_add(a0, off), sdesc_add(b0, off), idesc, kk > 0 ? 1u : 0u);
+      }
+      if (elect_one()) tc_commit(&bar_s[buf]);
+      __syncwarp();
+    }
+    if (it >= 1) {
+      const int jj = it - 1, buf = jj & 1, j = jj % T;
+      const bool ok = mbar_wait(&bar_s[buf], phase[buf], err);
+      phase[buf] ^= 1u;
+      if (__syncthreads_or(!ok)) {
+        failed = true;
+        break;
+      }
+      tc_fence_after();
+      if (it + 1 < 2 * T) load_k((it + 1) % T, (it + 1) & 1);
+      const int64_t k0 = static_cast<int64_t>(j) * 128;
+      // keys k0 + 64 hc + c with c <= lim are causal for this row
+      const int64_t lim64 = q_t - k0 - 64 * hc;
+      const int lim = row_ok ? static_cast<int>(lim64 > 63 ? 63 : (lim64 < -1 ? -1 : lim64)) : -1;
+      uint32_t r[64];
+      tmem_ld64(tmem + lane_base + buf * 128 + hc * 64, r);
+      if (jj < T) {
+        float mt = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 64; ++c)
+          if (c <= lim) mt = fmaxf(mt, __uint_as_float(r[c]) * scale_log2);
+        if (mt > -INFINITY) {
+          const float mn = fmaxf(m, ceilf(mt));
+          if (mn > m) {
+            l = (m == -INFINITY) ? 0.0 : ldexp(l, static_cast<int>(m - mn));
+            m = mn;
+          }
+          double a[4] = {0.0, 0.0, 0.0, 0.0};
+#pragma unroll
+          for (int c = 0; c < 64; ++c)
+            if (c <= lim) a[c % 4] += static_cast<double>(ex2(__uint_as_float(r[c]) * scale_log2 - m));
+          l += (a[0] + a[1]) + (a[2] + a[3]);
+        }
+        if (jj == T - 1) {
+          // merge the halves: the larger maximum, both sums rescaled by
+          // exact powers of two
+          sM[hc * 128 + t] = m;
+          sL[hc * 128 + t] = l;
+          __syncthreads();
+          const float m0 = sM[t], m1 = sM[128 + t];
+          const float mm = fmaxf(m0, m1);
+          double lt = 0.0;
+          if (m0 > -INFINITY) lt += ldexp(sL[t], static_cast<int>(m0 - mm));
+          if (m1 > -INFINITY) lt += ldexp(sL[128 + t], static_cast<int>(m1 - mm));
+          m = mm;
+          if (hc == 0) sW[t] = row_ok && lt > 0.0 ? 1.0 / lt : 0.0;
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          const int cc = hc * 64 + c;
+          const float e = c <= lim ? ex2(__uint_as_float(r[c]) * scale_log2 - m) : 0.f;
+          sP[t * 128 + ((cc - t) & 127)] = e;
+        }
+        __syncthreads();
+        const int x = tid & 127;
+        const int64_t base = static_cast<int64_t>(bh) * N;
+        if (tid < 128) {
+          // key column x: element (u, x) sits at column (x - u) mod 128
+          double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
+          for (int u = 0; u < blk; u += 4) {               // blk is a multiple of 4
+            a0 = fma(static_cast<double>(sP[u * 128 + ((x - u) & 127)]), sW[u], a0);
+            a1 = fma(static_cast<double>(sP[(u + 1) * 128 + ((x - u - 1) & 127)]), sW[u + 1], a1);
+            a2 = fma(static_cast<double>(sP[(u + 2) * 128 + ((x - u - 2) & 127)]), sW[u + 2], a2);
+            a3 = fma(static_cast<double>(sP[(u + 3) * 128 + ((x - u - 3) & 127)]), sW[u + 3], a3);
+          }
+          const double cs = (a0 + a1) + (a2 + a3);
+          if (cs != 0.0 && k0 + x < N) atomicAdd(col + base + k0 + x, cs);
+        } else {
+          // skew x: rows u < 128 - x lie on offset d0 - x, the rest on d0 + 128 - x
+          const int split = min(128 - x, blk);
+          double a0 = 0.0, a1 = 0.0, b0 = 0.0, b1 = 0.0;
+          int u = 0;
+          for (; u + 1 < split; u += 2) {
+            a0 = fma(static_cast<double>(sP[u * 128 + x]), sW[u], a0);
+            a1 = fma(static_cast<double>(sP[(u + 1) * 128 + x]), sW[u + 1], a1);
+          }
+          if (u < split) a0 = fma(static_cast<double>(sP[u * 128 + x]), sW[u], a0), ++u;
+          for (; u + 1 < blk; u += 2) {
+            b0 = fma(static_cast<double>(sP[u * 128 + x]), sW[u], b0);
+            b1 = fma(static_cast<double>(sP[(u + 1) * 128 + x]), sW[u + 1], b1);
+          }
+          if (u < blk) b0 = fma(static_cast<double>(sP[u * 128 + x]), sW[u], b0);
+          const double da = a0 + a1, db = b0 + b1;
+          const int64_t d0 = qbase - k0;
+          if (da != 0.0 && d0 - x >= 0 && d0 - x < N) atomicAdd(sl + base + d0 - x, da);
+          if (db != 0.0 && d0 + 128 - x >= 0 && d0 + 128 - x < N) atomicAdd(sl + base + d0 + 128 - x, db);
+        }
       }
     }
-    return acc * scale_log2;
-  };
-  // pass 1: running max and sum per lane, then across the warp
-  float m = -INFINITY, l = 0.f;
-  for (int64_t k = lane; k <= q; k += 32) {
-    const float x = logit(k);
-    if (x > m) {
-      l = l * ex2(m - x) + 1.f;
-      m = x;
-    } else {
-      l += ex2(x - m);
-    }
+    cp_async_wait_all();
+    fence_proxy_async();
+    tc_fence_before();
+    __syncthreads();
   }
-  for (int off = 16; off > 0; off >>= 1) {
-    const float m2 = __shfl_xor_sync(0xffffffffu, m, off), l2 = __shfl_xor_sync(0xffffffffu, l, off);
-    const float mn = fmaxf(m, m2);
-    l = (m == -INFINITY ? 0.f : l * ex2(m - mn)) + (m2 == -INFINITY ? 0.f : l2 * ex2(m2 - mn));
-    m = mn;
-  }
-  const float inv_l = 1.f / l;
-  // pass 2: probabilities into the column and slash sums
-  double* cb = col + (static_cast<int64_t>(b) * Hq + hq) * N;
-  double* sb = sl + (static_cast<int64_t>(b) * Hq + hq) * N;
-  for (int64_t k = lane; k <= q; k += 32) {
-    const double p = static_cast<double>(ex2(logit(k) - m) * inv_l);
-    atomicAdd(cb + k, p);
-    atomicAdd(sb + (q - k), p);
+  if (failed) cp_async_wait_all();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
   }
 }
 
@@ -109,10 +278,11 @@ __device__ double block_sum(double v, double* red) {
   return red[32];
 }
 
-// Stage 2, one family.  One CTA per (family, hq, b): the largest score
-// threshold whose upper set reaches alpha of the total (a bisection on the
-// order-preserving 64-bit image of the scores), then the entries at the
-// threshold in ascending index until the target is met.  Writes a bitmap.
+// Stage 2, one family.  One CTA of 1024 threads per (family, hq, b): the
+// largest score threshold whose upper set reaches alpha of the total (a
+// bisection on the order-preserving 64-bit image of the scores), then the
+// entries at the threshold in ascending index until the target is met.
+// Writes a bitmap.
 __global__ void __launch_bounds__(1024) sample_cut_kernel(const double* __restrict__ col,
                                                           const double* __restrict__ sl, int64_t N,
                                                           double alpha, uint32_t* __restrict__ keep_col,
@@ -153,15 +323,44 @@ __global__ void __launch_bounds__(1024) sample_cut_kernel(const double* __restri
     }
   }
   const double above = block_sum(part, red);
-  // at the threshold: ascending index while the accumulated score is below the goal
+  // at the threshold: equal scores in ascending index while the accumulated
+  // score is below the goal.  The number taken follows from the tie count
+  // and the tie value; a block-wide scan then ranks the ties by index.
+  double nt = 0.0;
+  for (int64_t k = threadIdx.x; k < N; k += blockDim.x) nt += ordered_f64(sc[k]) == lo ? 1.0 : 0.0;
+  const int64_t ntie = static_cast<int64_t>(block_sum(nt, red));
+  const uint64_t ubits = (lo & 0x8000000000000000ull) ? (lo & ~0x8000000000000000ull) : ~lo;
+  const double v = __longlong_as_double(static_cast<long long>(ubits));
+  __shared__ int64_t need_sh;
+  __shared__ int wcnt[32];
   if (threadIdx.x == 0) {
     double acc = above;
-    for (int64_t k = 0; k < N && acc < goal; ++k) {
-      if (ordered_f64(sc[k]) == lo) {
-        keep[k >> 5] |= 1u << (k & 31);
-        acc += sc[k];
-      }
+    int64_t n = 0;
+    while (n < ntie && acc < goal) {
+      acc += v;
+      ++n;
     }
+    need_sh = n;
+  }
+  __syncthreads();
+  const int64_t need = need_sh;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarp = blockDim.x >> 5;
+  int64_t running = 0;
+  for (int64_t base = 0; base < N && running < need; base += blockDim.x) {
+    const int64_t k = base + threadIdx.x;
+    const bool f = k < N && ordered_f64(sc[k]) == lo;
+    const uint32_t bal = __ballot_sync(0xffffffffu, f);
+    if (lane == 0) wcnt[warp] = __popc(bal);
+    __syncthreads();
+    int before = 0, tot = 0;
+    for (int w = 0; w < nwarp; ++w) {
+      before += w < warp ? wcnt[w] : 0;
+      tot += wcnt[w];
+    }
+    const int64_t rank = running + before + __popc(bal & ((1u << lane) - 1u));
+    if (f && rank < need) atomicOr(&keep[k >> 5], 1u << (k & 31));
+    running += tot;
+    __syncthreads();
   }
 }
 
@@ -256,13 +455,17 @@ cudaError_t launch_select_sample(const SelectParams& p, const TensorDesc& Q, con
   e = cudaMemsetAsync(sl, 0, nsc * sizeof(double), s);
   if (e != cudaSuccess) return e;
   const int nseg = static_cast<int>((p.N + p.seg - 1) / p.seg);
-  const int nrows = nseg * p.blk;
-  dim3 g1(static_cast<unsigned>((nrows + kSampleWarps - 1) / kSampleWarps), static_cast<unsigned>(p.Hq),
-          static_cast<unsigned>(p.B));
-  sample_scores_kernel<<<g1, kSampleWarps * 32, 0, s>>>(
-      static_cast<const __nv_bfloat16*>(Q.ptr), Q.sB, Q.sH, Q.sN, static_cast<const __nv_bfloat16*>(K.ptr),
-      K.sB, K.sH, K.sN, p.N, p.D, p.Hq / p.Hkv, p.blk, p.seg, scale_log2, col, sl);
-  e = cudaGetLastError();
+  const unsigned nblk = static_cast<unsigned>(nseg) * static_cast<unsigned>(p.B * p.Hq);
+  auto run = [&](auto kernel, int smem_bytes) -> cudaError_t {
+    cudaError_t e2 = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
+    if (e2 != cudaSuccess) return e2;
+    kernel<<<nblk, kScoreThreads, smem_bytes, s>>>(static_cast<const __nv_bfloat16*>(Q.ptr), Q.sB, Q.sH, Q.sN,
+                                         static_cast<const __nv_bfloat16*>(K.ptr), K.sB, K.sH, K.sN, p.N, p.B,
+                                         p.Hq, p.Hq / p.Hkv, p.blk, p.seg, scale_log2, col, sl, err);
+    return cudaGetLastError();
+  };
+  e = p.D == 64 ? run(sample_scores_kernel<64>, SampleCfg<64>::kSmem)
+                : run(sample_scores_kernel<128>, SampleCfg<128>::kSmem);
   if (e != cudaSuccess) return e;
   dim3 g2(2, static_cast<unsigned>(p.Hq), static_cast<unsigned>(p.B));
   sample_cut_kernel<<<g2, 1024, 0, s>>>(col, sl, p.N, p.tau, keep_col, keep_sl);
