@@ -35,24 +35,24 @@ constexpr int kSampleWarps = 8;
 //   Pass 1 (tiles 0 .. T-1): per row and half the running maximum m of
 //     x = S * log2(e) / sqrt(d) over the causal keys, kept rounded up to an
 //     integer so that every rescale of the running sum l = sum 2^(x - m)
-//     (fp64) is an exact power of two; the halves are merged at the end.
-//   Pass 2 (the same tiles again): p = 2^(x - m) (fp32) is written to a
-//     skewed 128 x 128 fp32 tile in shared memory -- element (t, c) at
-//     column (c - t) mod 128 -- so that thread c (< 128) reads key column c
-//     and thread 128 + u reads the two diagonals t - c = -u and 128 - u,
-//     both without bank conflicts.  Each reduction weighs row t by 1 / l_t
-//     in fp64 and adds its total to the key's column score or the offset's
-//     slash score.
+//     (fp32 within a tile, fp64 across tiles) is an exact power of two; the
+//     halves are merged at the end.
+//   Pass 2 (the same tiles again): p = 2^(x - m) / l (fp32) goes to a
+//     128 x 129 fp32 tile in shared memory (one word of padding per row), so
+//     that thread c (< 128) reads key column c and thread 128 + u reads the
+//     diagonals t - c = -u and 128 - u, all without bank conflicts.  The
+//     per-tile sums (fp32) are added to the key's column score and the
+//     offsets' slash scores with fp64 atomics.
 // The logits q.k of bf16 inputs are accumulated in fp32 by the tensor core.
 template <int D>
 struct SampleCfg {
   static constexpr int kHalfBytes = 128 * 128;               // 128 rows x 64 bf16
   static constexpr int kTileBytes = (D / 64) * kHalfBytes;   // Q or K tile
+  static constexpr int kPStride = 129;                       // floats per row of the P tile
   static constexpr int kQ = 0;
   static constexpr int kK = kQ + kTileBytes;
   static constexpr int kP = kK + 2 * kTileBytes;
-  static constexpr int kW = kP + 128 * 128 * 4;
-  static constexpr int kMl = kW + 128 * 8;                     // per-half (m, l) at the end of pass 1
+  static constexpr int kMl = kP + 128 * kPStride * 4;          // per-half (m, l) at the end of pass 1
   static constexpr int kBar = kMl + 2 * 128 * 16;
   static constexpr int kSlot = kBar + 2 * 8;
   static constexpr int kBytes = kSlot + 16;
@@ -67,11 +67,11 @@ __global__ void __launch_bounds__(kScoreThreads, 1) sample_scores_kernel(
     int G, int blk, int seg, float scale_log2, double* __restrict__ col, double* __restrict__ sl,
     int* __restrict__ err) {
   using C = SampleCfg<D>;
+  constexpr int PS = C::kPStride;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                          ~static_cast<uintptr_t>(1023));
   float* sP = reinterpret_cast<float*>(smem + C::kP);
-  double* sW = reinterpret_cast<double*>(smem + C::kW);
   float* sM = reinterpret_cast<float*>(smem + C::kMl);                   // [2][128]
   double* sL = reinterpret_cast<double*>(smem + C::kMl + 2 * 128 * 4);   // [2][128]
   uint64_t* bar_s = reinterpret_cast<uint64_t*>(smem + C::kBar);
@@ -135,8 +135,10 @@ __global__ void __launch_bounds__(kScoreThreads, 1) sample_scores_kernel(
   const bool row_ok = t < blk;
   float m = -INFINITY;                                         // integer-valued running maximum
   double l = 0.0;
+  float w = 0.f;                                               // 1 / l of this row (pass 2)
   uint32_t phase[2] = {0u, 0u};
   bool failed = false;
+  float* prow = sP + t * PS + hc * 64;
 
   for (int it = 0; it <= 2 * T; ++it) {
     if (it < 2 * T && warp == 0) {
@@ -163,27 +165,39 @@ __global__ void __launch_bounds__(kScoreThreads, 1) sample_scores_kernel(
       tc_fence_after();
       if (it + 1 < 2 * T) load_k((it + 1) % T, (it + 1) & 1);
       const int64_t k0 = static_cast<int64_t>(j) * 128;
-      // keys k0 + 64 hc + c with c <= lim are causal for this row
+      // every key of the tile is causal for every trunk row
+      const bool full = k0 + 127 <= qbase;
+      // otherwise keys k0 + 64 hc + c with c <= lim are causal for this row
       const int64_t lim64 = q_t - k0 - 64 * hc;
-      const int lim = row_ok ? static_cast<int>(lim64 > 63 ? 63 : (lim64 < -1 ? -1 : lim64)) : -1;
+      const int lim = static_cast<int>(lim64 > 63 ? 63 : (lim64 < -1 ? -1 : lim64));
       uint32_t r[64];
       tmem_ld64(tmem + lane_base + buf * 128 + hc * 64, r);
       if (jj < T) {
-        float mt = -INFINITY;
+        float mr = -INFINITY;                                  // max of the raw logits
+        if (full) {
 #pragma unroll
-        for (int c = 0; c < 64; ++c)
-          if (c <= lim) mt = fmaxf(mt, __uint_as_float(r[c]) * scale_log2);
-        if (mt > -INFINITY) {
-          const float mn = fmaxf(m, ceilf(mt));
+          for (int c = 0; c < 63; c += 2) mr = fmax3(mr, __uint_as_float(r[c]), __uint_as_float(r[c + 1]));
+        } else {
+#pragma unroll
+          for (int c = 0; c < 64; ++c)
+            if (c <= lim) mr = fmaxf(mr, __uint_as_float(r[c]));
+        }
+        if (mr > -INFINITY) {
+          const float mn = fmaxf(m, ceilf(mr * scale_log2));
           if (mn > m) {
             l = (m == -INFINITY) ? 0.0 : ldexp(l, static_cast<int>(m - mn));
             m = mn;
           }
-          double a[4] = {0.0, 0.0, 0.0, 0.0};
+          float a[4] = {0.f, 0.f, 0.f, 0.f};
+          if (full) {
 #pragma unroll
-          for (int c = 0; c < 64; ++c)
-            if (c <= lim) a[c % 4] += static_cast<double>(ex2(__uint_as_float(r[c]) * scale_log2 - m));
-          l += (a[0] + a[1]) + (a[2] + a[3]);
+            for (int c = 0; c < 64; ++c) a[c % 4] += ex2(fmaf(__uint_as_float(r[c]), scale_log2, -m));
+          } else {
+#pragma unroll
+            for (int c = 0; c < 64; ++c)
+              if (c <= lim) a[c % 4] += ex2(fmaf(__uint_as_float(r[c]), scale_log2, -m));
+          }
+          l += static_cast<double>((a[0] + a[1]) + (a[2] + a[3]));
         }
         if (jj == T - 1) {
           // merge the halves: the larger maximum, both sums rescaled by
@@ -197,45 +211,52 @@ __global__ void __launch_bounds__(kScoreThreads, 1) sample_scores_kernel(
           if (m0 > -INFINITY) lt += ldexp(sL[t], static_cast<int>(m0 - mm));
           if (m1 > -INFINITY) lt += ldexp(sL[128 + t], static_cast<int>(m1 - mm));
           m = mm;
-          if (hc == 0) sW[t] = row_ok && lt > 0.0 ? 1.0 / lt : 0.0;
+          w = row_ok && lt > 0.0 ? static_cast<float>(1.0 / lt) : 0.f;
         }
       } else {
+        if (full) {
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          const int cc = hc * 64 + c;
-          const float e = c <= lim ? ex2(__uint_as_float(r[c]) * scale_log2 - m) : 0.f;
-          sP[t * 128 + ((cc - t) & 127)] = e;
+          for (int c = 0; c < 64; ++c) prow[c] = ex2(fmaf(__uint_as_float(r[c]), scale_log2, -m)) * w;
+        } else {
+#pragma unroll
+          for (int c = 0; c < 64; ++c)
+            prow[c] = c <= lim ? ex2(fmaf(__uint_as_float(r[c]), scale_log2, -m)) * w : 0.f;
         }
         __syncthreads();
         const int x = tid & 127;
         const int64_t base = static_cast<int64_t>(bh) * N;
         if (tid < 128) {
-          // key column x: element (u, x) sits at column (x - u) mod 128
-          double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
-          for (int u = 0; u < blk; u += 4) {               // blk is a multiple of 4
-            a0 = fma(static_cast<double>(sP[u * 128 + ((x - u) & 127)]), sW[u], a0);
-            a1 = fma(static_cast<double>(sP[(u + 1) * 128 + ((x - u - 1) & 127)]), sW[u + 1], a1);
-            a2 = fma(static_cast<double>(sP[(u + 2) * 128 + ((x - u - 2) & 127)]), sW[u + 2], a2);
-            a3 = fma(static_cast<double>(sP[(u + 3) * 128 + ((x - u - 3) & 127)]), sW[u + 3], a3);
+          // key column x: rows u at u * PS + x
+          const float* pc = sP + x;
+          float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll 8
+          for (int u = 0; u < 128; u += 4) {
+            a0 += pc[u * PS];
+            a1 += pc[(u + 1) * PS];
+            a2 += pc[(u + 2) * PS];
+            a3 += pc[(u + 3) * PS];
           }
-          const double cs = (a0 + a1) + (a2 + a3);
+          const double cs = static_cast<double>((a0 + a1) + (a2 + a3));
           if (cs != 0.0 && k0 + x < N) atomicAdd(col + base + k0 + x, cs);
         } else {
-          // skew x: rows u < 128 - x lie on offset d0 - x, the rest on d0 + 128 - x
-          const int split = min(128 - x, blk);
-          double a0 = 0.0, a1 = 0.0, b0 = 0.0, b1 = 0.0;
+          // skew x: element (u, (u + x) mod 128) lies on offset d0 - x for
+          // u < 128 - x and on d0 + 128 - x after
+          const float* pd = sP + x;
+          const int split = 128 - x;
+          float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
           int u = 0;
           for (; u + 1 < split; u += 2) {
-            a0 = fma(static_cast<double>(sP[u * 128 + x]), sW[u], a0);
-            a1 = fma(static_cast<double>(sP[(u + 1) * 128 + x]), sW[u + 1], a1);
+            a0 += pd[u * (PS + 1)];
+            a1 += pd[(u + 1) * (PS + 1)];
           }
-          if (u < split) a0 = fma(static_cast<double>(sP[u * 128 + x]), sW[u], a0), ++u;
-          for (; u + 1 < blk; u += 2) {
-            b0 = fma(static_cast<double>(sP[u * 128 + x]), sW[u], b0);
-            b1 = fma(static_cast<double>(sP[(u + 1) * 128 + x]), sW[u + 1], b1);
+          if (u < split) a0 += pd[u * (PS + 1)], ++u;
+          const float* pe = pd - 128;
+          for (; u + 1 < 128; u += 2) {
+            b0 += pe[u * (PS + 1)];
+            b1 += pe[(u + 1) * (PS + 1)];
           }
-          if (u < blk) b0 = fma(static_cast<double>(sP[u * 128 + x]), sW[u], b0);
-          const double da = a0 + a1, db = b0 + b1;
+          if (u < 128) b0 += pe[u * (PS + 1)];
+          const double da = static_cast<double>(a0 + a1), db = static_cast<double>(b0 + b1);
           const int64_t d0 = qbase - k0;
           if (da != 0.0 && d0 - x >= 0 && d0 - x < N) atomicAdd(sl + base + d0 - x, da);
           if (db != 0.0 && d0 + 128 - x >= 0 && d0 + 128 - x < N) atomicAdd(sl + base + d0 + 128 - x, db);
