@@ -24,41 +24,51 @@ namespace {
 
 constexpr int kSampleWarps = 8;
 
-// Stage 1 on the tensor cores.  One CTA of 256 threads per (trunk s, hq, b),
+// Stage 1 on the tensor cores.  One CTA of 512 threads per (trunk s, hq, b),
 // heaviest trunks first.  The trunk's rows (the last blk queries of segment
 // s, zero rows up to 128) stay in shared memory; the keys 0 .. seg_end - 1
 // stream through in tiles of 128, and S = Q_trunk K_tile^T is computed by
 // tcgen05.mma into one of two tensor-memory buffers while the previous tile
-// is processed and the next one is copied in.  Warp w reads tensor-memory
-// lanes 32 (w mod 4) .. +31 (trunk rows) and columns 64 (w / 4) .. +63, so
-// each row has two threads, one per column half.
-//   Pass 1 (tiles 0 .. T-1): per row and half the running maximum m of
+// is processed; key tiles are copied in two tiles ahead through a ring of
+// three shared-memory buffers.  Warp w reads tensor-memory lanes
+// 32 (w mod 4) .. +31 (trunk rows) and columns 32 (w / 4) .. +31, so each
+// row has four threads, one per column quarter.
+//   Pass 1 (tiles 0 .. T-1): per row and quarter the running maximum m of
 //     x = S * log2(e) / sqrt(d) over the causal keys, kept rounded up to an
 //     integer so that every rescale of the running sum l = sum 2^(x - m)
 //     (fp32 within a tile, fp64 across tiles) is an exact power of two; the
-//     halves are merged at the end.
+//     quarters are merged at the end.
 //   Pass 2 (the same tiles again): p = 2^(x - m) / l (fp32) goes to a
-//     128 x 129 fp32 tile in shared memory (one word of padding per row), so
-//     that thread c (< 128) reads key column c and thread 128 + u reads the
-//     diagonals t - c = -u and 128 - u, all without bank conflicts.  The
-//     per-tile sums (fp32) are added to the key's column score and the
-//     offsets' slash scores with fp64 atomics.
+//     128 x 129 fp32 tile in shared memory (one word of padding per row).
+//     Threads 0-255 sum key columns (two threads per column, one per half
+//     of the rows), threads 256-511 sum the diagonals t - c = -u and 128 - u
+//     of skew u (two threads per skew, again by row halves); all these
+//     reads are free of bank conflicts.  The halves meet in shared memory
+//     and each per-tile sum (fp32) is added to the key's column score or
+//     the offset's slash score with one fp64 atomic.
 // The logits q.k of bf16 inputs are accumulated in fp32 by the tensor core.
 template <int D>
 struct SampleCfg {
   static constexpr int kHalfBytes = 128 * 128;               // 128 rows x 64 bf16
   static constexpr int kTileBytes = (D / 64) * kHalfBytes;   // Q or K tile
   static constexpr int kPStride = 129;                       // floats per row of the P tile
+  static constexpr int kStages = 3;                           // key tile ring
   static constexpr int kQ = 0;
   static constexpr int kK = kQ + kTileBytes;
-  static constexpr int kP = kK + 2 * kTileBytes;
-  static constexpr int kMl = kP + 128 * kPStride * 4;          // per-half (m, l) at the end of pass 1
-  static constexpr int kBar = kMl + 2 * 128 * 16;
+  static constexpr int kP = kK + kStages * kTileBytes;
+  static constexpr int kMl = kP + 128 * kPStride * 4;          // per-quarter (m, l) at the end of pass 1
+  static constexpr int kHalf = kMl + 4 * 128 * 12;             // second-half partial sums
+  static constexpr int kBar = kHalf + 3 * 128 * 4;
   static constexpr int kSlot = kBar + 2 * 8;
   static constexpr int kBytes = kSlot + 16;
   static constexpr int kSmem = kBytes + 1024;                // alignment slack
 };
-constexpr int kScoreThreads = 256;
+constexpr int kScoreThreads = 512;
+
+// Wait until at most one of this thread's cp.async groups is pending.
+__device__ __forceinline__ void cp_async_wait_group1() {
+  asm volatile("cp.async.wait_group 1;" ::: "memory");
+}
 
 template <int D>
 __global__ void __launch_bounds__(kScoreThreads, 1) sample_scores_kernel(
@@ -72,15 +82,16 @@ __global__ void __launch_bounds__(kScoreThreads, 1) sample_scores_kernel(
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                          ~static_cast<uintptr_t>(1023));
   float* sP = reinterpret_cast<float*>(smem + C::kP);
-  float* sM = reinterpret_cast<float*>(smem + C::kMl);                   // [2][128]
-  double* sL = reinterpret_cast<double*>(smem + C::kMl + 2 * 128 * 4);   // [2][128]
+  double* sL = reinterpret_cast<double*>(smem + C::kMl);                 // [4][128]
+  float* sM = reinterpret_cast<float*>(smem + C::kMl + 4 * 128 * 8);     // [4][128]
+  float* sH = reinterpret_cast<float*>(smem + C::kHalf);                 // [3][128]
   uint64_t* bar_s = reinterpret_cast<uint64_t*>(smem + C::kBar);
   uint32_t* slot = reinterpret_cast<uint32_t*>(smem + C::kSlot);
   const uint32_t sQ = smem_u32(smem + C::kQ), sK = smem_u32(smem + C::kK);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int t = (warp & 3) * 32 + lane;                        // trunk row of this thread
-  const int hc = warp >> 2;                                    // column half
+  const int qc = warp >> 2;                                    // column quarter
   const int nseg = static_cast<int>((N + seg - 1) / seg);
   const int BH = B * Hq;
   const int s = nseg - 1 - static_cast<int>(blockIdx.x / BH);
@@ -122,6 +133,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1) sample_scores_kernel(
   }
   load_k(0, 0);
   load_k(1 % T, 1);
+  load_k(2 % T, 2);
   cp_async_wait_all();
   fence_proxy_async();
   tc_fence_before();
@@ -138,14 +150,15 @@ __global__ void __launch_bounds__(kScoreThreads, 1) sample_scores_kernel(
   float w = 0.f;                                               // 1 / l of this row (pass 2)
   uint32_t phase[2] = {0u, 0u};
   bool failed = false;
-  float* prow = sP + t * PS + hc * 64;
+  float* prow = sP + t * PS + qc * 32;
+  const int role = tid >> 7, x = tid & 127;                    // reduction role and its index
 
   for (int it = 0; it <= 2 * T; ++it) {
     if (it < 2 * T && warp == 0) {
       const int buf = it & 1;
       tc_fence_after();
       const uint64_t a0 = sdesc_sw128(sQ, 16, 1024);
-      const uint64_t b0 = sdesc_sw128(sK + buf * C::kTileBytes, 16, 1024);
+      const uint64_t b0 = sdesc_sw128(sK + (it % C::kStages) * C::kTileBytes, 16, 1024);
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
         const uint32_t off = (kk / 4) * C::kHalfBytes + (kk % 4) * 32;
@@ -163,23 +176,25 @@ __global__ void __launch_bounds__(kScoreThreads, 1) sample_scores_kernel(
         break;
       }
       tc_fence_after();
-      if (it + 1 < 2 * T) load_k((it + 1) % T, (it + 1) & 1);
+      // the ring slot of MMA it - 1 is free: copy the tile of MMA it + 2
+      if (it + 2 < 2 * T) load_k((it + 2) % T, (it + 2) % C::kStages);
+      else cp_async_commit();                                  // empty group keeps the count
       const int64_t k0 = static_cast<int64_t>(j) * 128;
       // every key of the tile is causal for every trunk row
       const bool full = k0 + 127 <= qbase;
-      // otherwise keys k0 + 64 hc + c with c <= lim are causal for this row
-      const int64_t lim64 = q_t - k0 - 64 * hc;
-      const int lim = static_cast<int>(lim64 > 63 ? 63 : (lim64 < -1 ? -1 : lim64));
-      uint32_t r[64];
-      tmem_ld64(tmem + lane_base + buf * 128 + hc * 64, r);
+      // otherwise keys k0 + 32 qc + c with c <= lim are causal for this row
+      const int64_t lim64 = q_t - k0 - 32 * qc;
+      const int lim = static_cast<int>(lim64 > 31 ? 31 : (lim64 < -1 ? -1 : lim64));
+      uint32_t r[32];
+      tmem_ld32(tmem + lane_base + buf * 128 + qc * 32, r);
       if (jj < T) {
         float mr = -INFINITY;                                  // max of the raw logits
         if (full) {
 #pragma unroll
-          for (int c = 0; c < 63; c += 2) mr = fmax3(mr, __uint_as_float(r[c]), __uint_as_float(r[c + 1]));
+          for (int c = 0; c < 31; c += 2) mr = fmax3(mr, __uint_as_float(r[c]), __uint_as_float(r[c + 1]));
         } else {
 #pragma unroll
-          for (int c = 0; c < 64; ++c)
+          for (int c = 0; c < 32; ++c)
             if (c <= lim) mr = fmaxf(mr, __uint_as_float(r[c]));
         }
         if (mr > -INFINITY) {
@@ -191,79 +206,98 @@ __global__ void __launch_bounds__(kScoreThreads, 1) sample_scores_kernel(
           float a[4] = {0.f, 0.f, 0.f, 0.f};
           if (full) {
 #pragma unroll
-            for (int c = 0; c < 64; ++c) a[c % 4] += ex2(fmaf(__uint_as_float(r[c]), scale_log2, -m));
+            for (int c = 0; c < 32; ++c) a[c % 4] += ex2(fmaf(__uint_as_float(r[c]), scale_log2, -m));
           } else {
 #pragma unroll
-            for (int c = 0; c < 64; ++c)
+            for (int c = 0; c < 32; ++c)
               if (c <= lim) a[c % 4] += ex2(fmaf(__uint_as_float(r[c]), scale_log2, -m));
           }
           l += static_cast<double>((a[0] + a[1]) + (a[2] + a[3]));
         }
         if (jj == T - 1) {
-          // merge the halves: the larger maximum, both sums rescaled by
-          // exact powers of two
-          sM[hc * 128 + t] = m;
-          sL[hc * 128 + t] = l;
+          // merge the quarters: the largest maximum, every sum rescaled by
+          // an exact power of two
+          sM[qc * 128 + t] = m;
+          sL[qc * 128 + t] = l;
           __syncthreads();
-          const float m0 = sM[t], m1 = sM[128 + t];
-          const float mm = fmaxf(m0, m1);
+          float mm = -INFINITY;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) mm = fmaxf(mm, sM[q * 128 + t]);
           double lt = 0.0;
-          if (m0 > -INFINITY) lt += ldexp(sL[t], static_cast<int>(m0 - mm));
-          if (m1 > -INFINITY) lt += ldexp(sL[128 + t], static_cast<int>(m1 - mm));
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float mq = sM[q * 128 + t];
+            if (mq > -INFINITY) lt += ldexp(sL[q * 128 + t], static_cast<int>(mq - mm));
+          }
           m = mm;
           w = row_ok && lt > 0.0 ? static_cast<float>(1.0 / lt) : 0.f;
         }
       } else {
         if (full) {
 #pragma unroll
-          for (int c = 0; c < 64; ++c) prow[c] = ex2(fmaf(__uint_as_float(r[c]), scale_log2, -m)) * w;
+          for (int c = 0; c < 32; ++c) prow[c] = ex2(fmaf(__uint_as_float(r[c]), scale_log2, -m)) * w;
         } else {
 #pragma unroll
-          for (int c = 0; c < 64; ++c)
+          for (int c = 0; c < 32; ++c)
             prow[c] = c <= lim ? ex2(fmaf(__uint_as_float(r[c]), scale_log2, -m)) * w : 0.f;
         }
         __syncthreads();
-        const int x = tid & 127;
-        const int64_t base = static_cast<int64_t>(bh) * N;
-        if (tid < 128) {
+        const int u0 = (role & 1) * 64, u1 = u0 + 64;          // this thread's half of the rows
+        float ca = 0.f, cb = 0.f;                              // column, or the two diagonals
+        if (role < 2) {
           // key column x: rows u at u * PS + x
           const float* pc = sP + x;
           float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-#pragma unroll 8
-          for (int u = 0; u < 128; u += 4) {
+#pragma unroll 4
+          for (int u = u0; u < u1; u += 4) {
             a0 += pc[u * PS];
             a1 += pc[(u + 1) * PS];
             a2 += pc[(u + 2) * PS];
             a3 += pc[(u + 3) * PS];
           }
-          const double cs = static_cast<double>((a0 + a1) + (a2 + a3));
-          if (cs != 0.0 && k0 + x < N) atomicAdd(col + base + k0 + x, cs);
+          ca = (a0 + a1) + (a2 + a3);
         } else {
           // skew x: element (u, (u + x) mod 128) lies on offset d0 - x for
           // u < 128 - x and on d0 + 128 - x after
+          const int split = min(max(128 - x, u0), u1);
           const float* pd = sP + x;
-          const int split = 128 - x;
+          const float* pe = pd - 128;
           float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
-          int u = 0;
+          int u = u0;
           for (; u + 1 < split; u += 2) {
             a0 += pd[u * (PS + 1)];
             a1 += pd[(u + 1) * (PS + 1)];
           }
           if (u < split) a0 += pd[u * (PS + 1)], ++u;
-          const float* pe = pd - 128;
-          for (; u + 1 < 128; u += 2) {
+          for (; u + 1 < u1; u += 2) {
             b0 += pe[u * (PS + 1)];
             b1 += pe[(u + 1) * (PS + 1)];
           }
-          if (u < 128) b0 += pe[u * (PS + 1)];
-          const double da = static_cast<double>(a0 + a1), db = static_cast<double>(b0 + b1);
+          if (u < u1) b0 += pe[u * (PS + 1)];
+          ca = a0 + a1;
+          cb = b0 + b1;
+        }
+        // second row halves hand their sums to the first
+        if (role == 1) sH[x] = ca;
+        if (role == 3) {
+          sH[128 + x] = ca;
+          sH[256 + x] = cb;
+        }
+        __syncthreads();
+        const int64_t base = static_cast<int64_t>(bh) * N;
+        if (role == 0) {
+          const double cs = static_cast<double>(ca + sH[x]);
+          if (cs != 0.0 && k0 + x < N) atomicAdd(col + base + k0 + x, cs);
+        } else if (role == 2) {
+          const double da = static_cast<double>(ca + sH[128 + x]), db = static_cast<double>(cb + sH[256 + x]);
           const int64_t d0 = qbase - k0;
           if (da != 0.0 && d0 - x >= 0 && d0 - x < N) atomicAdd(sl + base + d0 - x, da);
           if (db != 0.0 && d0 + 128 - x >= 0 && d0 + 128 - x < N) atomicAdd(sl + base + d0 + 128 - x, db);
         }
       }
     }
-    cp_async_wait_all();
+    // the tile of MMA it + 1 (copied one iteration earlier) has landed
+    if (it >= 1) cp_async_wait_group1();
     fence_proxy_async();
     tc_fence_before();
     __syncthreads();
