@@ -24,51 +24,49 @@ namespace {
 
 constexpr int kSampleWarps = 8;
 
-// Stage 1 on the tensor cores.  One CTA of 512 threads per (trunk s, hq, b),
-// heaviest trunks first.  The trunk's rows (the last blk queries of segment
-// s, zero rows up to 128) stay in shared memory; the keys 0 .. seg_end - 1
-// stream through in tiles of 128, and S = Q_trunk K_tile^T is computed by
-// tcgen05.mma into one of two tensor-memory buffers while the previous tile
-// is processed; key tiles are copied in two tiles ahead through a ring of
-// three shared-memory buffers.  Warp w reads tensor-memory lanes
-// 32 (w mod 4) .. +31 (trunk rows) and columns 32 (w / 4) .. +31, so each
-// row has four threads, one per column quarter.
-//   Pass 1 (tiles 0 .. T-1): per row and quarter the running maximum m of
-//     x = S * log2(e) / sqrt(d) over the causal keys, kept rounded up to an
-//     integer so that every rescale of the running sum l = sum 2^(x - m)
-//     (fp32 within a tile, fp64 across tiles) is an exact power of two; the
-//     quarters are merged at the end.
-//   Pass 2 (the same tiles again): p = 2^(x - m) / l (fp32) goes to a
-//     128 x 129 fp32 tile in shared memory (one word of padding per row).
-//     Threads 0-255 sum key columns (two threads per column, one per half
-//     of the rows), threads 256-511 sum the diagonals t - c = -u and 128 - u
-//     of skew u (two threads per skew, again by row halves); all these
-//     reads are free of bank conflicts.  The halves meet in shared memory
-//     and each per-tile sum (fp32) is added to the key's column score or
-//     the offset's slash score with one fp64 atomic.
+// Stage 1 on the tensor cores.  One CTA per (trunk s, hq, b), heaviest
+// trunks first.  The trunk's rows (the last blk queries of segment s, zero
+// rows up to 128) stay in shared memory; the keys 0 .. seg_end - 1 stream
+// through twice in tiles of 128 (pass 1, then pass 2).  Warp-specialized:
+//   warp 0      issues S = Q_trunk K_tile^T (tcgen05.mma) into a ring of
+//               four tensor-memory buffers, as far ahead as the buffers and
+//               the key ring allow;
+//   warps 1-3   copy key tiles (cp.async) into a ring of three shared-memory
+//               slots;
+//   warps 4-11  read S: warp 4 + w takes tensor-memory lanes 32 (w mod 4)
+//               .. +31 (trunk rows) and columns 64 (w / 4) .. +63.
+//   Pass 1: per row and half the running maximum m of x = S log2(e)/sqrt(d)
+//     over the causal keys, kept rounded up to an integer so that every
+//     rescale of the running sum l = sum 2^(x - m) (fp32 within a tile, fp64
+//     across tiles) is an exact power of two; the halves merge at the end.
+//   Pass 2: p = 2^(x - m) / l (fp32) goes to a 128 x 129 fp32 tile in shared
+//     memory (one word of padding per row); consumer thread c < 128 sums key
+//     column c and thread 128 + u the diagonals t - c = -u and 128 - u of
+//     skew u, all without bank conflicts, and each per-tile sum is added to
+//     the key's column score or the offset's slash score with one fp64
+//     atomic.
 // The logits q.k of bf16 inputs are accumulated in fp32 by the tensor core.
+// Every wait is bounded; a shared abort flag ends all roles together.
 template <int D>
 struct SampleCfg {
   static constexpr int kHalfBytes = 128 * 128;               // 128 rows x 64 bf16
   static constexpr int kTileBytes = (D / 64) * kHalfBytes;   // Q or K tile
   static constexpr int kPStride = 129;                       // floats per row of the P tile
   static constexpr int kStages = 3;                           // key tile ring
+  static constexpr int kSBufs = 4;                            // S buffers in tensor memory
   static constexpr int kQ = 0;
   static constexpr int kK = kQ + kTileBytes;
   static constexpr int kP = kK + kStages * kTileBytes;
-  static constexpr int kMl = kP + 128 * kPStride * 4;          // per-quarter (m, l) at the end of pass 1
-  static constexpr int kHalf = kMl + 4 * 128 * 12;             // second-half partial sums
-  static constexpr int kBar = kHalf + 3 * 128 * 4;
-  static constexpr int kSlot = kBar + 2 * 8;
+  static constexpr int kMl = kP + 128 * kPStride * 4;          // per-half (m, l) at the end of pass 1
+  static constexpr int kBar = kMl + 2 * 128 * 12;
+  static constexpr int kNBar = 1 + 2 * kStages + 2 * kSBufs;
+  static constexpr int kSlot = kBar + kNBar * 8;
   static constexpr int kBytes = kSlot + 16;
   static constexpr int kSmem = kBytes + 1024;                // alignment slack
 };
-constexpr int kScoreThreads = 512;
-
-// Wait until at most one of this thread's cp.async groups is pending.
-__device__ __forceinline__ void cp_async_wait_group1() {
-  asm volatile("cp.async.wait_group 1;" ::: "memory");
-}
+constexpr int kScoreThreads = 384;
+constexpr int kScoreProducers = 96;                           // warps 1-3
+constexpr int kScoreConsumers = 256;                          // warps 4-11
 
 template <int D>
 __global__ void __launch_bounds__(kScoreThreads, 1) sample_scores_kernel(
@@ -77,21 +75,24 @@ __global__ void __launch_bounds__(kScoreThreads, 1) sample_scores_kernel(
     int G, int blk, int seg, float scale_log2, double* __restrict__ col, double* __restrict__ sl,
     int* __restrict__ err) {
   using C = SampleCfg<D>;
-  constexpr int PS = C::kPStride;
+  constexpr int PS = C::kPStride, NK = C::kStages, NS = C::kSBufs;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                          ~static_cast<uintptr_t>(1023));
   float* sP = reinterpret_cast<float*>(smem + C::kP);
-  double* sL = reinterpret_cast<double*>(smem + C::kMl);                 // [4][128]
-  float* sM = reinterpret_cast<float*>(smem + C::kMl + 4 * 128 * 8);     // [4][128]
-  float* sH = reinterpret_cast<float*>(smem + C::kHalf);                 // [3][128]
-  uint64_t* bar_s = reinterpret_cast<uint64_t*>(smem + C::kBar);
+  double* sL = reinterpret_cast<double*>(smem + C::kMl);                 // [2][128]
+  float* sM = reinterpret_cast<float*>(smem + C::kMl + 2 * 128 * 8);     // [2][128]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBar);
+  uint64_t* bar_q = bars;
+  uint64_t* bar_kfull = bars + 1;
+  uint64_t* bar_kempty = bar_kfull + NK;
+  uint64_t* bar_sfull = bar_kempty + NK;
+  uint64_t* bar_sfree = bar_sfull + NS;
   uint32_t* slot = reinterpret_cast<uint32_t*>(smem + C::kSlot);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kSlot + 4);
   const uint32_t sQ = smem_u32(smem + C::kQ), sK = smem_u32(smem + C::kK);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int t = (warp & 3) * 32 + lane;                        // trunk row of this thread
-  const int qc = warp >> 2;                                    // column quarter
   const int nseg = static_cast<int>((N + seg - 1) / seg);
   const int BH = B * Hq;
   const int s = nseg - 1 - static_cast<int>(blockIdx.x / BH);
@@ -100,101 +101,123 @@ __global__ void __launch_bounds__(kScoreThreads, 1) sample_scores_kernel(
   const int64_t seg_end = min(static_cast<int64_t>(s + 1) * seg, N);
   const int64_t qbase = seg_end - blk;
   const int T = static_cast<int>((seg_end + 127) / 128);
+  const int n_it = 2 * T;                                      // MMAs: pass 1 then pass 2
   constexpr int CH = D / 8;                                    // 16-byte chunks per row
 
-  const __nv_bfloat16* qb = Q + b * qsB + hq * qsH;
-  const __nv_bfloat16* kb = K + b * ksB + (hq / G) * ksH;
-  auto load_k = [&](int j, int buf) {
-    const int64_t k0 = static_cast<int64_t>(j) * 128;
-    const uint32_t dst = sK + buf * C::kTileBytes;
-    for (int id = tid; id < 128 * CH; id += kScoreThreads) {
-      const int r = id / CH, c = id % CH;
-      const bool valid = k0 + r < seg_end;
-      cp_async16_zfill(dst + (c / 8) * C::kHalfBytes + sw128_offset(r, c % 8),
-                       valid ? kb + (k0 + r) * ksN + c * 8 : kb, valid);
-    }
-    cp_async_commit();
-  };
-
   if (warp == 0) {
-    tmem_alloc(slot, 256);
+    tmem_alloc(slot, 512);
     tmem_relinquish();
   }
   if (tid == 0) {
-    mbar_init(&bar_s[0], 1);
-    mbar_init(&bar_s[1], 1);
+    mbar_init(bar_q, kScoreProducers);
+    for (int i = 0; i < NK; ++i) {
+      mbar_init(&bar_kfull[i], kScoreProducers);
+      mbar_init(&bar_kempty[i], 1);
+    }
+    for (int i = 0; i < NS; ++i) {
+      mbar_init(&bar_sfull[i], 1);
+      mbar_init(&bar_sfree[i], kScoreConsumers / 32);
+    }
+    *abort_flag = 0;
     fence_mbar_init();
   }
-  for (int id = tid; id < 128 * CH; id += kScoreThreads) {
-    const int r = id / CH, c = id % CH;
-    const bool valid = r < blk;
-    cp_async16_zfill(sQ + (c / 8) * C::kHalfBytes + sw128_offset(r, c % 8),
-                     valid ? qb + (qbase + r) * qsN + c * 8 : qb, valid);
-  }
-  load_k(0, 0);
-  load_k(1 % T, 1);
-  load_k(2 % T, 2);
-  cp_async_wait_all();
-  fence_proxy_async();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *slot;
-  const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-  constexpr uint32_t idesc = idesc_bf16(128, 128, false);
 
-  const int64_t q_t = qbase + t;
-  const bool row_ok = t < blk;
-  float m = -INFINITY;                                         // integer-valued running maximum
-  double l = 0.0;
-  float w = 0.f;                                               // 1 / l of this row (pass 2)
-  uint32_t phase[2] = {0u, 0u};
-  bool failed = false;
-  float* prow = sP + t * PS + qc * 32;
-  const int role = tid >> 7, x = tid & 127;                    // reduction role and its index
-
-  for (int it = 0; it <= 2 * T; ++it) {
-    if (it < 2 * T && warp == 0) {
-      const int buf = it & 1;
-      tc_fence_after();
-      const uint64_t a0 = sdesc_sw128(sQ, 16, 1024);
-      const uint64_t b0 = sdesc_sw128(sK + (it % C::kStages) * C::kTileBytes, 16, 1024);
-#pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        const uint32_t off = (kk / 4) * C::kHalfBytes + (kk % 4) * 32;
-        if (elect_one()) mma_ss(tmem + buf * 128, sdesc_add(a0, off), sdesc_add(b0, off), idesc, kk > 0 ? 1u : 0u);
-      }
-      if (elect_one()) tc_commit(&bar_s[buf]);
-      __syncwarp();
-    }
-    if (it >= 1) {
-      const int jj = it - 1, buf = jj & 1, j = jj % T;
-      const bool ok = mbar_wait(&bar_s[buf], phase[buf], err);
-      phase[buf] ^= 1u;
-      if (__syncthreads_or(!ok)) {
-        failed = true;
+  if (warp == 0) {
+    // ---------------------------------------------------------------- MMA
+    constexpr uint32_t idesc = idesc_bf16(128, 128, false);
+    // every lane waits; the warp goes on only if all of them saw the phase
+    bool ok = __all_sync(0xffffffffu, mbar_wait_or_abort(bar_q, 0, err, abort_flag));
+    for (int it = 0; ok && it < n_it; ++it) {
+      const int ks = it % NK, sb = it % NS;
+      ok = mbar_wait_or_abort(&bar_kfull[ks], (it / NK) & 1, err, abort_flag);
+      if (ok && it >= NS) ok = mbar_wait_or_abort(&bar_sfree[sb], ((it / NS) - 1) & 1, err, abort_flag);
+      if (!__all_sync(0xffffffffu, ok)) {
+        *abort_flag = 1;
         break;
       }
       tc_fence_after();
-      // the ring slot of MMA it - 1 is free: copy the tile of MMA it + 2
-      if (it + 2 < 2 * T) load_k((it + 2) % T, (it + 2) % C::kStages);
-      else cp_async_commit();                                  // empty group keeps the count
+      const uint64_t a0 = sdesc_sw128(sQ, 16, 1024);
+      const uint64_t b0 = sdesc_sw128(sK + ks * C::kTileBytes, 16, 1024);
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = (kk / 4) * C::kHalfBytes + (kk % 4) * 32;
+        if (elect_one()) mma_ss(tmem + sb * 128, sdesc_add(a0, off), sdesc_add(b0, off), idesc, kk > 0 ? 1u : 0u);
+      }
+      if (elect_one()) {
+        tc_commit(&bar_sfull[sb]);
+        tc_commit(&bar_kempty[ks]);
+      }
+      __syncwarp();
+    }
+  } else if (warp < 4) {
+    // ----------------------------------------------------------- producers
+    const int pt = tid - 32;
+    const __nv_bfloat16* qb = Q + b * qsB + hq * qsH;
+    const __nv_bfloat16* kb = K + b * ksB + (hq / G) * ksH;
+    for (int id = pt; id < 128 * CH; id += kScoreProducers) {
+      const int r = id / CH, c = id % CH;
+      const bool valid = r < blk;
+      cp_async16_zfill(sQ + (c / 8) * C::kHalfBytes + sw128_offset(r, c % 8),
+                       valid ? qb + (qbase + r) * qsN + c * 8 : qb, valid);
+    }
+    cp_async_mbar_arrive(bar_q);
+    for (int it = 0; it < n_it; ++it) {
+      const int ks = it % NK;
+      if (it >= NK && !mbar_wait_or_abort(&bar_kempty[ks], ((it / NK) - 1) & 1, err, abort_flag)) break;
+      const int64_t k0 = static_cast<int64_t>(it % T) * 128;
+      const uint32_t dst = sK + ks * C::kTileBytes;
+      for (int id = pt; id < 128 * CH; id += kScoreProducers) {
+        const int r = id / CH, c = id % CH;
+        const bool valid = k0 + r < seg_end;
+        cp_async16_zfill(dst + (c / 8) * C::kHalfBytes + sw128_offset(r, c % 8),
+                         valid ? kb + (k0 + r) * ksN + c * 8 : kb, valid);
+      }
+      cp_async_mbar_arrive(&bar_kfull[ks]);
+    }
+    cp_async_wait_all();
+  } else {
+    // ----------------------------------------------------------- consumers
+    const int ct = tid - 128, cw = ct >> 5;
+    const int t = (cw & 3) * 32 + lane;                        // trunk row of this thread
+    const int hc = cw >> 2;                                    // column half
+    const uint32_t lane_base = static_cast<uint32_t>((cw & 3) * 32) << 16;
+    const int64_t q_t = qbase + t;
+    const bool row_ok = t < blk;
+    float m = -INFINITY;                                       // integer-valued running maximum
+    double l = 0.0;
+    float w = 0.f;                                             // 1 / l of this row (pass 2)
+    float* prow = sP + t * PS + hc * 64;
+    const int x = ct & 127;
+    const int64_t base = static_cast<int64_t>(bh) * N;
+    for (int it = 0; it < n_it; ++it) {
+      const int sb = it % NS, j = it % T;
+      const bool ok = mbar_wait_or_abort(&bar_sfull[sb], (it / NS) & 1, err, abort_flag);
+      if (named_sync_or(1, kScoreConsumers, !ok)) break;
+      tc_fence_after();
+      uint32_t r[64];
+      tmem_ld32(tmem + lane_base + sb * 128 + hc * 64, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+      tmem_ld32(tmem + lane_base + sb * 128 + hc * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar_sfree[sb]);
       const int64_t k0 = static_cast<int64_t>(j) * 128;
       // every key of the tile is causal for every trunk row
       const bool full = k0 + 127 <= qbase;
-      // otherwise keys k0 + 32 qc + c with c <= lim are causal for this row
-      const int64_t lim64 = q_t - k0 - 32 * qc;
-      const int lim = static_cast<int>(lim64 > 31 ? 31 : (lim64 < -1 ? -1 : lim64));
-      uint32_t r[32];
-      tmem_ld32(tmem + lane_base + buf * 128 + qc * 32, r);
-      if (jj < T) {
+      // otherwise keys k0 + 64 hc + c with c <= lim are causal for this row
+      const int64_t lim64 = q_t - k0 - 64 * hc;
+      const int lim = static_cast<int>(lim64 > 63 ? 63 : (lim64 < -1 ? -1 : lim64));
+      if (it < T) {
         float mr = -INFINITY;                                  // max of the raw logits
         if (full) {
 #pragma unroll
-          for (int c = 0; c < 31; c += 2) mr = fmax3(mr, __uint_as_float(r[c]), __uint_as_float(r[c + 1]));
+          for (int c = 0; c < 63; c += 2) mr = fmax3(mr, __uint_as_float(r[c]), __uint_as_float(r[c + 1]));
         } else {
 #pragma unroll
-          for (int c = 0; c < 32; ++c)
+          for (int c = 0; c < 64; ++c)
             if (c <= lim) mr = fmaxf(mr, __uint_as_float(r[c]));
         }
         if (mr > -INFINITY) {
@@ -206,108 +229,83 @@ __global__ void __launch_bounds__(kScoreThreads, 1) sample_scores_kernel(
           float a[4] = {0.f, 0.f, 0.f, 0.f};
           if (full) {
 #pragma unroll
-            for (int c = 0; c < 32; ++c) a[c % 4] += ex2(fmaf(__uint_as_float(r[c]), scale_log2, -m));
+            for (int c = 0; c < 64; ++c) a[c % 4] += ex2(fmaf(__uint_as_float(r[c]), scale_log2, -m));
           } else {
 #pragma unroll
-            for (int c = 0; c < 32; ++c)
+            for (int c = 0; c < 64; ++c)
               if (c <= lim) a[c % 4] += ex2(fmaf(__uint_as_float(r[c]), scale_log2, -m));
           }
           l += static_cast<double>((a[0] + a[1]) + (a[2] + a[3]));
         }
-        if (jj == T - 1) {
-          // merge the quarters: the largest maximum, every sum rescaled by
-          // an exact power of two
-          sM[qc * 128 + t] = m;
-          sL[qc * 128 + t] = l;
-          __syncthreads();
-          float mm = -INFINITY;
-#pragma unroll
-          for (int q = 0; q < 4; ++q) mm = fmaxf(mm, sM[q * 128 + t]);
+        if (it == T - 1) {
+          // merge the halves: the larger maximum, both sums rescaled by
+          // exact powers of two
+          sM[hc * 128 + t] = m;
+          sL[hc * 128 + t] = l;
+          named_sync(1, kScoreConsumers);
+          const float m0 = sM[t], m1 = sM[128 + t];
+          const float mm = fmaxf(m0, m1);
           double lt = 0.0;
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const float mq = sM[q * 128 + t];
-            if (mq > -INFINITY) lt += ldexp(sL[q * 128 + t], static_cast<int>(mq - mm));
-          }
+          if (m0 > -INFINITY) lt += ldexp(sL[t], static_cast<int>(m0 - mm));
+          if (m1 > -INFINITY) lt += ldexp(sL[128 + t], static_cast<int>(m1 - mm));
           m = mm;
           w = row_ok && lt > 0.0 ? static_cast<float>(1.0 / lt) : 0.f;
         }
       } else {
         if (full) {
 #pragma unroll
-          for (int c = 0; c < 32; ++c) prow[c] = ex2(fmaf(__uint_as_float(r[c]), scale_log2, -m)) * w;
+          for (int c = 0; c < 64; ++c) prow[c] = ex2(fmaf(__uint_as_float(r[c]), scale_log2, -m)) * w;
         } else {
 #pragma unroll
-          for (int c = 0; c < 32; ++c)
+          for (int c = 0; c < 64; ++c)
             prow[c] = c <= lim ? ex2(fmaf(__uint_as_float(r[c]), scale_log2, -m)) * w : 0.f;
         }
-        __syncthreads();
-        const int u0 = (role & 1) * 64, u1 = u0 + 64;          // this thread's half of the rows
-        float ca = 0.f, cb = 0.f;                              // column, or the two diagonals
-        if (role < 2) {
+        named_sync(1, kScoreConsumers);
+        if (ct < 128) {
           // key column x: rows u at u * PS + x
           const float* pc = sP + x;
           float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-#pragma unroll 4
-          for (int u = u0; u < u1; u += 4) {
+#pragma unroll 8
+          for (int u = 0; u < 128; u += 4) {
             a0 += pc[u * PS];
             a1 += pc[(u + 1) * PS];
             a2 += pc[(u + 2) * PS];
             a3 += pc[(u + 3) * PS];
           }
-          ca = (a0 + a1) + (a2 + a3);
+          const double cs = static_cast<double>((a0 + a1) + (a2 + a3));
+          if (cs != 0.0 && k0 + x < N) atomicAdd(col + base + k0 + x, cs);
         } else {
           // skew x: element (u, (u + x) mod 128) lies on offset d0 - x for
           // u < 128 - x and on d0 + 128 - x after
-          const int split = min(max(128 - x, u0), u1);
           const float* pd = sP + x;
           const float* pe = pd - 128;
+          const int split = 128 - x;
           float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
-          int u = u0;
+          int u = 0;
           for (; u + 1 < split; u += 2) {
             a0 += pd[u * (PS + 1)];
             a1 += pd[(u + 1) * (PS + 1)];
           }
           if (u < split) a0 += pd[u * (PS + 1)], ++u;
-          for (; u + 1 < u1; u += 2) {
+          for (; u + 1 < 128; u += 2) {
             b0 += pe[u * (PS + 1)];
             b1 += pe[(u + 1) * (PS + 1)];
           }
-          if (u < u1) b0 += pe[u * (PS + 1)];
-          ca = a0 + a1;
-          cb = b0 + b1;
-        }
-        // second row halves hand their sums to the first
-        if (role == 1) sH[x] = ca;
-        if (role == 3) {
-          sH[128 + x] = ca;
-          sH[256 + x] = cb;
-        }
-        __syncthreads();
-        const int64_t base = static_cast<int64_t>(bh) * N;
-        if (role == 0) {
-          const double cs = static_cast<double>(ca + sH[x]);
-          if (cs != 0.0 && k0 + x < N) atomicAdd(col + base + k0 + x, cs);
-        } else if (role == 2) {
-          const double da = static_cast<double>(ca + sH[128 + x]), db = static_cast<double>(cb + sH[256 + x]);
+          if (u < 128) b0 += pe[u * (PS + 1)];
+          const double da = static_cast<double>(a0 + a1), db = static_cast<double>(b0 + b1);
           const int64_t d0 = qbase - k0;
           if (da != 0.0 && d0 - x >= 0 && d0 - x < N) atomicAdd(sl + base + d0 - x, da);
           if (db != 0.0 && d0 + 128 - x >= 0 && d0 + 128 - x < N) atomicAdd(sl + base + d0 + 128 - x, db);
         }
+        named_sync(1, kScoreConsumers);                        // the P tile is free again
       }
     }
-    // the tile of MMA it + 1 (copied one iteration earlier) has landed
-    if (it >= 1) cp_async_wait_group1();
-    fence_proxy_async();
-    tc_fence_before();
-    __syncthreads();
   }
-  if (failed) cp_async_wait_all();
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem, 256);
+    tmem_dealloc(tmem, 512);
   }
 }
 
