@@ -33,18 +33,20 @@ constexpr int kSampleWarps = 8;
 //               the key ring allow;
 //   warps 1-3   copy key tiles (cp.async) into a ring of three shared-memory
 //               slots;
-//   warps 4-11  read S: warp 4 + w takes tensor-memory lanes 32 (w mod 4)
-//               .. +31 (trunk rows) and columns 64 (w / 4) .. +63.
-//   Pass 1: per row and half the running maximum m of x = S log2(e)/sqrt(d)
-//     over the causal keys, kept rounded up to an integer so that every
-//     rescale of the running sum l = sum 2^(x - m) (fp32 within a tile, fp64
-//     across tiles) is an exact power of two; the halves merge at the end.
+//   warps 4-19  read S: warp 4 + w takes tensor-memory lanes 32 (w mod 4)
+//               .. +31 (trunk rows) and columns 32 (w / 4) .. +31.
+//   Pass 1: per row and quarter the running maximum m of x = S log2(e) /
+//     sqrt(d) over the causal keys, kept rounded up to an integer so that
+//     every rescale of the running sum l = sum 2^(x - m) (fp32 within a
+//     tile, fp64 across tiles) is an exact power of two; the quarters merge
+//     at the end.
 //   Pass 2: p = 2^(x - m) / l (fp32) goes to a 128 x 129 fp32 tile in shared
-//     memory (one word of padding per row); consumer thread c < 128 sums key
-//     column c and thread 128 + u the diagonals t - c = -u and 128 - u of
-//     skew u, all without bank conflicts, and each per-tile sum is added to
-//     the key's column score or the offset's slash score with one fp64
-//     atomic.
+//     memory (one word of padding per row).  Consumer threads 0-255 sum key
+//     columns (two per column, one per half of the rows), threads 256-511
+//     the diagonals t - c = -u and 128 - u of skew u (two per skew, again by
+//     row halves), all without bank conflicts; the halves meet in shared
+//     memory and each per-tile sum is added to the key's column score or the
+//     offset's slash score with one fp64 atomic.
 // The logits q.k of bf16 inputs are accumulated in fp32 by the tensor core.
 // Every wait is bounded; a shared abort flag ends all roles together.
 template <int D>
@@ -57,16 +59,17 @@ struct SampleCfg {
   static constexpr int kQ = 0;
   static constexpr int kK = kQ + kTileBytes;
   static constexpr int kP = kK + kStages * kTileBytes;
-  static constexpr int kMl = kP + 128 * kPStride * 4;          // per-half (m, l) at the end of pass 1
-  static constexpr int kBar = kMl + 2 * 128 * 12;
+  static constexpr int kMl = kP + 128 * kPStride * 4;          // per-quarter (m, l) at the end of pass 1
+  static constexpr int kHalf = kMl + 4 * 128 * 12;             // second-half partial sums
+  static constexpr int kBar = kHalf + 3 * 128 * 4;
   static constexpr int kNBar = 1 + 2 * kStages + 2 * kSBufs;
   static constexpr int kSlot = kBar + kNBar * 8;
   static constexpr int kBytes = kSlot + 16;
   static constexpr int kSmem = kBytes + 1024;                // alignment slack
 };
-constexpr int kScoreThreads = 384;
+constexpr int kScoreThreads = 640;
 constexpr int kScoreProducers = 96;                           // warps 1-3
-constexpr int kScoreConsumers = 256;                          // warps 4-11
+constexpr int kScoreConsumers = 512;                          // warps 4-19
 
 template <int D>
 __global__ void __launch_bounds__(kScoreThreads, 1) sample_scores_kernel(
@@ -80,8 +83,9 @@ __global__ void __launch_bounds__(kScoreThreads, 1) sample_scores_kernel(
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                          ~static_cast<uintptr_t>(1023));
   float* sP = reinterpret_cast<float*>(smem + C::kP);
-  double* sL = reinterpret_cast<double*>(smem + C::kMl);                 // [2][128]
-  float* sM = reinterpret_cast<float*>(smem + C::kMl + 2 * 128 * 8);     // [2][128]
+  double* sL = reinterpret_cast<double*>(smem + C::kMl);                 // [4][128]
+  float* sM = reinterpret_cast<float*>(smem + C::kMl + 4 * 128 * 8);     // [4][128]
+  float* sH = reinterpret_cast<float*>(smem + C::kHalf);                 // [3][128]
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBar);
   uint64_t* bar_q = bars;
   uint64_t* bar_kfull = bars + 1;
@@ -183,41 +187,40 @@ __global__ void __launch_bounds__(kScoreThreads, 1) sample_scores_kernel(
     // ----------------------------------------------------------- consumers
     const int ct = tid - 128, cw = ct >> 5;
     const int t = (cw & 3) * 32 + lane;                        // trunk row of this thread
-    const int hc = cw >> 2;                                    // column half
+    const int qc = cw >> 2;                                    // column quarter
     const uint32_t lane_base = static_cast<uint32_t>((cw & 3) * 32) << 16;
     const int64_t q_t = qbase + t;
     const bool row_ok = t < blk;
     float m = -INFINITY;                                       // integer-valued running maximum
     double l = 0.0;
     float w = 0.f;                                             // 1 / l of this row (pass 2)
-    float* prow = sP + t * PS + hc * 64;
-    const int x = ct & 127;
+    float* prow = sP + t * PS + qc * 32;
+    const int role = ct >> 7, x = ct & 127;                    // reduction role and its index
     const int64_t base = static_cast<int64_t>(bh) * N;
     for (int it = 0; it < n_it; ++it) {
       const int sb = it % NS, j = it % T;
       const bool ok = mbar_wait_or_abort(&bar_sfull[sb], (it / NS) & 1, err, abort_flag);
       if (named_sync_or(1, kScoreConsumers, !ok)) break;
       tc_fence_after();
-      uint32_t r[64];
-      tmem_ld32(tmem + lane_base + sb * 128 + hc * 64, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
-      tmem_ld32(tmem + lane_base + sb * 128 + hc * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+      uint32_t r[32];
+      tmem_ld32(tmem + lane_base + sb * 128 + qc * 32, r);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar_sfree[sb]);
       const int64_t k0 = static_cast<int64_t>(j) * 128;
       // every key of the tile is causal for every trunk row
       const bool full = k0 + 127 <= qbase;
-      // otherwise keys k0 + 64 hc + c with c <= lim are causal for this row
-      const int64_t lim64 = q_t - k0 - 64 * hc;
-      const int lim = static_cast<int>(lim64 > 63 ? 63 : (lim64 < -1 ? -1 : lim64));
+      // otherwise keys k0 + 32 qc + c with c <= lim are causal for this row
+      const int64_t lim64 = q_t - k0 - 32 * qc;
+      const int lim = static_cast<int>(lim64 > 31 ? 31 : (lim64 < -1 ? -1 : lim64));
       if (it < T) {
         float mr = -INFINITY;                                  // max of the raw logits
         if (full) {
 #pragma unroll
-          for (int c = 0; c < 63; c += 2) mr = fmax3(mr, __uint_as_float(r[c]), __uint_as_float(r[c + 1]));
+          for (int c = 0; c < 31; c += 2) mr = fmax3(mr, __uint_as_float(r[c]), __uint_as_float(r[c + 1]));
         } else {
 #pragma unroll
-          for (int c = 0; c < 64; ++c)
+          for (int c = 0; c < 32; ++c)
             if (c <= lim) mr = fmaxf(mr, __uint_as_float(r[c]));
         }
         if (mr > -INFINITY) {
@@ -229,75 +232,94 @@ __global__ void __launch_bounds__(kScoreThreads, 1) sample_scores_kernel(
           float a[4] = {0.f, 0.f, 0.f, 0.f};
           if (full) {
 #pragma unroll
-            for (int c = 0; c < 64; ++c) a[c % 4] += ex2(fmaf(__uint_as_float(r[c]), scale_log2, -m));
+            for (int c = 0; c < 32; ++c) a[c % 4] += ex2(fmaf(__uint_as_float(r[c]), scale_log2, -m));
           } else {
 #pragma unroll
-            for (int c = 0; c < 64; ++c)
+            for (int c = 0; c < 32; ++c)
               if (c <= lim) a[c % 4] += ex2(fmaf(__uint_as_float(r[c]), scale_log2, -m));
           }
           l += static_cast<double>((a[0] + a[1]) + (a[2] + a[3]));
         }
         if (it == T - 1) {
-          // merge the halves: the larger maximum, both sums rescaled by
-          // exact powers of two
-          sM[hc * 128 + t] = m;
-          sL[hc * 128 + t] = l;
+          // merge the quarters: the largest maximum, every sum rescaled by
+          // an exact power of two
+          sM[qc * 128 + t] = m;
+          sL[qc * 128 + t] = l;
           named_sync(1, kScoreConsumers);
-          const float m0 = sM[t], m1 = sM[128 + t];
-          const float mm = fmaxf(m0, m1);
+          float mm = -INFINITY;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) mm = fmaxf(mm, sM[q * 128 + t]);
           double lt = 0.0;
-          if (m0 > -INFINITY) lt += ldexp(sL[t], static_cast<int>(m0 - mm));
-          if (m1 > -INFINITY) lt += ldexp(sL[128 + t], static_cast<int>(m1 - mm));
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float mq = sM[q * 128 + t];
+            if (mq > -INFINITY) lt += ldexp(sL[q * 128 + t], static_cast<int>(mq - mm));
+          }
           m = mm;
           w = row_ok && lt > 0.0 ? static_cast<float>(1.0 / lt) : 0.f;
         }
       } else {
         if (full) {
 #pragma unroll
-          for (int c = 0; c < 64; ++c) prow[c] = ex2(fmaf(__uint_as_float(r[c]), scale_log2, -m)) * w;
+          for (int c = 0; c < 32; ++c) prow[c] = ex2(fmaf(__uint_as_float(r[c]), scale_log2, -m)) * w;
         } else {
 #pragma unroll
-          for (int c = 0; c < 64; ++c)
+          for (int c = 0; c < 32; ++c)
             prow[c] = c <= lim ? ex2(fmaf(__uint_as_float(r[c]), scale_log2, -m)) * w : 0.f;
         }
         named_sync(1, kScoreConsumers);
-        if (ct < 128) {
+        const int u0 = (role & 1) * 64, u1 = u0 + 64;          // this thread's half of the rows
+        float ca = 0.f, cb = 0.f;                              // column, or the two diagonals
+        if (role < 2) {
           // key column x: rows u at u * PS + x
           const float* pc = sP + x;
           float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-#pragma unroll 8
-          for (int u = 0; u < 128; u += 4) {
+#pragma unroll 4
+          for (int u = u0; u < u1; u += 4) {
             a0 += pc[u * PS];
             a1 += pc[(u + 1) * PS];
             a2 += pc[(u + 2) * PS];
             a3 += pc[(u + 3) * PS];
           }
-          const double cs = static_cast<double>((a0 + a1) + (a2 + a3));
-          if (cs != 0.0 && k0 + x < N) atomicAdd(col + base + k0 + x, cs);
+          ca = (a0 + a1) + (a2 + a3);
         } else {
           // skew x: element (u, (u + x) mod 128) lies on offset d0 - x for
           // u < 128 - x and on d0 + 128 - x after
+          const int split = min(max(128 - x, u0), u1);
           const float* pd = sP + x;
           const float* pe = pd - 128;
-          const int split = 128 - x;
           float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
-          int u = 0;
+          int u = u0;
           for (; u + 1 < split; u += 2) {
             a0 += pd[u * (PS + 1)];
             a1 += pd[(u + 1) * (PS + 1)];
           }
           if (u < split) a0 += pd[u * (PS + 1)], ++u;
-          for (; u + 1 < 128; u += 2) {
+          for (; u + 1 < u1; u += 2) {
             b0 += pe[u * (PS + 1)];
             b1 += pe[(u + 1) * (PS + 1)];
           }
-          if (u < 128) b0 += pe[u * (PS + 1)];
-          const double da = static_cast<double>(a0 + a1), db = static_cast<double>(b0 + b1);
+          if (u < u1) b0 += pe[u * (PS + 1)];
+          ca = a0 + a1;
+          cb = b0 + b1;
+        }
+        // second row halves hand their sums to the first; after this barrier
+        // the P tile is free again
+        if (role == 1) sH[x] = ca;
+        if (role == 3) {
+          sH[128 + x] = ca;
+          sH[256 + x] = cb;
+        }
+        named_sync(1, kScoreConsumers);
+        if (role == 0) {
+          const double cs = static_cast<double>(ca + sH[x]);
+          if (cs != 0.0 && k0 + x < N) atomicAdd(col + base + k0 + x, cs);
+        } else if (role == 2) {
+          const double da = static_cast<double>(ca + sH[128 + x]), db = static_cast<double>(cb + sH[256 + x]);
           const int64_t d0 = qbase - k0;
           if (da != 0.0 && d0 - x >= 0 && d0 - x < N) atomicAdd(sl + base + d0 - x, da);
           if (db != 0.0 && d0 + 128 - x >= 0 && d0 + 128 - x < N) atomicAdd(sl + base + d0 + 128 - x, db);
         }
-        named_sync(1, kScoreConsumers);                        // the P tile is free again
       }
     }
   }
