@@ -357,11 +357,22 @@ __device__ double block_sum(double v, double* red) {
 // largest score threshold whose upper set reaches alpha of the total (a
 // bisection on the order-preserving 64-bit image of the scores), then the
 // entries at the threshold in ascending index until the target is met.
-// Writes a bitmap.
-__global__ void __launch_bounds__(1024) sample_cut_kernel(const double* __restrict__ col,
-                                                          const double* __restrict__ sl, int64_t N,
-                                                          double alpha, uint32_t* __restrict__ keep_col,
-                                                          uint32_t* __restrict__ keep_sl) {
+// Writes a bitmap.  With CACHED (N <= 32768) each thread keeps its 32
+// scores for the 64 bisection steps, 4 in registers and 28 in shared memory
+// (entries past N hold -1, which no threshold counts); otherwise every step
+// re-reads them from global memory.  Both visit a thread's entries in the
+// same order, so the result does not depend on the variant.
+constexpr int kCutThreads = 1024;
+constexpr int kCutRegs = 4;
+constexpr int kCutSmem = 28;
+constexpr int64_t kCutCachedMax = static_cast<int64_t>(kCutThreads) * (kCutRegs + kCutSmem);
+
+template <bool CACHED>
+__global__ void __launch_bounds__(kCutThreads) sample_cut_kernel(const double* __restrict__ col,
+                                                                 const double* __restrict__ sl, int64_t N,
+                                                                 double alpha, uint32_t* __restrict__ keep_col,
+                                                                 uint32_t* __restrict__ keep_sl) {
+  extern __shared__ double cache[];                            // CACHED: [kCutSmem][kCutThreads]
   __shared__ double red[33];
   const int fam = blockIdx.x, hq = blockIdx.y, b = blockIdx.z, Hq = gridDim.y;
   const int64_t row = static_cast<int64_t>(b) * Hq + hq;
@@ -379,13 +390,31 @@ __global__ void __launch_bounds__(1024) sample_cut_kernel(const double* __restri
     return;
   }
   const double goal = alpha * total;
+  double rv[kCutRegs];
+  if (CACHED) {
+#pragma unroll
+    for (int i = 0; i < kCutRegs + kCutSmem; ++i) {
+      const int64_t k = threadIdx.x + static_cast<int64_t>(i) * kCutThreads;
+      const double v = k < N ? sc[k] : -1.0;
+      if (i < kCutRegs) rv[i] = v;
+      else cache[(i - kCutRegs) * kCutThreads + threadIdx.x] = v;
+    }
+  }
   // bisection for the largest t with mass(score image >= t) >= goal
   uint64_t lo = 0, hi = ~0ull;             // invariant: mass(>= lo) >= goal
   while (lo < hi) {
     const uint64_t mid = lo + (hi - lo) / 2 + 1;
     double part = 0.0;
-    for (int64_t k = threadIdx.x; k < N; k += blockDim.x)
-      if (ordered_f64(sc[k]) >= mid) part += sc[k];
+    if (CACHED) {
+#pragma unroll
+      for (int i = 0; i < kCutRegs + kCutSmem; ++i) {
+        const double v = i < kCutRegs ? rv[i] : cache[(i - kCutRegs) * kCutThreads + threadIdx.x];
+        if (ordered_f64(v) >= mid) part += v;
+      }
+    } else {
+      for (int64_t k = threadIdx.x; k < N; k += blockDim.x)
+        if (ordered_f64(sc[k]) >= mid) part += sc[k];
+    }
     const double mass = block_sum(part, red);
     if (mass >= goal) lo = mid; else hi = mid - 1;
   }
@@ -543,7 +572,14 @@ cudaError_t launch_select_sample(const SelectParams& p, const TensorDesc& Q, con
                 : run(sample_scores_kernel<128>, SampleCfg<128>::kSmem);
   if (e != cudaSuccess) return e;
   dim3 g2(2, static_cast<unsigned>(p.Hq), static_cast<unsigned>(p.B));
-  sample_cut_kernel<<<g2, 1024, 0, s>>>(col, sl, p.N, p.tau, keep_col, keep_sl);
+  if (p.N <= kCutCachedMax) {
+    const int cache_bytes = kCutSmem * kCutThreads * static_cast<int>(sizeof(double));
+    e = cudaFuncSetAttribute(sample_cut_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, cache_bytes);
+    if (e != cudaSuccess) return e;
+    sample_cut_kernel<true><<<g2, kCutThreads, cache_bytes, s>>>(col, sl, p.N, p.tau, keep_col, keep_sl);
+  } else {
+    sample_cut_kernel<false><<<g2, kCutThreads, 0, s>>>(col, sl, p.N, p.tau, keep_col, keep_sl);
+  }
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int64_t rows = static_cast<int64_t>(p.B) * p.Hq * p.nb;

@@ -55,8 +55,11 @@ def _compare(w, Q, K, alpha, min_heads):
 
 @pytest.mark.parametrize("shape,alpha", [((1, 4, 2, 2048, 128, 128, 512), 0.9),
                                          ((2, 2, 1, 1024, 64, 64, 256), 0.8),
-                                         ((1, 2, 1, 1536, 128, 128, 512), 1.0)])
+                                         ((1, 2, 1, 1536, 128, 128, 512), 1.0),
+                                         ((1, 2, 1, 40960, 64, 128, 4096), 0.7)])
 def test_sample_lists_match_oracle(shape, alpha):
+    """Small shapes, and one with N > 32768 (the cut re-reads its scores
+    from global memory instead of keeping them on chip)."""
     B, Hq, Hkv, N, d, blk, seg = shape
     w = synth.Workload("smp", B=B, Hq=Hq, Hkv=Hkv, N=N, d=d, blk=blk, seg=seg, mode="topk",
                        stripe_frac=0.01, c_lo=3.0, c_hi=6.0)
