@@ -14,6 +14,8 @@
 // its total (ties to the lower index); query block i lists every key block
 // of earlier segments that holds a kept column, or a key q - d for one of
 // its queries q and a kept offset d.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <math.h>
 
 #include "pbs_common.cuh"
@@ -31,8 +33,9 @@ constexpr int kSampleWarps = 8;
 //   warp 0      issues S = Q_trunk K_tile^T (tcgen05.mma) into a ring of
 //               four tensor-memory buffers, as far ahead as the buffers and
 //               the key ring allow;
-//   warps 1-3   copy key tiles (cp.async) into a ring of three shared-memory
-//               slots;
+//   warp 1      loads the trunk's query tile once and the key tiles into a
+//               ring of three shared-memory slots with TMA (cp.async.bulk
+//               .tensor, 128-byte swizzle, no multicast);
 //   warps 4-19  read S: warp 4 + w takes tensor-memory lanes 32 (w mod 4)
 //               .. +31 (trunk rows) and columns 32 (w / 4) .. +31.
 //   Pass 1: per row and quarter the running maximum m of x = S log2(e) /
@@ -67,14 +70,29 @@ struct SampleCfg {
   static constexpr int kBytes = kSlot + 16;
   static constexpr int kSmem = kBytes + 1024;                // alignment slack
 };
-constexpr int kScoreThreads = 640;
-constexpr int kScoreProducers = 96;                           // warps 1-3
+constexpr int kScoreThreads = 640;                            // warps 2-3 only join the teardown
 constexpr int kScoreConsumers = 512;                          // warps 4-19
+
+// mbarrier arrive that also announces `bytes` of asynchronous copies.
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+// One 64-column x 128-row box of a [B, H, N, D] bf16 tensor (coordinates
+// d, n, h, b) into shared memory, completing on `bar`.  d is 0 or 64, so the
+// innermost coordinate is always a multiple of 16 bytes.
+__device__ __forceinline__ void tma_rows_4d(uint32_t dst, const CUtensorMap* map, int d, int n, int h, int b,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+      "[%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(d), "r"(n), "r"(h), "r"(b), "r"(smem_u32(bar))
+      : "memory");
+}
 
 template <int D>
 __global__ void __launch_bounds__(kScoreThreads, 1) sample_scores_kernel(
-    const __nv_bfloat16* __restrict__ Q, int64_t qsB, int64_t qsH, int64_t qsN,
-    const __nv_bfloat16* __restrict__ K, int64_t ksB, int64_t ksH, int64_t ksN, int64_t N, int B, int Hq,
+    const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk, int64_t N, int B, int Hq,
     int G, int blk, int seg, float scale_log2, double* __restrict__ col, double* __restrict__ sl,
     int* __restrict__ err) {
   using C = SampleCfg<D>;
@@ -106,16 +124,15 @@ __global__ void __launch_bounds__(kScoreThreads, 1) sample_scores_kernel(
   const int64_t qbase = seg_end - blk;
   const int T = static_cast<int>((seg_end + 127) / 128);
   const int n_it = 2 * T;                                      // MMAs: pass 1 then pass 2
-  constexpr int CH = D / 8;                                    // 16-byte chunks per row
 
   if (warp == 0) {
     tmem_alloc(slot, 512);
     tmem_relinquish();
   }
   if (tid == 0) {
-    mbar_init(bar_q, kScoreProducers);
+    mbar_init(bar_q, 1);
     for (int i = 0; i < NK; ++i) {
-      mbar_init(&bar_kfull[i], kScoreProducers);
+      mbar_init(&bar_kfull[i], 1);
       mbar_init(&bar_kempty[i], 1);
     }
     for (int i = 0; i < NS; ++i) {
@@ -157,32 +174,24 @@ __global__ void __launch_bounds__(kScoreThreads, 1) sample_scores_kernel(
       }
       __syncwarp();
     }
-  } else if (warp < 4) {
-    // ----------------------------------------------------------- producers
-    const int pt = tid - 32;
-    const __nv_bfloat16* qb = Q + b * qsB + hq * qsH;
-    const __nv_bfloat16* kb = K + b * ksB + (hq / G) * ksH;
-    for (int id = pt; id < 128 * CH; id += kScoreProducers) {
-      const int r = id / CH, c = id % CH;
-      const bool valid = r < blk;
-      cp_async16_zfill(sQ + (c / 8) * C::kHalfBytes + sw128_offset(r, c % 8),
-                       valid ? qb + (qbase + r) * qsN + c * 8 : qb, valid);
-    }
-    cp_async_mbar_arrive(bar_q);
-    for (int it = 0; it < n_it; ++it) {
-      const int ks = it % NK;
-      if (it >= NK && !mbar_wait_or_abort(&bar_kempty[ks], ((it / NK) - 1) & 1, err, abort_flag)) break;
-      const int64_t k0 = static_cast<int64_t>(it % T) * 128;
-      const uint32_t dst = sK + ks * C::kTileBytes;
-      for (int id = pt; id < 128 * CH; id += kScoreProducers) {
-        const int r = id / CH, c = id % CH;
-        const bool valid = k0 + r < seg_end;
-        cp_async16_zfill(dst + (c / 8) * C::kHalfBytes + sw128_offset(r, c % 8),
-                         valid ? kb + (k0 + r) * ksN + c * 8 : kb, valid);
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      constexpr uint32_t kTileTx = 128 * D * 2;
+      mbar_expect_tx(bar_q, kTileTx);
+      for (int h = 0; h < D / 64; ++h) tma_rows_4d(sQ + h * C::kHalfBytes, &mq, 64 * h, static_cast<int>(qbase), hq, b, bar_q);
+      for (int it = 0; it < n_it; ++it) {
+        const int ks = it % NK;
+        if (it >= NK && !mbar_wait_or_abort(&bar_kempty[ks], ((it / NK) - 1) & 1, err, abort_flag)) break;
+        const int k0 = (it % T) * 128;
+        mbar_expect_tx(&bar_kfull[ks], kTileTx);
+        for (int h = 0; h < D / 64; ++h)
+          tma_rows_4d(sK + ks * C::kTileBytes + h * C::kHalfBytes, &mk, 64 * h, k0, hq / G, b, &bar_kfull[ks]);
       }
-      cp_async_mbar_arrive(&bar_kfull[ks]);
     }
-    cp_async_wait_all();
+    __syncwarp();
+  } else if (warp < 4) {
+    // warps 2-3 have no role
   } else {
     // ----------------------------------------------------------- consumers
     const int ct = tid - 128, cw = ct >> 5;
@@ -548,6 +557,40 @@ __global__ void __launch_bounds__(kSampleWarps * 32) sample_lists_kernel(
   }
 }
 
+// cuTensorMapEncodeTiled from the driver, looked up once through the runtime.
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static const PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      f = nullptr;
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  }();
+  return fn;
+}
+
+// Tensor map of a [B, H, N, D] bf16 tensor for 64-column x 128-row boxes,
+// 128-byte swizzle, rows past N read as zeros.  The stride of an extent-1
+// dimension is never used, so it is replaced by a valid one; a zero stride
+// over several heads or batches (a broadcast view) is not supported.
+bool encode_rows_map(CUtensorMap* map, const TensorDesc& t) {
+  const PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (!enc) return false;
+  cuuint64_t sn = static_cast<cuuint64_t>(t.sN) * 2;
+  cuuint64_t sh = t.H > 1 ? static_cast<cuuint64_t>(t.sH) * 2 : sn * static_cast<cuuint64_t>(t.N);
+  cuuint64_t sb = t.B > 1 ? static_cast<cuuint64_t>(t.sB) * 2 : sh * static_cast<cuuint64_t>(t.H);
+  if (sh == 0 || sb == 0) return false;
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(t.D), static_cast<cuuint64_t>(t.N), static_cast<cuuint64_t>(t.H),
+                        static_cast<cuuint64_t>(t.B)};
+  cuuint64_t strides[3] = {sn, sh, sb};
+  cuuint32_t box[4] = {64, 128, 1, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(t.ptr), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace
 
 cudaError_t launch_select_sample(const SelectParams& p, const TensorDesc& Q, const TensorDesc& K,
@@ -560,12 +603,13 @@ cudaError_t launch_select_sample(const SelectParams& p, const TensorDesc& Q, con
   if (e != cudaSuccess) return e;
   const int nseg = static_cast<int>((p.N + p.seg - 1) / p.seg);
   const unsigned nblk = static_cast<unsigned>(nseg) * static_cast<unsigned>(p.B * p.Hq);
+  CUtensorMap mq, mk;
+  if (!encode_rows_map(&mq, Q) || !encode_rows_map(&mk, K)) return cudaErrorNotSupported;
   auto run = [&](auto kernel, int smem_bytes) -> cudaError_t {
     cudaError_t e2 = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
     if (e2 != cudaSuccess) return e2;
-    kernel<<<nblk, kScoreThreads, smem_bytes, s>>>(static_cast<const __nv_bfloat16*>(Q.ptr), Q.sB, Q.sH, Q.sN,
-                                         static_cast<const __nv_bfloat16*>(K.ptr), K.sB, K.sH, K.sN, p.N, p.B,
-                                         p.Hq, p.Hq / p.Hkv, p.blk, p.seg, scale_log2, col, sl, err);
+    kernel<<<nblk, kScoreThreads, smem_bytes, s>>>(mq, mk, p.N, p.B, p.Hq, p.Hq / p.Hkv, p.blk, p.seg, scale_log2,
+                                                    col, sl, err);
     return cudaGetLastError();
   };
   e = p.D == 64 ? run(sample_scores_kernel<64>, SampleCfg<64>::kSmem)
