@@ -51,7 +51,8 @@ constexpr int kSampleWarps = 8;
 //     memory and each per-tile sum is added to the key's column score or the
 //     offset's slash score with one fp64 atomic.
 // The logits q.k of bf16 inputs are accumulated in fp32 by the tensor core.
-// Every wait is bounded; a shared abort flag ends all roles together.
+// Every wait is bounded; a shared abort flag ends the MMA and producer roles
+// and turns the consumers' remaining waits into no-ops.
 template <int D>
 struct SampleCfg {
   static constexpr int kHalfBytes = 128 * 128;               // 128 rows x 64 bf16
@@ -208,8 +209,10 @@ __global__ void __launch_bounds__(kScoreThreads, 1) sample_scores_kernel(
     const int64_t base = static_cast<int64_t>(bh) * N;
     for (int it = 0; it < n_it; ++it) {
       const int sb = it % NS, j = it % T;
-      const bool ok = mbar_wait_or_abort(&bar_sfull[sb], (it / NS) & 1, err, abort_flag);
-      if (named_sync_or(1, kScoreConsumers, !ok)) break;
+      // After an abort (the wait gave up) the loop still runs to its end, so
+      // that every consumer takes the same named barriers; the results are
+      // then meaningless and the error word says so.
+      mbar_wait_or_abort(&bar_sfull[sb], (it / NS) & 1, err, abort_flag);
       tc_fence_after();
       uint32_t r[32];
       tmem_ld32(tmem + lane_base + sb * 128 + qc * 32, r);
