@@ -134,7 +134,9 @@ def workspace_size(op: int, Q: torch.Tensor, K: torch.Tensor, blk: int, seg: int
 
 def select_capacity(N: int, blk: int, seg: int, mode: str, density_or_tau: float,
                     band: int = 0, n_sink: int = 0) -> int:
-    m = _MODES.get(mode, PBS_SELECT_TOPK)
+    if mode not in _MODES:
+        raise ValueError(f"unknown selection mode {mode!r}; expected one of {sorted(_MODES)}")
+    m = _MODES[mode]
     rc = load().pbs_select_capacity(N, blk, seg, m, float(density_or_tau), band, n_sink)
     _check(min(rc, 0))
     return rc

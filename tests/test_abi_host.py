@@ -172,3 +172,35 @@ def test_binding_refuses_cpu_tensors(lib):
     x = torch.zeros(1, 1, 128, 64, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         pbs.pbs_permute(x, x, 64, 128)
+
+
+def test_sample_selector_host_checks(lib):
+    """PBS_SELECT_SAMPLE: a null permutation is accepted (it reads none);
+    the visiting-order and per-segment flags, a non-positive CIA target and
+    a too-small capacity are refused before anything runs; the capacity is
+    every candidate block; the workspace holds fp64 column and slash scores
+    and two bitmaps per (b, query head)."""
+    SAMPLE = 2
+    q, k = _desc(H=2, N=1024), _desc(H=1, N=1024)
+    cap = pbs.select_capacity(1024, 128, 256, "sample", 0.9)
+    assert cap == pbs.select_capacity(1024, 128, 256, "tau", 0.9) == 6
+    args = (ctypes.c_void_p(0x3000), ctypes.c_void_p(0x5000))
+    for mode, target, c, code in ((SAMPLE | 0x10, 0.9, cap, -2), (SAMPLE | 0x20, 0.9, cap, -2),
+                                  (SAMPLE, 0.0, cap, -1), (SAMPLE, -1.0, cap, -1),
+                                  (SAMPLE, float("nan"), cap, -1), (SAMPLE, 0.9, cap - 1, -3)):
+        rc = lib.pbs_select(ctypes.byref(q), ctypes.byref(k), None, 128, 256, mode, target, 0, 0, *args, c,
+                            ctypes.c_void_p(0x4000), 1 << 30, None)
+        assert rc == code, (mode, target, c, rc)
+    # other modes still need a permutation
+    rc = lib.pbs_select(ctypes.byref(q), ctypes.byref(k), None, 128, 256, 0, 0.5, 0, 0, *args, cap,
+                        ctypes.c_void_p(0x4000), 1 << 30, None)
+    assert rc == -1 and b"perm" in lib.pbs_get_last_error()
+    Q, K = _desc(B=1, H=32, N=32768), _desc(B=1, H=8, N=32768)
+    words = 32768 // 32
+    expect = 2 * 32 * 32768 * 8 + 2 * 32 * words * 4
+    assert lib.pbs_workspace_size(pbs.PBS_OP_SELECT_SAMPLE, ctypes.byref(Q), ctypes.byref(K), 128, 2048) == expect
+
+
+def test_binding_rejects_unknown_selection_mode(lib):
+    with pytest.raises(ValueError):
+        pbs.select_capacity(1024, 128, 256, "bogus", 0.5)
