@@ -78,6 +78,31 @@ def tile_flops(w) -> float:
     return 4.0 * w.blk * w.blk * w.d
 
 
+def permute_bytes(w):
+    """Algorithmic bytes of pbs_permute: K once, the last query block of every
+    head, the permutation written (one per query segment when segmented)."""
+    if w.mode in ("gate", "sample"):
+        return None
+    nseg = (w.N + w.seg - 1) // w.seg
+    n_perm = w.B * w.Hkv * w.N * (nseg if w.perm_per_segment else 1)
+    q_read = w.B * w.Hq * (w.N if w.perm_per_segment else w.blk) * w.d * 2
+    return w.B * w.Hkv * w.N * w.d * 2 + q_read + n_perm * 4
+
+
+def select_bytes(w, cap):
+    """Algorithmic bytes of pbs_select (top-k / tau): Q and K once, the pooled
+    fp32 block sums written and read back, and the block lists."""
+    if w.mode in ("gate", "sample"):
+        return None
+    pooled = w.B * w.Hq * w.nb * w.d * 4 + 2 * w.B * w.Hkv * w.nb * w.d * 4
+    lists = w.B * w.Hq * w.nb * (1 + cap) * 4
+    return w.B * w.Hq * w.N * w.d * 2 + w.B * w.Hkv * w.N * w.d * 2 + 2 * pooled + lists
+
+
+def _gbs(nbytes, ms):
+    return None if nbytes is None or ms <= 0 else nbytes / (ms * 1e-3) / 1e9
+
+
 # --------------------------------------------------------------------- clocks
 class ClockSampler:
     """Samples SM clock and throttle reasons with NVML (read-only) while running."""
@@ -404,34 +429,22 @@ def run_pbs(args):
             del lse_all
         del d_idx, Od
 
-    # end to end through the C ABI with host buffers: H2D of Q, K, V from
-    # pinned memory and D2H of O inside the timed region
+    # end to end through the public API with host buffers: H2D of Q, K, V
+    # from pinned memory and D2H of O inside the timed region.  HostPrefill
+    # overlaps the copies of one KV head's unit with the kernels of another
+    # on three streams; the result must equal the device-resident run's O.
     e2e = None
     if not args.no_e2e:
+        from permuted_block_sparse_b200.host_pipeline import HostPrefill
         Qh = torch.from_numpy(Qn).to(torch.bfloat16).pin_memory()
         Kh = torch.from_numpy(Kn).to(torch.bfloat16).pin_memory()
         Vh = torch.from_numpy(Vn).to(torch.bfloat16).pin_memory()
         Oh = torch.empty(Qh.shape, dtype=torch.bfloat16).pin_memory()
-        Qd, Kd, Vd = torch.empty_like(Q), torch.empty_like(K), torch.empty_like(V)
-
-        def e2e_step():
-            Qd.copy_(Qh, non_blocking=True)
-            Kd.copy_(Kh, non_blocking=True)
-            Vd.copy_(Vh, non_blocking=True)
-            if not gate:
-                if not sample:
-                    permute(Qd, Kd, w.blk, w.seg, w.n_sink, perm=perm, ws=ws_p)
-                pbs.pbs_select(Qd, Kd, None if sample else perm, w.blk, w.seg, w.mode, dt, w.band, w.n_sink,
-                               cap=cap, counts=counts, idx=idx, ws=ws_s, score_order=early)
-            if early:
-                pbs.pbs_attn_fwd_early_stop(Qd, Kd, Vd, perm, counts, idx, w.blk, w.seg, w.stop_tau, out=O,
-                                            lse=lse)
-            else:
-                pbs.pbs_attn_fwd(Qd, Kd, Vd, perm, counts, idx, w.blk, w.seg, out=O, lse=lse, gate_thr=thr)
-            Oh.copy_(O, non_blocking=True)
-
-        e2e_step()
+        hp = HostPrefill(w.B, w.Hq, w.Hkv, w.N, w.d, w.blk, w.seg, "gate" if gate else w.mode, dt, w.band,
+                         w.n_sink, w.stop_tau, w.perm_per_segment, gate_thr=thr, device=dev)
+        hp.run(Qh, Kh, Vh, Oh)
         torch.cuda.synchronize()
+        same = bool(torch.equal(Oh, O.cpu()))
         if world > 1:
             dist.barrier()
         a = torch.cuda.Event(enable_timing=True)
@@ -439,16 +452,20 @@ def run_pbs(args):
         k_e2e = max(1, min(args.steps, 5))
         a.record(s)
         for _ in range(k_e2e):
-            e2e_step()
+            hp.run(Qh, Kh, Vh, Oh)
         b.record(s)
         torch.cuda.synchronize()
+        pbs.pbs_check_device()
         ems = a.elapsed_time(b) / k_e2e
         if world > 1:
             ems = shard.max_over_ranks([ems], dist)[0]
         e2e = {"value": dense_causal_flops(w) * world / (ems * 1e-3) / 1e12, "unit": "TFLOP/s",
                "ms_per_step": ems,
                "h2d_bytes_per_step": int(Qh.numel() * 2 + Kh.numel() * 2 + Vh.numel() * 2),
-               "d2h_bytes_per_step": int(Oh.numel() * 2)}
+               "d2h_bytes_per_step": int(Oh.numel() * 2),
+               "pipeline": f"{len(hp.units)} units of one KV head, copies and kernels on three streams",
+               "matches_device_run": same}
+        del hp
 
     peaks, peak_src = load_peaks()
     peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
@@ -483,6 +500,7 @@ def run_pbs(args):
                    "per_gpu": "one full workload per GPU",
                    "l2": "inputs larger than L2 (Q alone is %.2f GB)" % (Q.numel() * 2 / 1e9)},
         "breakdown": {"permute_ms": ms_perm, "select_ms": ms_sel, "attn_ms": ms_attn,
+                      "permute_gbs": _gbs(permute_bytes(w), ms_perm), "select_gbs": _gbs(select_bytes(w, cap), ms_sel),
                       "executed_tiles": n_qk, ("skipped_tiles" if early else "gated_tiles"): n_gated,
                       "causal_tiles": causal_tiles,
                       "density": n_qk / causal_tiles, "executed_tflops": achieved,

@@ -1,8 +1,9 @@
 """Permuted block-sparse attention prefill on B200 (sm_100a).
 
 The compute lives in libpbs.so (hand-written CUDA behind a C ABI, see
-include/pbs.h); this package is its Python binding plus the seeded synthetic
-input generator used by the tests and the benchmark.
+include/pbs.h); this package is its Python binding, a host-memory prefill
+driver that overlaps copies and kernels on CUDA streams (host_pipeline), and
+the seeded synthetic input generator used by the tests and the benchmark.
 """
 from ._binding import (EXPORTS, LIB_PATH, PBS_OP_ATTN, PBS_OP_PERMUTE, PBS_OP_PERMUTE_SEGMENTED,  # noqa: F401
                        PBS_OP_SELECT, PBS_OP_SELECT_SAMPLE, PBS_OP_SELECT_SEGMENTED,
