@@ -572,12 +572,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
     float m_run = -INFINITY, l_run = 0.f;
     bool o_init = false;
     int k = 0, n_qk = 0, n_gated = 0;
+    // ok turns false once a wait gave up (after an abort); the loop then runs
+    // to its end with every wait returning at once, so the warpgroup takes
+    // the same named barriers without a vote each tile.
     bool ok = true;
-    for (int t = 0; active && ok && t < T; ++t) {
+    for (int t = 0; active && t < T; ++t) {
       if (!((tile_mask(t) >> h) & 1u)) continue;
-      ok = mbar_wait_or_abort(&sh.bar_s[h], k & 1, p.err, abort_flag);
-      ok = !named_sync_or(2 + h, 128, !ok);          // the warpgroup leaves together
-      if (!ok) break;
+      if (!mbar_wait_or_abort(&sh.bar_s[h], k & 1, p.err, abort_flag)) ok = false;
       tc_fence_after();
       ++n_qk;
       // Block-max gate first: the tile's raw maximum over all rows decides
@@ -744,6 +745,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
       if (stop_now) break;
     }
     // ---- epilogue: O / l -> bf16, LSE
+    if (active) ok = !named_sync_or(2 + h, 128, !ok);  // one vote for the whole loop
     if (active && ok && k > 0) {
       ok = mbar_wait_or_abort(&sh.bar_o[h], 0, p.err, abort_flag);
       ok = !named_sync_or(2 + h, 128, !ok);
