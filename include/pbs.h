@@ -175,10 +175,13 @@ int pbs_select_capacity(int64_t N, int blk, int seg, int mode,
  *     and a kept offset d.  perm is not read (may be NULL): the lists index
  *     natural key blocks, to be attended with the identity permutation.
  *     band, n_sink and the flags do not apply.  ws: pbs_workspace_size(
- *     PBS_OP_SELECT_SAMPLE, ...) bytes.  The probabilities are fp32, summed
- *     in fp64, so a column or slash whose accumulated score lies within
- *     about 1e-6 of the cut may be decided differently from an fp64
- *     reference.
+ *     PBS_OP_SELECT_SAMPLE, ...) bytes.  The probabilities and their sums
+ *     within a 128-key tile are fp32, the sums across tiles fp64, so a
+ *     column or slash whose accumulated score lies within about 1e-6
+ *     (relative) of the cut may be decided differently from an fp64
+ *     reference.  Q and K are read through TMA tensor maps: a zero head
+ *     or batch stride over more than one head or batch entry (a broadcast
+ *     view) returns PBS_ERR_UNSUPPORTED.
  * With mode | PBS_SELECT_PERM_PER_SEGMENT, perm is [B, Hkv, nseg, N] from
  * pbs_permute_segmented and block i pools and scores the keys of its own
  * segment's permutation; ws then needs pbs_workspace_size(

@@ -191,6 +191,12 @@ def test_sample_selector_host_checks(lib):
         rc = lib.pbs_select(ctypes.byref(q), ctypes.byref(k), None, 128, 256, mode, target, 0, 0, *args, c,
                             ctypes.c_void_p(0x4000), 1 << 30, None)
         assert rc == code, (mode, target, c, rc)
+    # broadcast views (a zero head stride over two heads) cannot be read by TMA
+    qb = _desc(H=2, N=1024)
+    qb.sH = 0
+    rc = lib.pbs_select(ctypes.byref(qb), ctypes.byref(k), None, 128, 256, SAMPLE, 0.9, 0, 0, *args, cap,
+                        ctypes.c_void_p(0x4000), 1 << 30, None)
+    assert rc == -2 and b"broadcast" in lib.pbs_get_last_error()
     # other modes still need a permutation
     rc = lib.pbs_select(ctypes.byref(q), ctypes.byref(k), None, 128, 256, 0, 0.5, 0, 0, *args, cap,
                         ctypes.c_void_p(0x4000), 1 << 30, None)
