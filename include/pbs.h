@@ -126,8 +126,8 @@ int pbs_permute_noalloc(const pbs_tensor* Q, const pbs_tensor* K, int blk, int s
 /* pbs_permute_segmented: one key permutation per query segment,
  * perm[b, hkv, s, p] = original key position at logical position p as read
  * by query segment s ("S2O ...", Technical Summary, 1. Online Permutation
- * via Index-Driven Loading: historical keys are scored against a
- * representative query of the segment, prefix keys only).
+ * via Index-Driven Loading: each query segment ranks the keys that precede
+ * it by one query standing for the whole segment).
  *   1. qbar_s[b,hkv] = sum of every query row of segment s of every query
  *      head of KV head hkv's group (fp64);
  *   2. score s_j = qbar_s . K[b,hkv,j] (fp64); positions j < n_sink get +inf;

@@ -162,10 +162,10 @@ def permute_segmented(Q: np.ndarray, K: np.ndarray, blk: int, seg: int, n_sink: 
     """One key permutation per query segment (S2O's historical KV permutation).
 
     "S2O: Early Stopping for Sparse Attention via Online Permutation",
-    Technical Summary, 1. Online Permutation via Index-Driven Loading: the
-    historical keys are scored against a representative query of the
-    segment, and only prefix keys are considered.  For query segment s the
-    keys are scored against s's representative query (segment_queries; sinks
+    Technical Summary, 1. Online Permutation via Index-Driven Loading: each
+    query segment ranks the keys that precede it by one query standing for
+    the whole segment.  For query segment s the keys are scored against that
+    query (segment_queries; sinks
     get +inf); each key segment before s is sorted by those scores
     (descending, ties in ascending position); key segments from s on are not
     s's history and keep their natural order.  Returns perm[b, hkv, s, p],

@@ -2,9 +2,9 @@
 //
 // "S2O: Early Stopping for Sparse Attention via Online Permutation",
 // Technical Summary, 1. Online Permutation via Index-Driven Loading
-// (Historical KV Permutation): the keys before a query segment are scored
-// against a representative query of that segment (only prefix keys count)
-// and the resulting index map orders them for loading.
+// (Historical KV Permutation): each query segment ranks the keys that come
+// before it by one query standing for the whole segment, and that ranking
+// is the order in which the segment loads them.
 //
 // Here the representative query of segment s is the sum of its query rows
 // over the KV head's group; for each key segment j < s the keys of j are

@@ -4,9 +4,10 @@
 // "SampleAttention" (MLSys 2025 talk), Technical Deep Dive:
 //   Stage 1, Trunk Sampling -- estimate attention scores from queries sampled
 //     in chunks (trunks) across the sequence;
-//   Stage 2, Score-Based Filtering -- keep the key-column and slash patterns
-//     needed to preserve the target attention mass (CIA), the two families
-//     filtered separately ("decoupled"), and turn them into a block mask.
+//   Stage 2, Score-Based Filtering -- choose the key columns and slash
+//     offsets that together hold the required share of the attention mass
+//     (the CIA target), each family cut on its own, and turn them into a
+//     block mask.
 // Here the trunks are the last query block of every segment.  Per query
 // head, their softmax probabilities are summed per key column and per slash
 // offset q - k (fp64 accumulation); each family keeps its highest entries up

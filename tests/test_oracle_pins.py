@@ -561,7 +561,7 @@ def test_coverage_definition():
 
 # ---------------------------------------------------------------------------
 # per-query-segment key permutation (S2O, Technical Summary 1: historical
-# KV permutation against a representative query of each segment)
+# KV permutation, one ranking of the earlier keys per query segment)
 # ---------------------------------------------------------------------------
 
 def test_segment_queries_closed_form():
