@@ -74,6 +74,15 @@ def selection_label(w) -> str:
     return sel + (f" band={w.band}" if w.band else "") + (f" n_sink={w.n_sink}" if w.n_sink else "")
 
 
+def arm_config(w) -> dict:
+    """The workload description both arms print."""
+    q_gb = w.B * w.Hq * w.N * w.d * 2 / 1e9
+    return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d, "blk": w.blk,
+            "seg": w.seg, "selection": selection_label(w), "per_gpu": "one full workload per GPU",
+            "l2": "inputs larger than L2 (Q alone is %.2f GB)" % q_gb if q_gb > 0.126 else
+                  "inputs smaller than L2 (Q is %.3f GB)" % q_gb}
+
+
 def tile_flops(w) -> float:
     return 4.0 * w.blk * w.blk * w.d
 
@@ -495,10 +504,7 @@ def run_pbs(args):
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d, "blk": w.blk,
-                   "seg": w.seg, "selection": selection_label(w),
-                   "per_gpu": "one full workload per GPU",
-                   "l2": "inputs larger than L2 (Q alone is %.2f GB)" % (Q.numel() * 2 / 1e9)},
+        "config": arm_config(w),
         "breakdown": {"permute_ms": ms_perm, "select_ms": ms_sel, "attn_ms": ms_attn,
                       "permute_gbs": _gbs(permute_bytes(w), ms_perm), "select_gbs": _gbs(select_bytes(w, cap), ms_sel),
                       "executed_tiles": n_qk, ("skipped_tiles" if early else "gated_tiles"): n_gated,
@@ -541,8 +547,7 @@ def run_reference(args):
         "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": statistics.median(totals) * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d, "blk": w.blk,
-                   "seg": w.seg},
+        "config": arm_config(w),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cpu["cores"], "kind": "oracle",
                          "sample": cpu["sample"]},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
