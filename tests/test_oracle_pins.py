@@ -724,3 +724,44 @@ def test_select_sample_matches_position_mask(alpha):
             assert lists[(0, h, i)].tolist() == sorted(want), (h, i)
             if alpha >= 1.0:
                 assert lists[(0, h, i)].tolist() == list(range(ncand))
+
+
+def test_select_sample_lists_grow_with_alpha():
+    """Each family's cut keeps the highest scores up to the target, so a
+    larger target keeps a superset of columns and offsets, and every block
+    list at a smaller target is contained in the list at a larger one."""
+    B, Hq, Hkv, N, d, blk, seg = 1, 2, 1, 256, 16, 16, 64
+    Q, K, V = _small(B, Hq, Hkv, N, d, seed=71, scale=2.0)
+    prev = None
+    for alpha in (0.2, 0.5, 0.8, 0.95, 1.0):
+        _, lists = oracle.select_sample(Q, K, blk, seg, alpha)
+        if prev is not None:
+            for key, arr in lists.items():
+                assert set(prev[key].tolist()) <= set(arr.tolist()), (alpha, key)
+        prev = lists
+
+
+def test_select_sample_single_sink_column():
+    """All attention on key 0 (a sink): a key aligned with every query at a
+    logit of about 34 against 0 elsewhere.  Every trunk row puts more than
+    1 - 1e-12 of its mass on key 0, so the column cut keeps key 0 alone for
+    any target up to 0.99, and every query block past the first segment
+    lists block 0 (the first segment has no candidates)."""
+    N, d, blk, seg = 128, 8, 16, 32
+    Q = np.zeros((1, 1, N, d), np.float32)
+    K = np.zeros((1, 1, N, d), np.float32)
+    Q[..., 0] = 4.0
+    K[0, 0, 0, 0] = 24.0                         # logit 96 / sqrt(8) ~ 33.9 against 0 elsewhere
+    scale = 1.0 / math.sqrt(d)
+    col, sl = oracle.sample_pattern_scores(Q, K, 0, 0, blk, seg, scale)
+    rows = oracle.sample_trunk_rows(N, blk, seg)
+    assert col[0] > len(rows) * (1 - 1e-12)
+    for alpha in (0.3, 0.9, 0.99):
+        kc = oracle.cumulative_cut(col, alpha)
+        assert np.flatnonzero(kc).tolist() == [0]
+    counts, lists = oracle.select_sample(Q, K, blk, seg, 0.5)
+    for i in range(N // blk):
+        if oracle.n_candidates(i, blk, seg) > 0:
+            assert 0 in lists[(0, 0, i)].tolist(), i
+        else:
+            assert lists[(0, 0, i)].size == 0
