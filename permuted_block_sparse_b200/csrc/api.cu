@@ -306,6 +306,9 @@ int pbs_select(const pbs_tensor* Qt, const pbs_tensor* Kt, const int32_t* perm, 
     return fail(PBS_ERR_UNSUPPORTED, "the sample selector lists natural blocks in ascending order only");
   if (mode == PBS_SELECT_SAMPLE && !(density_or_tau > 0.0))
     return fail(PBS_ERR_INVALID_ARG, "CIA target %g must be positive", density_or_tau);
+  if (mode == PBS_SELECT_SAMPLE &&
+      (Q.B * Q.H * ((Q.N + seg - 1) / seg) >= (1ll << 31) || Q.B * Q.H * (Q.N / blk) >= (1ll << 31)))
+    return fail(PBS_ERR_UNSUPPORTED, "B * Hq * segments or B * Hq * blocks above 2^31");
   if (mode == PBS_SELECT_SAMPLE && ((Q.H > 1 && Q.sH == 0) || (Q.B > 1 && Q.sB == 0) ||
                                     (K.H > 1 && K.sH == 0) || (K.B > 1 && K.sB == 0)))
     return fail(PBS_ERR_UNSUPPORTED, "the sample selector reads Q and K by TMA: zero head/batch strides "

@@ -606,7 +606,7 @@ cudaError_t launch_select_sample(const SelectParams& p, const TensorDesc& Q, con
   e = cudaMemsetAsync(sl, 0, nsc * sizeof(double), s);
   if (e != cudaSuccess) return e;
   const int nseg = static_cast<int>((p.N + p.seg - 1) / p.seg);
-  const unsigned nblk = static_cast<unsigned>(nseg) * static_cast<unsigned>(p.B * p.Hq);
+  const unsigned nblk = static_cast<unsigned>(static_cast<int64_t>(nseg) * p.B * p.Hq);   // < 2^31, checked
   CUtensorMap mq, mk;
   if (!encode_rows_map(&mq, Q) || !encode_rows_map(&mk, K)) return cudaErrorNotSupported;
   auto run = [&](auto kernel, int smem_bytes) -> cudaError_t {

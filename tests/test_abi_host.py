@@ -197,6 +197,11 @@ def test_sample_selector_host_checks(lib):
     rc = lib.pbs_select(ctypes.byref(qb), ctypes.byref(k), None, 128, 256, SAMPLE, 0.9, 0, 0, *args, cap,
                         ctypes.c_void_p(0x4000), 1 << 30, None)
     assert rc == -2 and b"broadcast" in lib.pbs_get_last_error()
+    # grids above 2^31 CTAs are refused on the host
+    big_q, big_k = _desc(B=65535, H=65535, N=128 * 8192), _desc(B=65535, H=1, N=128 * 8192)
+    rc = lib.pbs_select(ctypes.byref(big_q), ctypes.byref(big_k), None, 128, 128, SAMPLE, 0.9, 0, 0, *args,
+                        8192, ctypes.c_void_p(0x4000), 1 << 62, None)
+    assert rc == -2 and b"2^31" in lib.pbs_get_last_error(), rc
     # other modes still need a permutation
     rc = lib.pbs_select(ctypes.byref(q), ctypes.byref(k), None, 128, 256, 0, 0.5, 0, 0, *args, cap,
                         ctypes.c_void_p(0x4000), 1 << 30, None)
