@@ -446,6 +446,85 @@ def select_sample(Q, K, blk: int, seg: int, alpha: float,
     return counts, lists
 
 
+def guide_vectors(K: np.ndarray) -> np.ndarray:
+    """S2O's shared guide vector for ranking queries ("S2O: Early Stopping
+    for Sparse Attention via Online Permutation", Technical Summary, 1.
+    Online Permutation via Index-Driven Loading, Query Permutation).  Read
+    here as the sum of every key of the KV head, so that a query's score
+    q . g is the sum of its logits over all keys: large for the queries that
+    attend broadly, which draw horizontal stripes.  fp64 [B, Hkv, d]."""
+    return K.astype(F64).sum(axis=2)
+
+
+def permute_queries(Q: np.ndarray, K: np.ndarray, seg: int) -> np.ndarray:
+    """Q_perm: per (b, query head, segment), the query positions in
+    descending q . g (g the KV head's guide vector), equal scores in ascending
+    position.  qperm[b, hq, p] = original query position at permuted
+    position p; a bijection of each segment onto itself.  [B, Hq, N] int32."""
+    B, Hq, N, d = Q.shape
+    Hkv = K.shape[1]
+    G = Hq // Hkv
+    g = guide_vectors(K)
+    sc = np.zeros((B, Hq, N), F64)
+    for b in range(B):
+        for h in range(Hq):
+            sc[b, h] = Q[b, h].astype(F64) @ g[b, h // G]
+    return sort_segments(sc, seg)
+
+
+def gather_queries(Q: np.ndarray, qperm: np.ndarray) -> np.ndarray:
+    """Qp[b, hq, p] = Q[b, hq, qperm[b, hq, p]]: the queries in permuted
+    order.  Selection on Qp pools each permuted query block."""
+    B, Hq, N, d = Q.shape
+    Qp = np.empty_like(Q)
+    for b in range(B):
+        for h in range(Hq):
+            Qp[b, h] = Q[b, h, qperm[b, h]]
+    return Qp
+
+
+def attn_block_qperm(Q, K, V, perm, qperm, listed, b, hq, i, blk, seg, scale):
+    """O [blk, d] and LSE [blk] (fp64) for permuted query block i of (b, hq):
+    rows are the queries at positions qperm[b, hq, i*blk + r].  Each row q
+    attends the keys of its own segment up to q (natural order, causal, as
+    in S2O's Pass 1) and the keys of the listed permuted blocks (all in
+    earlier segments).  Row r's results belong at position qperm[..]."""
+    Hq, Hkv = Q.shape[1], K.shape[1]
+    hk = hq // (Hq // Hkv)
+    q_pos = qperm[b, hq, i * blk:(i + 1) * blk].astype(np.int64)
+    q = Q[b, hq, q_pos].astype(F64)
+    s0 = segment_of_block(i, blk, seg) * seg
+    perm_row = perm_for_block(perm, b, hk, i, blk, seg)
+    keys = [perm_row[pb * blk:(pb + 1) * blk].astype(np.int64) for pb in listed]
+    keys.append(np.arange(s0, q_pos.max() + 1, dtype=np.int64))
+    keys = np.concatenate(keys)
+    vis = keys[None, :] <= q_pos[:, None]
+    logits = np.where(vis, (q @ K[b, hk, keys].astype(F64).T) * scale, -np.inf)
+    m = logits.max(axis=1, keepdims=True)
+    e = np.exp(logits - m)
+    l = e.sum(axis=1, keepdims=True)
+    return (e @ V[b, hk, keys].astype(F64)) / l, (m + np.log(l))[:, 0]
+
+
+def attn_qperm(Q, K, V, perm, qperm, lists: dict, blk: int, seg: int, scale: Optional[float] = None):
+    """O [B,Hq,N,d] and LSE [B,Hq,N] (fp64) at the queries' original
+    positions, for lists indexed by permuted query block (b, hq, i)."""
+    B, Hq, N, d = Q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    O = np.full((B, Hq, N, d), np.nan, F64)
+    L = np.full((B, Hq, N), np.nan, F64)
+    for b in range(B):
+        for h in range(Hq):
+            for i in range(N // blk):
+                listed = lists.get((b, h, i), np.zeros(0, np.int32))
+                o, lse = attn_block_qperm(Q, K, V, perm, qperm, listed, b, h, i, blk, seg, scale)
+                pos = qperm[b, h, i * blk:(i + 1) * blk]
+                O[b, h, pos] = o
+                L[b, h, pos] = lse
+    return O, L
+
+
 def lists_to_array(counts: np.ndarray, lists: dict, cap: int) -> np.ndarray:
     """Pack lists into idx[B,Hq,nb,cap] (unused entries -1)."""
     B, H, nb = counts.shape

@@ -765,3 +765,77 @@ def test_select_sample_single_sink_column():
             assert 0 in lists[(0, 0, i)].tolist(), i
         else:
             assert lists[(0, 0, i)].size == 0
+
+
+# ---------------------------------------------------------------------------
+# S2O query permutation (Technical Summary 1: Query Permutation); oracle
+# only, no GPU path yet
+# ---------------------------------------------------------------------------
+
+def test_permute_queries_orders_by_summed_logits():
+    """Within each segment the queries come in descending order of the sum
+    of their logits over all keys (explicit Q K^T row sums), equal sums in
+    ascending position; each segment maps onto itself."""
+    B, Hq, Hkv, N, d, seg = 1, 4, 2, 64, 8, 16
+    Q, K, V = _small(B, Hq, Hkv, N, d, seed=81, scale=2.0)
+    K[0, 0, :, :] = np.round(K[0, 0, :, :])                  # encourage exact ties
+    qperm = oracle.permute_queries(Q, K, seg)
+    G = Hq // Hkv
+    for h in range(Hq):
+        lg = Q[0, h].astype(np.float64) @ K[0, h // G].astype(np.float64).T
+        rowsum = lg.sum(axis=1)
+        for lo in range(0, N, seg):
+            p = qperm[0, h, lo:lo + seg]
+            assert sorted(p.tolist()) == list(range(lo, lo + seg))
+            sc = rowsum[p]
+            for a in range(seg - 1):
+                assert sc[a] > sc[a + 1] or (sc[a] == sc[a + 1] and p[a] < p[a + 1]), (h, lo, a)
+
+
+def test_attn_qperm_identity_is_natural_attention():
+    B, Hq, Hkv, N, d, blk, seg = 1, 2, 1, 128, 16, 16, 32
+    Q, K, V = _small(B, Hq, Hkv, N, d, seed=82)
+    perm = oracle.permute(Q, K, blk, seg)
+    _, lists = oracle.select(Q, K, perm, blk, seg, "topk", density=0.4)
+    ident = np.broadcast_to(np.arange(N, dtype=np.int32), (B, Hq, N)).copy()
+    O1, L1 = oracle.attn_qperm(Q, K, V, perm, ident, lists, blk, seg)
+    O2, L2 = oracle.attn(Q, K, V, perm, lists, blk, seg)
+    assert np.max(np.abs(O1 - O2)) < 1e-12 and np.max(np.abs(L1 - L2)) < 1e-12
+
+
+def test_attn_qperm_matches_position_mask():
+    """With permuted queries, row q (in permuted block i) sees its own
+    segment up to q and the keys of block i's listed permuted blocks: equal to
+    torch SDPA with that mask built position by position."""
+    B, Hq, Hkv, N, d, blk, seg = 1, 2, 1, 128, 16, 16, 64
+    Q, K, V = _small(B, Hq, Hkv, N, d, seed=83, scale=1.5)
+    perm = oracle.permute(Q, K, blk, seg)
+    qperm = oracle.permute_queries(Q, K, seg)
+    Qp = oracle.gather_queries(Q, qperm)
+    _, lists = oracle.select(Qp, K, perm, blk, seg, "topk", density=0.3)
+    O, L = oracle.attn_qperm(Q, K, V, perm, qperm, lists, blk, seg)
+    for h in range(Hq):
+        inv = np.empty(N, np.int64)
+        inv[qperm[0, h]] = np.arange(N)
+        mask = np.zeros((N, N), bool)
+        for q in range(N):
+            i = inv[q] // blk
+            s0 = (q // seg) * seg
+            mask[q, s0:q + 1] = True
+            for pb in lists.get((0, h, i), []):
+                mask[q, perm[0, 0, pb * blk:(pb + 1) * blk]] = True
+        ref = _sdpa(Q[0, h][None], K[0, 0][None], V[0, 0][None], mask=mask[None])[0]
+        assert np.max(np.abs(O[0, h] - ref)) < 1e-12, h
+
+
+def test_attn_qperm_dense_lists_give_causal_attention():
+    """Listing every candidate makes each row's key set its whole causal
+    prefix, whatever the query order."""
+    B, Hq, Hkv, N, d, blk, seg = 1, 2, 1, 128, 16, 16, 32
+    Q, K, V = _small(B, Hq, Hkv, N, d, seed=84)
+    perm = oracle.permute(Q, K, blk, seg)
+    qperm = oracle.permute_queries(Q, K, seg)
+    _, lists = oracle.dense_lists(B, Hq, N // blk, blk, seg)
+    O, L = oracle.attn_qperm(Q, K, V, perm, qperm, lists, blk, seg)
+    ref = _sdpa(Q, np.repeat(K, Hq // Hkv, axis=1), np.repeat(V, Hq // Hkv, axis=1), causal=True)
+    assert np.max(np.abs(O - ref)) < 1e-12
