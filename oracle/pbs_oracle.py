@@ -48,6 +48,10 @@ leave a step open the plainest reading is taken; the readings are:
   * a gated tile is excluded entirely; the query block's own tile is never
     gated; thresholds and tile maxima are raw (unscaled) q.k values.
 
+The variants beside the main path (S2O early stopping, one key permutation
+per query segment, S2O's query permutation, the SampleAttention-style
+selector, attention coverage) carry their own readings in their docstrings.
+
 Parity pins: tests/test_oracle_pins.py checks every function here against
 brute force, closed forms, library routines and invariants.
 """
