@@ -409,6 +409,25 @@ def test_inputs_are_bf16_exact_lattice():
     assert np.array_equal(Q, Q2) and np.array_equal(K, K2)
 
 
+def test_local_window_recipe():
+    """The planted local window draws no random numbers (without it the
+    same seed gives the same Q and K as before, up to the positional
+    vector), keeps values bf16-exact, and raises q.k near the diagonal."""
+    base = synth.WORKLOADS["sample_32k_local"].with_(N=2048, seg=512, Hq=4, Hkv=1)
+    Q, K, V, _ = synth.make_inputs(base)
+    Q0, K0, V0, _ = synth.make_inputs(base.with_(local_amp=0.0))
+    assert np.array_equal(V, V0)                     # V never gets the positional vector
+    for X in (Q, K):
+        assert np.all(X * 8 == np.round(X * 8)) and np.abs(X).max() <= 31.875
+    lg = Q[0, 0].astype(np.float64) @ K[0, 0].astype(np.float64).T
+    n = np.arange(base.N)
+    near = np.abs(n[:, None] - n[None, :]) < 8
+    far = np.abs(n[:, None] - n[None, :]) > 512
+    assert lg[near].mean() > lg[far].mean() + 50.0
+    lg0 = Q0[0, 0].astype(np.float64) @ K0[0, 0].astype(np.float64).T
+    assert abs(lg0[near].mean() - lg0[far].mean()) < 5.0
+
+
 def test_stripe_keys_cluster_in_leading_blocks():
     """With planted stripes, the permutation must gather the stripe keys into
     the first permuted block of their segment (the clustering the method is
