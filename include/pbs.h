@@ -143,7 +143,12 @@ int pbs_permute_segmented(const pbs_tensor* Q, const pbs_tensor* K, int blk, int
                           int32_t* perm, void* ws, size_t ws_bytes, void* stream);
 
 /* Upper bound on the list length pbs_select can produce for these settings
- * (host-only arithmetic).  Pass at least this as `cap`.                    */
+ * (host-only arithmetic).  Pass at least this as `cap`.  For
+ * PBS_SELECT_TAU and PBS_SELECT_SAMPLE it is the largest number of
+ * candidate blocks (the permuted or natural blocks of earlier segments);
+ * for PBS_SELECT_TOPK the top-k budget plus the forced band and sink
+ * blocks, capped by the candidates.  The flag bits of mode are ignored.
+ * Returns PBS_ERR_INVALID_ARG for a bad geometry.                          */
 int pbs_select_capacity(int64_t N, int blk, int seg, int mode,
                         double density_or_tau, int band, int n_sink);
 
