@@ -858,3 +858,64 @@ def test_attn_qperm_dense_lists_give_causal_attention():
     O, L = oracle.attn_qperm(Q, K, V, perm, qperm, lists, blk, seg)
     ref = _sdpa(Q, np.repeat(K, Hq // Hkv, axis=1), np.repeat(V, Hq // Hkv, axis=1), causal=True)
     assert np.max(np.abs(O - ref)) < 1e-12
+
+
+# ---------------------------------------------------------------------------
+# property-based variants of the brute-force pins (random shapes and seeds)
+# ---------------------------------------------------------------------------
+
+from hypothesis import given, settings, strategies as st  # noqa: E402
+
+
+@settings(max_examples=25, deadline=None)
+@given(seed=st.integers(0, 10_000), G=st.sampled_from([1, 2]), blk=st.sampled_from([4, 8]),
+       spb=st.sampled_from([2, 3]), nseg=st.sampled_from([2, 3, 4]), density=st.sampled_from([0.1, 0.25, 0.5]),
+       n_sink=st.sampled_from([0, 4]))
+def test_topk_selection_brute_force_random(seed, G, blk, spb, nseg, density, n_sink):
+    d, Hkv = 8, 1
+    seg = blk * spb
+    N = seg * nseg
+    Q, K, V = _small(1, G * Hkv, Hkv, N, d, seed=seed, scale=2.0)
+    perm = oracle.permute(Q, K, blk, seg, n_sink)
+    counts, lists = oracle.select(Q, K, perm, blk, seg, "topk", density=density, n_sink=n_sink)
+    for h in range(G):
+        inv = oracle.inverse_permutation(perm[0, 0])
+        for i in range(N // blk):
+            s = i // spb
+            ncand, D = s * spb, i - s * spb + 1
+            if ncand == 0:
+                assert counts[0, h, i] == 0
+                continue
+            S = [_tile_logit_sum(Q, K, perm, 0, h, i, pb, blk, G) for pb in range(ncand)]
+            forced = {int(inv[pos]) // blk for pos in range(min(n_sink, s * seg))}
+            k = max(D + len(forced), math.ceil(Fraction(round(density * 1000), 1000) * (i + 1)))
+            k = min(k, D + ncand)
+            assert list(lists[(0, h, i)]) == _brute_topk(S, forced, k - D), (h, i)
+
+
+@settings(max_examples=20, deadline=None)
+@given(seed=st.integers(0, 10_000), blk=st.sampled_from([4, 8]), spb=st.sampled_from([2, 4]),
+       nseg=st.sampled_from([2, 3]), keep=st.floats(0.0, 1.0))
+def test_attention_matches_position_mask_random(seed, blk, spb, nseg, keep):
+    """Any lists of candidate blocks: the oracle equals torch fp64 SDPA with
+    the key set built position by position (own segment causal, plus the
+    listed permuted blocks' keys)."""
+    d, seg = 8, blk * spb
+    N = seg * nseg
+    Q, K, V = _small(1, 1, 1, N, d, seed=seed, scale=1.5)
+    perm = oracle.permute(Q, K, blk, seg)
+    rng = np.random.default_rng(seed)
+    lists = {}
+    for i in range(N // blk):
+        ncand = (i // spb) * spb
+        chosen = [pb for pb in range(ncand) if rng.random() < keep]
+        lists[(0, 0, i)] = np.array(chosen, np.int32)
+    O, L = oracle.attn(Q, K, V, perm, lists, blk, seg)
+    mask = np.zeros((N, N), bool)
+    for q in range(N):
+        i, s0 = q // blk, (q // seg) * seg
+        mask[q, s0:q + 1] = True
+        for pb in lists[(0, 0, i)]:
+            mask[q, perm[0, 0, pb * blk:(pb + 1) * blk]] = True
+    ref = _sdpa(Q[0, 0][None], K[0, 0][None], V[0, 0][None], mask=mask[None])[0]
+    assert np.max(np.abs(O[0, 0] - ref)) < 1e-12
