@@ -919,3 +919,40 @@ def test_attention_matches_position_mask_random(seed, blk, spb, nseg, keep):
             mask[q, perm[0, 0, pb * blk:(pb + 1) * blk]] = True
     ref = _sdpa(Q[0, 0][None], K[0, 0][None], V[0, 0][None], mask=mask[None])[0]
     assert np.max(np.abs(O[0, 0] - ref)) < 1e-12
+
+
+@settings(max_examples=40, deadline=None)
+@given(seed=st.integers(0, 10_000), n=st.integers(1, 9), alpha=st.floats(0.01, 0.999),
+       ties=st.booleans())
+def test_cumulative_cut_random(seed, n, alpha, ties):
+    """The cut is a smallest set of entries reaching alpha of the total, made
+    of the highest scores, equal scores taken in ascending index."""
+    rng = np.random.default_rng(seed)
+    sc = rng.random(n)
+    if ties:
+        sc = np.round(sc * 3) / 3                      # repeated values
+    if sc.sum() == 0:
+        sc[0] = 1.0
+    keep = oracle.cumulative_cut(sc, alpha)
+    goal = alpha * sc.sum()
+    assert sc[keep].sum() >= goal - 1e-12
+    smallest = next(size for size in range(n + 1)
+                    if any(sum(sc[list(c)]) >= goal for c in itertools.combinations(range(n), size)))
+    assert keep.sum() == smallest
+    order = sorted(range(n), key=lambda x: (-sc[x], x))
+    assert np.flatnonzero(keep).tolist() == sorted(order[:smallest])
+
+
+@settings(max_examples=25, deadline=None)
+@given(seed=st.integers(0, 10_000), seg=st.sampled_from([3, 5, 8]), nseg=st.integers(1, 3),
+       ties=st.booleans())
+def test_sort_segments_random(seed, seg, nseg, ties):
+    rng = np.random.default_rng(seed)
+    N = seg * nseg - (seed % seg if nseg > 1 else 0)          # ragged last segment
+    sc = rng.standard_normal((1, 1, N))
+    if ties:
+        sc = np.round(sc)
+    perm = oracle.sort_segments(sc, seg)
+    for lo in range(0, N, seg):
+        hi = min(lo + seg, N)
+        assert perm[0, 0, lo:hi].tolist() == [lo + x for x in _brute_force_segment_order(list(sc[0, 0, lo:hi]))]
