@@ -956,3 +956,52 @@ def test_sort_segments_random(seed, seg, nseg, ties):
     for lo in range(0, N, seg):
         hi = min(lo + seg, N)
         assert perm[0, 0, lo:hi].tolist() == [lo + x for x in _brute_force_segment_order(list(sc[0, 0, lo:hi]))]
+
+
+@settings(max_examples=20, deadline=None)
+@given(seed=st.integers(0, 10_000), tau_q=st.floats(0.05, 0.95))
+def test_early_stop_brute_force_random(seed, tau_q):
+    """Random inputs and a threshold at a random quantile of the explicit
+    gains: the early-stopped block equals masked attention over the prefix
+    of the visiting order that ends at the first tile below the threshold."""
+    blk, seg, d = 8, 32, 8
+    Q, K, V = _small(1, 1, 1, 160, d, seed=seed, scale=2.0)
+    perm = oracle.permute(Q, K, blk, seg)
+    _, lists = oracle.select(Q, K, perm, blk, seg, "topk", density=1.0, list_order="score")
+    scale = 1.0 / math.sqrt(d)
+    for (b, h, i), listed in lists.items():
+        if listed.size < 2:
+            continue
+        gains = _explicit_gains(Q, K, perm, h, i, listed, blk, seg, scale)
+        tau = float(np.quantile(gains, tau_q))
+        if min(abs(g - tau) for g in gains) < 1e-9 * max(tau, 1e-300):
+            tau *= 1.0 + 1e-6                                   # keep the decision away from ties
+        k_star = next((k + 1 for k, g in enumerate(gains) if g < tau), len(gains))
+        O, L, n = oracle.attn_early_stop_block(Q, K, V, perm, listed, b, h, i, blk, seg, scale, tau)
+        O_ref, L_ref = oracle.attn_block(Q, K, V, perm, listed[:k_star], b, h, i, blk, seg, scale)
+        assert n == k_star, (i, tau)
+        np.testing.assert_allclose(O, O_ref, rtol=0, atol=1e-12)
+
+
+@settings(max_examples=20, deadline=None)
+@given(seed=st.integers(0, 10_000), tau=st.sampled_from([0.3, 0.6, 0.9, 0.99]))
+def test_tau_selection_brute_force_random(seed, tau):
+    B, Hq, Hkv, N, d, blk, seg = 1, 1, 1, 96, 8, 8, 24
+    Q, K, V = _small(B, Hq, Hkv, N, d, seed=seed, scale=3.0)
+    perm = oracle.permute(Q, K, blk, seg)
+    counts, lists = oracle.select(Q, K, perm, blk, seg, "tau", tau=tau)
+    spb = seg // blk
+    scale = 1.0 / (blk * blk * math.sqrt(d))
+    for i in range(N // blk):
+        s = i // spb
+        ncand = s * spb
+        if ncand == 0:
+            continue
+        lc = [_tile_logit_sum(Q, K, perm, 0, 0, i, pb, blk, 1) * scale for pb in range(ncand)]
+        ld = [_nat_tile_logit_sum(Q, K, 0, 0, i, j, blk, 1) * scale for j in range(s * spb, i + 1)]
+        p = torch.softmax(torch.tensor(lc + ld, dtype=torch.float64), 0).numpy()
+        # decisions within 1e-12 of tau are left to rounding on both sides
+        cum = np.cumsum(np.sort(p[:ncand])[::-1]) + p[ncand:].sum()
+        if np.min(np.abs(cum - tau)) < 1e-12 or abs(p[ncand:].sum() - tau) < 1e-12:
+            continue
+        assert list(lists[(0, 0, i)]) == _brute_tau(p[ncand:], p[:ncand], set(), tau), i
