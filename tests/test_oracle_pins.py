@@ -1005,3 +1005,44 @@ def test_tau_selection_brute_force_random(seed, tau):
         if np.min(np.abs(cum - tau)) < 1e-12 or abs(p[ncand:].sum() - tau) < 1e-12:
             continue
         assert list(lists[(0, 0, i)]) == _brute_tau(p[ncand:], p[:ncand], set(), tau), i
+
+
+@settings(max_examples=15, deadline=None)
+@given(seed=st.integers(0, 10_000), blk=st.sampled_from([4, 8]), spb=st.sampled_from([2, 3]),
+       nseg=st.sampled_from([2, 3]), alpha=st.floats(0.2, 1.0))
+def test_select_sample_position_mask_random(seed, blk, spb, nseg, alpha):
+    """Random shapes: the block lists are the blocks touched by the
+    position-level column/slash mask, restricted to earlier segments."""
+    d, seg = 8, blk * spb
+    N = seg * nseg
+    Q, K, V = _small(1, 1, 1, N, d, seed=seed, scale=2.0)
+    counts, lists = oracle.select_sample(Q, K, blk, seg, alpha)
+    col, sl = oracle.sample_pattern_scores(Q, K, 0, 0, blk, seg, 1.0 / math.sqrt(d))
+    kc, ks = oracle.cumulative_cut(col, alpha), oracle.cumulative_cut(sl, alpha)
+    for i in range(N // blk):
+        ncand = oracle.n_candidates(i, blk, seg)
+        want = {k // blk for q in range(i * blk, (i + 1) * blk) for k in range(ncand * blk)
+                if k <= q and (kc[k] or ks[q - k])}
+        assert lists[(0, 0, i)].tolist() == sorted(want), i
+
+
+@settings(max_examples=15, deadline=None)
+@given(seed=st.integers(0, 10_000), seg=st.sampled_from([4, 6]), nseg=st.integers(2, 3))
+def test_permute_segmented_random(seed, seg, nseg):
+    """Random inputs: for query segment s, every key segment before s is in
+    descending order of its score against s's summed queries (stable), and
+    every later key segment keeps its natural order."""
+    d, blk = 8, 2
+    N = seg * nseg
+    Q, K, V = _small(1, 2, 1, N, d, seed=seed, scale=2.0)
+    perm = oracle.permute_segmented(Q, K, blk, seg)
+    for t in range(nseg):
+        qsum = Q[0, :, t * seg:(t + 1) * seg].astype(np.float64).reshape(-1, d).sum(axis=0)
+        sc = K[0, 0].astype(np.float64) @ qsum
+        for j in range(nseg):
+            got = perm[0, 0, t, j * seg:(j + 1) * seg].tolist()
+            if j < t:
+                ref = [j * seg + x for x in _brute_force_segment_order(list(sc[j * seg:(j + 1) * seg]))]
+            else:
+                ref = list(range(j * seg, (j + 1) * seg))
+            assert got == ref, (t, j)
