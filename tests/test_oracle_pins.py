@@ -1046,3 +1046,31 @@ def test_permute_segmented_random(seed, seg, nseg):
             else:
                 ref = list(range(j * seg, (j + 1) * seg))
             assert got == ref, (t, j)
+
+
+@settings(max_examples=12, deadline=None)
+@given(seed=st.integers(0, 10_000), keep=st.integers(1, 5), nb=st.integers(2, 8))
+def test_gate_brute_force_random(seed, keep, nb):
+    """Random inputs: thresholds are the keep-th largest brute-force tile
+    maximum (or -inf), and gated attention equals SDPA over the kept tiles
+    (the own tile always kept)."""
+    blk, d = 4, 8
+    N = nb * blk
+    Q, K, V = _small(1, 1, 1, N, d, seed=seed, scale=2.0)
+    perm = np.arange(N, dtype=np.int32)[None, None].copy()
+    _, lists = oracle.dense_lists(1, 1, nb, blk, blk)
+    thr = oracle.calibrate_thresholds(Q, K, blk, keep)
+    Og, _ = oracle.attn(Q, K, V, perm, lists, blk, blk, gate_thr=thr)
+    mask = np.zeros((N, N), bool)
+    for i in range(nb):
+        qpos = np.arange(i * blk, (i + 1) * blk)
+        M = [_brute_tile_max(Q[0, 0, qpos], K[0, 0, j * blk:(j + 1) * blk], qpos, np.arange(j * blk, (j + 1) * blk))
+             for j in range(i + 1)]
+        t = -math.inf if i + 1 <= keep else sorted(M, reverse=True)[keep - 1]
+        assert t == thr[0, 0, i]
+        for j in range(i + 1):
+            if j == i or M[j] >= t:
+                for a in qpos:
+                    mask[a, j * blk:min((j + 1) * blk, a + 1)] = True
+    ref = _sdpa(Q[0, 0], K[0, 0], V[0, 0], mask=mask)
+    assert np.max(np.abs(Og[0, 0] - ref)) < 1e-12
