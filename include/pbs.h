@@ -87,7 +87,7 @@ enum { PBS_SELECT_TOPK = 0, PBS_SELECT_TAU = 1, PBS_SELECT_SAMPLE = 2 };
  * one permutation per query segment (see there). */
 enum { PBS_SELECT_SCORE_ORDER = 0x10, PBS_SELECT_PERM_PER_SEGMENT = 0x20 };
 /* pbs_attn_fwd_ex flags. */
-enum { PBS_ATTN_EARLY_STOP = 1, PBS_ATTN_PERM_PER_SEGMENT = 2 };
+enum { PBS_ATTN_EARLY_STOP = 1, PBS_ATTN_PERM_PER_SEGMENT = 2, PBS_ATTN_CTA_PAIR = 4 };
 
 /* Bytes of workspace the given op needs for these shapes (0 if none).
  * Q and K may not be NULL; only their shapes are read.                     */
@@ -116,8 +116,11 @@ int pbs_permute(const pbs_tensor* Q, const pbs_tensor* K, int blk, int seg,
  * every GPU that loads the library until the process exits), so
  * B * Hkv * D must not exceed 65536; larger inputs return PBS_ERR_CAPACITY.
  * The call allocates nothing.  Its first call on a device looks up the
- * array's device address with that device current; make that first call
- * before any stream capture.  All calls on a device share the array and it
+ * array's device address with that device current and keeps it for the
+ * life of the process; make that first call before any stream capture.  The
+ * kept address belongs to the device's primary context: do not use this
+ * entry point from another context of the device, or after
+ * cudaDeviceReset() on it.  All calls on a device share the array and it
  * keeps the last call's contents (each call overwrites what it reads), so
  * calls whose GPU work may overlap race and must not be issued together.    */
 int pbs_permute_noalloc(const pbs_tensor* Q, const pbs_tensor* K, int blk, int seg,
@@ -248,7 +251,14 @@ int pbs_attn_fwd_early_stop(const pbs_tensor* Q, const pbs_tensor* K, const pbs_
  *   flags: PBS_ATTN_EARLY_STOP -- lists in visiting order, stop_tau as for
  *            pbs_attn_fwd_early_stop (gate_thr must then be NULL);
  *          PBS_ATTN_PERM_PER_SEGMENT -- perm is [B, Hkv, nseg, N] from
- *            pbs_permute_segmented and each query block reads its segment's.
+ *            pbs_permute_segmented and each query block reads its segment's;
+ *          PBS_ATTN_CTA_PAIR -- where D = blk = 128, Hq / Hkv is a multiple
+ *            of 4 and neither gating nor early stopping is asked for, run
+ *            the CTA-pair kernel: four query heads of a KV head per cluster
+ *            of two CTAs, tensor-core MMAs spanning both (M = 256), each CTA
+ *            gathering half of every K/V tile.  Same results (the same
+ *            arithmetic per head, bit for bit); elsewhere the flag is
+ *            ignored.
  *   Other arguments as for pbs_attn_fwd; unknown flags are rejected.       */
 int pbs_attn_fwd_ex(const pbs_tensor* Q, const pbs_tensor* K, const pbs_tensor* V, const int32_t* perm,
                     const int32_t* counts, const int32_t* idx, int cap, int blk, int seg, unsigned flags,
@@ -258,6 +268,18 @@ int pbs_attn_fwd_ex(const pbs_tensor* Q, const pbs_tensor* K, const pbs_tensor* 
 /* Synchronises `stream`, then returns and clears the sticky device error
  * word of the current device (PBS_OK if no device-side check failed).      */
 int pbs_check_device(void* stream);
+
+/* pbs_test_inject_timeout: a test hook for the failure path; the pages have
+ * no counterpart.  With limit_polls > 0, every later pbs_attn_fwd* launch
+ * (from any host thread) withholds the "query tile landed" arrival that its
+ * MMA role waits for, and bounds the waits of the producer, MMA and softmax
+ * roles by limit_polls polls: the wait for the query tile runs out, the
+ * kernel raises its abort flag, every role leaves its loop, the tensor core
+ * is drained (that wait keeps its normal bound), tensor memory is freed and
+ * PBS_ERR_TIMEOUT is left in the device error word, with no fault.
+ * limit_polls = 0 (the default) turns the hook off.  Not for production
+ * use: outputs of a launch made while it is on are undefined.             */
+void pbs_test_inject_timeout(unsigned limit_polls);
 
 /* Message of the most recent failing call on this host thread ("" if none). */
 const char* pbs_get_last_error(void);

@@ -23,12 +23,12 @@ PBS_OP_SELECT_SAMPLE = 5
 PBS_SELECT_TOPK, PBS_SELECT_TAU, PBS_SELECT_SAMPLE = 0, 1, 2
 _MODES = {"topk": PBS_SELECT_TOPK, "tau": PBS_SELECT_TAU, "sample": PBS_SELECT_SAMPLE}
 PBS_SELECT_SCORE_ORDER, PBS_SELECT_PERM_PER_SEGMENT = 0x10, 0x20
-PBS_ATTN_EARLY_STOP, PBS_ATTN_PERM_PER_SEGMENT = 1, 2
+PBS_ATTN_EARLY_STOP, PBS_ATTN_PERM_PER_SEGMENT, PBS_ATTN_CTA_PAIR = 1, 2, 4
 STATUS = {0: "PBS_OK", -1: "PBS_ERR_INVALID_ARG", -2: "PBS_ERR_UNSUPPORTED", -3: "PBS_ERR_CAPACITY",
           -4: "PBS_ERR_CUDA", -5: "PBS_ERR_TIMEOUT", -6: "PBS_ERR_DEVICE_CHECK"}
 EXPORTS = ("pbs_workspace_size", "pbs_permute", "pbs_permute_segmented", "pbs_select_capacity", "pbs_select",
            "pbs_attn_fwd", "pbs_attn_fwd_early_stop", "pbs_attn_fwd_ex", "pbs_check_device",
-           "pbs_get_last_error", "pbs_version")
+           "pbs_get_last_error", "pbs_version", "pbs_permute_noalloc", "pbs_test_inject_timeout")
 
 
 class PbsError(RuntimeError):
@@ -76,6 +76,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.pbs_attn_fwd_early_stop.restype = i32
     lib.pbs_check_device.argtypes = [vp]
     lib.pbs_check_device.restype = i32
+    lib.pbs_test_inject_timeout.argtypes = [ctypes.c_uint]
+    lib.pbs_test_inject_timeout.restype = None
     lib.pbs_get_last_error.argtypes = []
     lib.pbs_get_last_error.restype = ctypes.c_char_p
     lib.pbs_version.argtypes = []
@@ -219,8 +221,10 @@ def pbs_attn_fwd(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, perm: torch.
                  gate_thr: Optional[torch.Tensor] = None, softmax_scale: Optional[float] = None,
                  out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
                  want_lse: bool = True, stats: Optional[torch.Tensor] = None,
-                 stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
-    """(O [B, Hq, N, D] bf16, LSE [B, Hq, N] fp32 or None)."""
+                 stream=None, cta_pair: bool = False) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """(O [B, Hq, N, D] bf16, LSE [B, Hq, N] fp32 or None).  ``cta_pair``
+    runs the CTA-pair kernel where it applies (d = blk = 128, query heads per
+    KV head a multiple of 4, no gate); its results are the same."""
     lib = load()
     B, Hq, N, D = Q.shape
     if out is None:
@@ -234,10 +238,11 @@ def pbs_attn_fwd(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, perm: torch.
     if stats is not None and stats.dtype != torch.int64:
         raise TypeError("stats must be int64")
     q, k, v, o = describe(Q), describe(K), describe(V), describe(out)
-    if perm.dim() == 4:                      # one permutation per query segment
+    flags = (PBS_ATTN_PERM_PER_SEGMENT if perm.dim() == 4 else 0) | (PBS_ATTN_CTA_PAIR if cta_pair else 0)
+    if flags:                                # one permutation per query segment / one-CTA kernel
         _check(lib.pbs_attn_fwd_ex(ctypes.byref(q), ctypes.byref(k), ctypes.byref(v), perm.data_ptr(),
                                    counts.data_ptr(), idx.data_ptr(), idx.shape[-1], blk, seg,
-                                   PBS_ATTN_PERM_PER_SEGMENT, _ptr(gate_thr), 0.0, float(softmax_scale),
+                                   flags, _ptr(gate_thr), 0.0, float(softmax_scale),
                                    ctypes.byref(o), _ptr(lse), _ptr(stats), _stream(stream)))
         return out, lse
     _check(lib.pbs_attn_fwd(ctypes.byref(q), ctypes.byref(k), ctypes.byref(v), perm.data_ptr(),
@@ -283,6 +288,12 @@ def pbs_attn_fwd_early_stop(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, p
 def pbs_check_device(stream=None) -> None:
     """Synchronise and raise if a device-side check or bounded wait failed."""
     _check(load().pbs_check_device(_stream(stream)))
+
+
+def test_inject_timeout(limit_polls: int) -> None:
+    """Failure-path test hook (see pbs.h): > 0 makes later attention launches
+    time out on purpose (bounded waits, no fault); 0 turns it off."""
+    load().pbs_test_inject_timeout(int(limit_polls))
 
 
 def version() -> str:

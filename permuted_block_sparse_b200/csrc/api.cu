@@ -2,7 +2,9 @@
 // the sticky device error word, and kernel launches.  See include/pbs.h for
 // the contract of every entry point.
 #include <algorithm>
+#include <atomic>
 #include <cmath>
+#include <mutex>
 #include <cstdarg>
 #include <cstdio>
 #include <string>
@@ -18,6 +20,9 @@ __device__ int g_device_error = 0;
 namespace {
 
 thread_local std::string g_last_error;
+
+// Failure-path test hook (pbs_test_inject_timeout): 0 in normal use.
+std::atomic<unsigned> g_test_wait_limit{0};
 
 int fail(int code, const char* fmt, ...) {
   char buf[512];
@@ -42,9 +47,11 @@ size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 // Device address of the error word, cached per device.
 int* device_error_word() {
+  static std::mutex mu;
   static int* cache[128] = {nullptr};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
   if (!cache[dev]) {
     void* ptr = nullptr;
     if (cudaGetSymbolAddress(&ptr, pbs::g_device_error) != cudaSuccess) return nullptr;
@@ -155,7 +162,8 @@ namespace {
 int attn_common(const pbs_tensor* Qt, const pbs_tensor* Kt, const pbs_tensor* Vt,
                 const int32_t* perm, const int32_t* counts, const int32_t* idx, int cap, int blk,
                 int seg, const float* gate_thr, int early_stop, float stop_tau, int per_segment,
-                float softmax_scale, pbs_tensor* Ot, float* lse, long long* stats, void* stream) {
+                float softmax_scale, pbs_tensor* Ot, float* lse, long long* stats, void* stream,
+                int cta_pair = 0) {
   pbs::TensorDesc Q, K, V, O;
   int rc;
   if ((rc = check_tensor(Qt, "Q", &Q)) || (rc = check_tensor(Kt, "K", &K)) ||
@@ -189,6 +197,8 @@ int attn_common(const pbs_tensor* Qt, const pbs_tensor* Kt, const pbs_tensor* Vt
   p.early_stop = early_stop;
   p.stop_tau = stop_tau;
   p.perm_nseg = per_segment ? static_cast<int>((Q.N + seg - 1) / seg) : 1;
+  p.cta_pair = cta_pair;
+  p.test_wait_limit = g_test_wait_limit.load();
   p.scale_log2 = softmax_scale * 1.4426950408889634f;
   p.lse = lse;
   p.stats = stats;
@@ -411,7 +421,7 @@ int pbs_attn_fwd_ex(const pbs_tensor* Qt, const pbs_tensor* Kt, const pbs_tensor
                     const int32_t* counts, const int32_t* idx, int cap, int blk, int seg, unsigned flags,
                     const float* gate_thr, float stop_tau, float softmax_scale, pbs_tensor* Ot, float* lse,
                     long long* stats, void* stream) {
-  if (flags & ~static_cast<unsigned>(PBS_ATTN_EARLY_STOP | PBS_ATTN_PERM_PER_SEGMENT))
+  if (flags & ~static_cast<unsigned>(PBS_ATTN_EARLY_STOP | PBS_ATTN_PERM_PER_SEGMENT | PBS_ATTN_CTA_PAIR))
     return fail(PBS_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
   const int early = (flags & PBS_ATTN_EARLY_STOP) ? 1 : 0;
   if (early) {
@@ -420,8 +430,11 @@ int pbs_attn_fwd_ex(const pbs_tensor* Qt, const pbs_tensor* Kt, const pbs_tensor
       return fail(PBS_ERR_INVALID_ARG, "stop_tau must be finite and >= 0");
   }
   return attn_common(Qt, Kt, Vt, perm, counts, idx, cap, blk, seg, gate_thr, early, early ? stop_tau : 0.0f,
-                     (flags & PBS_ATTN_PERM_PER_SEGMENT) ? 1 : 0, softmax_scale, Ot, lse, stats, stream);
+                     (flags & PBS_ATTN_PERM_PER_SEGMENT) ? 1 : 0, softmax_scale, Ot, lse, stats, stream,
+                     (flags & PBS_ATTN_CTA_PAIR) ? 1 : 0);
 }
+
+void pbs_test_inject_timeout(unsigned limit_polls) { g_test_wait_limit.store(limit_polls); }
 
 int pbs_check_device(void* stream) {
   cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));

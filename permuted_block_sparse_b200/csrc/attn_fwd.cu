@@ -247,6 +247,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
   tc_fence_after();
   const uint32_t tmem = sh.tmem_base;
   const int T = n_diag + sh.n_union;
+  // Poll limit of the role waits (the drain before tensor memory is freed
+  // keeps the full limit).
+  const uint32_t lim = p.test_wait_limit ? p.test_wait_limit : kSpinLimit;
   const uint32_t both = has1 ? 3u : 1u;
   volatile int* abort_flag = &sh.abort;
   volatile int* limit = sh.limit;
@@ -301,7 +304,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
                          valid ? qb + (q0 + r) * p.Q.sN + c * 8 : qb, valid);
       }
     }
-    cp_async_mbar_arrive(&sh.bar_q);
+    // (the failure-path test hook withholds this arrival, so the MMA role's
+    // wait for Q runs out)
+    if (!p.test_wait_limit) cp_async_mbar_arrive(&sh.bar_q);
     // Row indices of a tile: natural rows, or the permutation's entries for
     // a permuted block.  Loaded one tile ahead into registers and checked
     // when used, so the load latency overlaps the previous tile.
@@ -321,9 +326,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
     // nothing is run.
     auto wait_slot = [&](uint64_t* bar, uint32_t parity, int t) -> bool {
       if constexpr (!ES) {
-        return mbar_wait_or_abort(bar, parity, p.err, abort_flag);
+        return mbar_wait_or_abort(bar, parity, p.err, abort_flag, lim);
       } else {
-        for (uint32_t it = 0; it < kSpinLimit; ++it) {
+        for (uint32_t it = 0; it < lim; ++it) {
           if (mbar_try_wait(bar, parity)) return true;
           if ((it & 15u) == 15u && (*abort_flag || past_all(t))) return false;
         }
@@ -389,7 +394,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
     bool ok = true;
     {
       bool v = true;
-      if (leader) v = mbar_wait_or_abort(&sh.bar_q, 0, p.err, abort_flag);
+      if (leader) v = mbar_wait_or_abort(&sh.bar_q, 0, p.err, abort_flag, lim);
       ok = __shfl_sync(0xffffffffu, v, 0);
       if (leader) fence_proxy_async();   // cp.async (generic proxy) writes -> tensor-core reads
       tc_fence_after();
@@ -538,7 +543,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
         if (!pending) break;
         if (progress) {
           idle = 0;
-        } else if (++idle >= 4u * kSpinLimit) {
+        } else if (++idle >= 4u * lim) {
           if (leader) {
             set_error(p.err, kErrTimeout);
             *abort_flag = 1;
@@ -578,14 +583,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
     bool ok = true;
     for (int t = 0; active && t < T; ++t) {
       if (!((tile_mask(t) >> h) & 1u)) continue;
-      if (!mbar_wait_or_abort(&sh.bar_s[h], k & 1, p.err, abort_flag)) ok = false;
+      if (!mbar_wait_or_abort(&sh.bar_s[h], k & 1, p.err, abort_flag, lim)) ok = false;
       tc_fence_after();
       ++n_qk;
       // Block-max gate first: the tile's raw maximum over all rows decides
       // before any exponential is taken, so a dropped tile costs one read of
       // S and a reduction.  A dropped tile leaves m, l and O as they were;
-      // the diagonal tile (t == 0) is never gated.
-      if (p.gate_thr && t != 0) {
+      // the diagonal tile (t == 0) is never gated.  A row whose threshold is
+      // -inf (no more causal tiles than the calibration keeps) can never drop
+      // a tile, so its warpgroup skips the gate altogether: thr is the same
+      // for every thread of the warpgroup, so this costs no divergence.
+      if (p.gate_thr && t != 0 && thr > -INFINITY) {
         float rm = -INFINITY;
 #pragma unroll 1
         for (int c = 0; c < BLK / 64; ++c) {
@@ -747,7 +755,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
     // ---- epilogue: O / l -> bf16, LSE
     if (active) ok = !named_sync_or(2 + h, 128, !ok);  // one vote for the whole loop
     if (active && ok && k > 0) {
-      ok = mbar_wait_or_abort(&sh.bar_o[h], 0, p.err, abort_flag);
+      ok = mbar_wait_or_abort(&sh.bar_o[h], 0, p.err, abort_flag, lim);
       ok = !named_sync_or(2 + h, 128, !ok);
       tc_fence_after();
     }
@@ -817,6 +825,7 @@ cudaError_t launch_mode(const AttnParams& p, cudaStream_t s) {
 cudaError_t launch_attn_fwd(const AttnParams& p, cudaStream_t s) {
   const int D = static_cast<int>(p.Q.D);
   if (p.nb > 8192) return cudaErrorInvalidValue;
+  if (attn_fwd_pair_applies(p)) return launch_attn_fwd_pair(p, s);
   if (D == 128 && p.blk == 128) return launch_mode<128, 128>(p, s);
   if (D == 128 && p.blk == 64) return launch_mode<128, 64>(p, s);
   if (D == 64 && p.blk == 128) return launch_mode<64, 128>(p, s);

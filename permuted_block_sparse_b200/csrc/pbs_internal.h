@@ -61,6 +61,10 @@ struct AttnParams {
   const float* gate_thr;
   int early_stop;         // S2O early stopping: lists in visiting order, cut by stop_tau
   int perm_nseg;          // 1: one permutation per KV head; else one per query segment
+  int cta_pair;           // run the CTA-pair kernel where it applies
+  // Failure-path test hook (0 in normal use): bound the role waits by this
+  // many polls and withhold the "Q landed" arrival, so the kernel times out.
+  uint32_t test_wait_limit;
   float stop_tau;
   float scale_log2;       // softmax scale * log2(e)
   float* lse;
@@ -68,5 +72,9 @@ struct AttnParams {
   int* err;
 };
 cudaError_t launch_attn_fwd(const AttnParams& p, cudaStream_t s);
+// The CTA-pair forward (four query heads per pair of CTAs); used by
+// launch_attn_fwd where it applies.
+bool attn_fwd_pair_applies(const AttnParams& p);
+cudaError_t launch_attn_fwd_pair(const AttnParams& p, cudaStream_t s);
 
 }  // namespace pbs

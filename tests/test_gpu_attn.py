@@ -127,13 +127,46 @@ def test_gated_attention_small():
     assert int(st[1]) == n_causal - kept
 
 
-def test_gated_attention_workload_sampled():
+@pytest.mark.parametrize("name", ["gate_b8_2k", "gate_b8_4k"])
+def test_gated_attention_short_n_workloads(name):
+    """The short-N gating workloads as the bench runs them (B = 8, every
+    earlier block listed, the stored offline thresholds).  With at most 32
+    causal tiles per row every threshold is -inf, so no tile may be gated:
+    the gated run must execute every causal tile, gate none, and give the
+    same bits as the run without thresholds; sampled query blocks match the
+    oracle (first, last, interior blocks of several heads and batches)."""
+    import os
+    w, Q, K, V = workload_inputs(name)
+    thr = np.load(os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", f"gate_thr_{name}.npy"))
+    assert np.all(np.isneginf(thr))
+    perm = np.broadcast_to(np.arange(w.N, dtype=np.int32), (w.B, w.Hkv, w.N)).copy()
+    counts, lists = oracle.dense_lists(w.B, w.Hq, w.nb, w.blk, w.seg)
+    O, L, st = _run(w, Q, K, V, perm, counts, lists, gate=thr.astype(np.float64), stats=True)
+    n_causal = w.B * w.Hq * w.nb * (w.nb + 1) // 2
+    assert int(st[0]) == n_causal and int(st[1]) == 0
+    O_plain, L_plain, _ = _run(w, Q, K, V, perm, counts, lists)
+    assert torch.equal(O, O_plain) and torch.equal(L, L_plain)
+    last = w.nb - 1
+    blocks = [(b, h, i) for b in (0, 5, 7) for h in (0, 17, 31) for i in (0, 3, last // 2, last)]
+    ref = oracle.attn_blocks(Q, K, V, perm, lists, w.blk, w.seg, blocks, gate_thr=thr.astype(np.float64))
+    O_np = O.float().cpu().numpy().astype(np.float64)
+    L_np = L.cpu().numpy()
+    for (b, h, i), (o_ref, l_ref) in ref.items():
+        sl = slice(i * w.blk, (i + 1) * w.blk)
+        assert_close(torch.from_numpy(O_np[b, h, sl]), o_ref, what=str((b, h, i)))
+        assert np.max(np.abs(L_np[b, h, sl] - l_ref)) <= LSE_MAX_ABS
+
+
+def test_gated_attention_sampled_calibrated():
+    """gate_b8_2k's inputs with thresholds calibrated to keep 5 tiles (so the
+    gate does fire at this length): sampled blocks against the oracle."""
     w, Q, K, V = workload_inputs("gate_b8_2k")
     perm = np.broadcast_to(np.arange(w.N, dtype=np.int32), (w.B, w.Hkv, w.N)).copy()
     counts, lists = oracle.dense_lists(w.B, w.Hq, w.nb, w.blk, w.seg)
     blocks = [(b, h, i) for b in (0, 7) for h in (0, 17, 31) for i in (0, 3, 8, 15)]
-    thr = oracle.calibrate_thresholds(Q, K, w.blk, w.gate_keep, blocks=blocks)
-    O, L, _ = _run(w, Q, K, V, perm, counts, lists, gate=thr)
+    thr = oracle.calibrate_thresholds(Q, K, w.blk, 5, blocks=blocks)
+    O, L, st = _run(w, Q, K, V, perm, counts, lists, gate=thr, stats=True)
+    assert int(st[1]) > 0
     ref = oracle.attn_blocks(Q, K, V, perm, lists, w.blk, w.seg, blocks, gate_thr=thr)
     O_np = O.float().cpu().numpy().astype(np.float64)
     for (b, h, i), (o_ref, _) in ref.items():
