@@ -16,9 +16,12 @@ from permuted_block_sparse_b200 import synth  # noqa: E402
 
 
 def test_reference_arm_prints_one_json_line():
+    import time
+    t0 = time.perf_counter()
     out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload",
-                          "single_head_1k", "--steps", "1", "--warmup", "0"], capture_output=True, text=True,
+                          "single_head_1k", "--steps", "2", "--warmup", "0"], capture_output=True, text=True,
                          timeout=600, cwd=ROOT)
+    wall = time.perf_counter() - t0
     assert out.returncode == 0, out.stderr[-2000:]
     lines = [ln for ln in out.stdout.splitlines() if ln.strip().startswith("{")]
     assert len(lines) == 1
@@ -28,6 +31,21 @@ def test_reference_arm_prints_one_json_line():
     assert d["config"] == bench.arm_config(synth.WORKLOADS["single_head_1k"])
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
+    # ms_per_step is the time a step actually ran, so the steps fit in the run's wall time;
+    # the 1K workload (16 query blocks) is small enough to run in full
+    assert 0 < d["ms_per_step"] * d["steps"] <= wall * 1e3
+    assert "the whole workload" in d["cpu_baseline"]["sample"]
+    assert d["est_full_run_s"] == pytest.approx(d["ms_per_step"] / 1e3, rel=0.5)
+
+
+def test_oracle_baseline_sample_states_its_fraction():
+    w = synth.WORKLOADS["gqa_8k_band"]
+    Q, K, V, _ = synth.make_inputs(w)
+    cpu = bench.oracle_baseline(w, Q, K, V, budget_s=2.0, n_blocks=4)
+    n_rows = w.B * w.Hq * w.nb
+    assert f"of {n_rows} query blocks" in cpu["sample"] and "divided by its sampled fraction" in cpu["sample"]
+    assert 0 < cpu["fraction_of_attention"] <= 4 / n_rows
+    assert cpu["est_full_run_s"] > cpu["sample_s"] > 0
 
 
 def test_algorithmic_bytes():
