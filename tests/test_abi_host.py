@@ -2,6 +2,7 @@
 include/pbs.h declares, and rejects bad arguments before touching a GPU."""
 import ctypes
 import os
+import subprocess
 import re
 
 import pytest
@@ -215,3 +216,67 @@ def test_sample_selector_host_checks(lib):
 def test_binding_rejects_unknown_selection_mode(lib):
     with pytest.raises(ValueError):
         pbs.select_capacity(1024, 128, 256, "bogus", 0.5)
+
+
+def _c_prototypes():
+    """name -> list of parameter type strings, from include/pbs.h."""
+    import re
+    text = open(os.path.join(ROOT, "include", "pbs.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    protos = {}
+    for m in re.finditer(r"(?:^|\n)\s*(?:const\s+)?\w+\s*\*?\s*(pbs_\w+)\s*\(([^;{]*?)\)\s*;", text, flags=re.S):
+        params = [" ".join(x.split()) for x in m.group(2).split(",")]
+        types = []
+        for prm in params:
+            if prm in ("", "void"):
+                continue
+            t = re.sub(r"\b\w+$", "", prm).strip()      # drop the parameter name
+            types.append(t.replace(" *", "*"))
+        protos[m.group(1)] = types
+    return protos
+
+
+def _ctype_of(c_type):
+    import ctypes
+    if "pbs_tensor*" in c_type:
+        return ctypes.POINTER(bd.PbsTensor)
+    if c_type.endswith("*"):
+        return ctypes.c_void_p
+    return {"int": ctypes.c_int, "int64_t": ctypes.c_int64, "double": ctypes.c_double, "float": ctypes.c_float,
+            "size_t": ctypes.c_size_t, "unsigned": ctypes.c_uint}[c_type]
+
+
+def test_binding_signatures_match_the_header(lib):
+    """Every ctypes declaration in the binding has the header's parameter
+    list (count and C types), so drift between the two fails here."""
+    protos = _c_prototypes()
+    assert set(bd.EXPORTS) <= set(protos)
+    checked = 0
+    for name, types in protos.items():
+        fn = getattr(lib, name)
+        if fn.argtypes is None:
+            continue
+        want = [_ctype_of(t) for t in types]
+        assert len(fn.argtypes) == len(want), name
+        for got, exp in zip(fn.argtypes, want):
+            assert got == exp or (exp is __import__("ctypes").c_void_p and got.__name__.startswith("LP_")), (name, got, exp)
+        checked += 1
+    assert checked >= 12
+
+
+def test_c_caller_compiles_against_the_header_and_runs(tmp_path):
+    """tests/c_abi/abi_check.c includes include/pbs.h, is compiled as C and
+    linked against libpbs.so; every call is rejected on the host with its
+    documented status."""
+    import shutil
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    exe = str(tmp_path / "abi_check")
+    libdir = os.path.dirname(bd.LIB_PATH)
+    build = subprocess.run([cc, "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"),
+                            os.path.join(ROOT, "tests", "c_abi", "abi_check.c"), "-o", exe, "-L", libdir, "-l:libpbs.so",
+                            "-Wl,-rpath," + libdir], capture_output=True, text=True)
+    assert build.returncode == 0, build.stderr
+    run = subprocess.run([exe], capture_output=True, text=True, timeout=120)
+    assert run.returncode == 0 and "abi ok" in run.stdout, run.stdout + run.stderr

@@ -56,6 +56,29 @@ def test_noalloc_matches_workspace_entry_point_twice():
         assert torch.equal(out, ref), (seed, B, Hq, Hkv, N)
 
 
+def test_noalloc_at_exactly_its_scratch_size():
+    """B * Hkv * D = 512 * 128 = 65536 floats fills the static scratch
+    exactly: still served, and equal to the workspace entry point."""
+    lib = pbs.load()
+    fn = _noalloc(lib)
+    stream = torch.cuda.current_stream().cuda_stream
+    Qd, Kd = _case(3, 1, 512, 512, 256, 128, 128, 256, 0)
+    ref = pbs.pbs_permute(Qd, Kd, 128, 256, 0)
+    out = torch.full_like(ref, -1)
+    q, k = bd.describe(Qd), bd.describe(Kd)
+    rc = fn(ctypes.byref(q), ctypes.byref(k), 128, 256, 0, out.data_ptr(), stream)
+    assert rc == 0, lib.pbs_get_last_error()
+    pbs.pbs_check_device()
+    assert torch.equal(out, ref)
+    # one KV head more (65536 + 128 floats) is refused before any launch
+    Qd, Kd = _case(3, 1, 513, 513, 128, 128, 128, 128, 0)
+    q, k = bd.describe(Qd), bd.describe(Kd)
+    out = torch.full((1, 513, 128), -1, dtype=torch.int32, device="cuda")
+    rc = fn(ctypes.byref(q), ctypes.byref(k), 128, 128, 0, out.data_ptr(), stream)
+    assert rc == -3
+    assert int(out.min()) == -1 and int(out.max()) == -1
+
+
 def test_noalloc_rejects_inputs_beyond_its_scratch():
     lib = pbs.load()
     fn = _noalloc(lib)
