@@ -81,7 +81,7 @@ typedef enum pbs_status {
 } pbs_status;
 
 enum { PBS_OP_PERMUTE = 0, PBS_OP_SELECT = 1, PBS_OP_ATTN = 2, PBS_OP_PERMUTE_SEGMENTED = 3,
-       PBS_OP_SELECT_SEGMENTED = 4, PBS_OP_SELECT_SAMPLE = 5 };
+       PBS_OP_SELECT_SEGMENTED = 4, PBS_OP_SELECT_SAMPLE = 5, PBS_OP_PERMUTE_QUERIES = 6 };
 enum { PBS_SELECT_TOPK = 0, PBS_SELECT_TAU = 1, PBS_SELECT_SAMPLE = 2 };
 /* OR-ed into pbs_select's mode: write lists in visiting order, and/or read
  * one permutation per query segment (see there). */
@@ -144,6 +144,23 @@ int pbs_permute_noalloc(const pbs_tensor* Q, const pbs_tensor* K, int blk, int s
  * are multiples of 1/8 (any bf16 input sorts by its fp64-rounded scores). */
 int pbs_permute_segmented(const pbs_tensor* Q, const pbs_tensor* K, int blk, int seg, int n_sink,
                           int32_t* perm, void* ws, size_t ws_bytes, void* stream);
+
+/* pbs_permute_queries: S2O's query permutation ("S2O ...", Technical
+ * Summary, 1. Online Permutation via Index-Driven Loading, Query
+ * Permutation: queries are reordered by their score against a guide vector
+ * shared by the head).  qperm[b, hq, p] = original query position at
+ * permuted position p:
+ *   1. guide vector g[b, hkv] = sum of every key row of KV head hkv (fp64);
+ *   2. score of query n of head hq: Q[b, hq, n] . g[b, hq / G] (fp64);
+ *   3. within each segment [t*seg, (t+1)*seg) the queries of (b, hq) are
+ *      ordered by descending score, equal scores by ascending position;
+ *      segment order is kept, so qperm maps each segment onto itself.
+ * qperm: device int32 [B, Hq, N].  blk only takes part in the shape checks.
+ * ws: pbs_workspace_size(PBS_OP_PERMUTE_QUERIES, ...) bytes (partial and
+ * final guide vectors).  Select with pbs_select_qperm and attend with
+ * pbs_attn_fwd_qperm to use it.                                            */
+int pbs_permute_queries(const pbs_tensor* Q, const pbs_tensor* K, int blk, int seg, int32_t* qperm,
+                        void* ws, size_t ws_bytes, void* stream);
 
 /* Upper bound on the list length pbs_select can produce for these settings
  * (host-only arithmetic).  Pass at least this as `cap`.  For
@@ -246,6 +263,30 @@ int pbs_attn_fwd_early_stop(const pbs_tensor* Q, const pbs_tensor* K, const pbs_
                             const int32_t* perm, const int32_t* counts, const int32_t* idx,
                             int cap, int blk, int seg, float stop_tau, float softmax_scale,
                             pbs_tensor* O, float* lse, long long* stats, void* stream);
+
+/* pbs_select_qperm: pbs_select over permuted query blocks.  Query block i
+ * is made of the queries at positions qperm[b, hq, i*blk .. i*blk+blk-1]
+ * (all in block i's segment; an entry outside it sets the device error word
+ * and is left out of the pooled sum); its pooled query is their sum, and
+ * candidates, budget and rule are those of pbs_select for block i.  mode is
+ * PBS_SELECT_TOPK or PBS_SELECT_TAU, with no flag bits; no band.  Other
+ * arguments as for pbs_select; `cap` as pbs_select_capacity gives with
+ * band = 0.                                                                */
+int pbs_select_qperm(const pbs_tensor* Q, const pbs_tensor* K, const int32_t* perm, const int32_t* qperm,
+                     int blk, int seg, int mode, double density_or_tau, int n_sink, int32_t* counts,
+                     int32_t* idx, int cap, void* ws, size_t ws_bytes, void* stream);
+
+/* pbs_attn_fwd_qperm: pbs_attn_fwd over permuted query blocks ("S2O ...",
+ * Technical Summary, 1. Online Permutation via Index-Driven Loading, Query
+ * Permutation and Coordinate-Planned Loading).  Row r of query block i is
+ * the query at q = qperm[b, hq, i*blk + r]; it attends the keys of its own
+ * segment up to q (Pass 1: natural blocks with an element-wise causal mask)
+ * and the keys of block i's listed permuted blocks (Pass 2).  O[b, hq, q]
+ * and lse[b, hq, q] are written at the query's original position.  No
+ * gating, no early stopping.  Other arguments as for pbs_attn_fwd.        */
+int pbs_attn_fwd_qperm(const pbs_tensor* Q, const pbs_tensor* K, const pbs_tensor* V, const int32_t* perm,
+                       const int32_t* qperm, const int32_t* counts, const int32_t* idx, int cap, int blk, int seg,
+                       float softmax_scale, pbs_tensor* O, float* lse, long long* stats, void* stream);
 
 /* pbs_attn_fwd_ex: pbs_attn_fwd and pbs_attn_fwd_early_stop in one call.
  *   flags: PBS_ATTN_EARLY_STOP -- lists in visiting order, stop_tau as for

@@ -20,6 +20,7 @@ LIB_PATH = os.path.join(_HERE, "libpbs.so")
 
 PBS_OP_PERMUTE, PBS_OP_SELECT, PBS_OP_ATTN, PBS_OP_PERMUTE_SEGMENTED, PBS_OP_SELECT_SEGMENTED = 0, 1, 2, 3, 4
 PBS_OP_SELECT_SAMPLE = 5
+PBS_OP_PERMUTE_QUERIES = 6
 PBS_SELECT_TOPK, PBS_SELECT_TAU, PBS_SELECT_SAMPLE = 0, 1, 2
 _MODES = {"topk": PBS_SELECT_TOPK, "tau": PBS_SELECT_TAU, "sample": PBS_SELECT_SAMPLE}
 PBS_SELECT_SCORE_ORDER, PBS_SELECT_PERM_PER_SEGMENT = 0x10, 0x20
@@ -28,7 +29,8 @@ STATUS = {0: "PBS_OK", -1: "PBS_ERR_INVALID_ARG", -2: "PBS_ERR_UNSUPPORTED", -3:
           -4: "PBS_ERR_CUDA", -5: "PBS_ERR_TIMEOUT", -6: "PBS_ERR_DEVICE_CHECK"}
 EXPORTS = ("pbs_workspace_size", "pbs_permute", "pbs_permute_segmented", "pbs_select_capacity", "pbs_select",
            "pbs_attn_fwd", "pbs_attn_fwd_early_stop", "pbs_attn_fwd_ex", "pbs_check_device",
-           "pbs_get_last_error", "pbs_version", "pbs_permute_noalloc", "pbs_test_inject_timeout")
+           "pbs_get_last_error", "pbs_version", "pbs_permute_noalloc", "pbs_test_inject_timeout",
+           "pbs_permute_queries", "pbs_select_qperm", "pbs_attn_fwd_qperm")
 
 
 class PbsError(RuntimeError):
@@ -76,6 +78,12 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.pbs_attn_fwd_early_stop.restype = i32
     lib.pbs_check_device.argtypes = [vp]
     lib.pbs_check_device.restype = i32
+    lib.pbs_permute_queries.argtypes = [P, P, i32, i32, vp, vp, sz, vp]
+    lib.pbs_permute_queries.restype = i32
+    lib.pbs_select_qperm.argtypes = [P, P, vp, vp, i32, i32, i32, dbl, i32, vp, vp, i32, vp, sz, vp]
+    lib.pbs_select_qperm.restype = i32
+    lib.pbs_attn_fwd_qperm.argtypes = [P, P, P, vp, vp, vp, vp, i32, i32, i32, ctypes.c_float, P, vp, vp, vp]
+    lib.pbs_attn_fwd_qperm.restype = i32
     lib.pbs_test_inject_timeout.argtypes = [ctypes.c_uint]
     lib.pbs_test_inject_timeout.restype = None
     lib.pbs_get_last_error.argtypes = []
@@ -249,6 +257,77 @@ def pbs_attn_fwd(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, perm: torch.
                             counts.data_ptr(), idx.data_ptr(), idx.shape[-1], blk, seg, _ptr(gate_thr),
                             float(softmax_scale), ctypes.byref(o), _ptr(lse), _ptr(stats), None, 0,
                             _stream(stream)))
+    return out, lse
+
+
+def pbs_permute_queries(Q: torch.Tensor, K: torch.Tensor, blk: int, seg: int,
+                        qperm: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
+                        stream=None) -> torch.Tensor:
+    """qperm [B, Hq, N] int32: S2O's query permutation (per segment, queries
+    by descending score against the KV head's guide vector)."""
+    lib = load()
+    q, k = describe(Q), describe(K)
+    B, Hq, N, _ = Q.shape
+    if qperm is None:
+        qperm = torch.empty((B, Hq, N), dtype=torch.int32, device=Q.device)
+    if ws is None:
+        ws = _workspace(lib.pbs_workspace_size(PBS_OP_PERMUTE_QUERIES, ctypes.byref(q), ctypes.byref(k), blk, seg),
+                        Q.device)
+    wp, wn = _aligned(ws)
+    _check(lib.pbs_permute_queries(ctypes.byref(q), ctypes.byref(k), blk, seg, qperm.data_ptr(), wp, wn,
+                                   _stream(stream)))
+    return qperm
+
+
+def pbs_select_qperm(Q: torch.Tensor, K: torch.Tensor, perm: torch.Tensor, qperm: torch.Tensor, blk: int,
+                     seg: int, mode: str = "topk", density_or_tau: float = 1.0, n_sink: int = 0,
+                     cap: Optional[int] = None, counts: Optional[torch.Tensor] = None,
+                     idx: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
+                     stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """(counts, idx) block lists of the permuted query blocks (ascending)."""
+    lib = load()
+    q, k = describe(Q), describe(K)
+    B, Hq, N, _ = Q.shape
+    nb = N // blk
+    if mode not in ("topk", "tau"):
+        raise ValueError(f"permuted queries take mode 'topk' or 'tau', not {mode!r}")
+    if cap is None:
+        cap = max(1, select_capacity(N, blk, seg, mode, density_or_tau, 0, n_sink))
+    if counts is None:
+        counts = torch.empty((B, Hq, nb), dtype=torch.int32, device=Q.device)
+    if idx is None:
+        idx = torch.empty((B, Hq, nb, cap), dtype=torch.int32, device=Q.device)
+    if ws is None:
+        ws = _workspace(lib.pbs_workspace_size(PBS_OP_SELECT, ctypes.byref(q), ctypes.byref(k), blk, seg), Q.device)
+    wp, wn = _aligned(ws)
+    _check(lib.pbs_select_qperm(ctypes.byref(q), ctypes.byref(k), perm.data_ptr(), qperm.data_ptr(), blk, seg,
+                                _MODES[mode], float(density_or_tau), n_sink, counts.data_ptr(), idx.data_ptr(), cap,
+                                wp, wn, _stream(stream)))
+    return counts, idx
+
+
+def pbs_attn_fwd_qperm(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, perm: torch.Tensor,
+                       qperm: torch.Tensor, counts: torch.Tensor, idx: torch.Tensor, blk: int, seg: int,
+                       softmax_scale: Optional[float] = None, out: Optional[torch.Tensor] = None,
+                       lse: Optional[torch.Tensor] = None, want_lse: bool = True,
+                       stats: Optional[torch.Tensor] = None,
+                       stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """(O, LSE) at the queries' original positions, for lists indexed by
+    permuted query block."""
+    lib = load()
+    B, Hq, N, D = Q.shape
+    if out is None:
+        out = torch.empty_like(Q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq, N), dtype=torch.float32, device=Q.device)
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(D)
+    if stats is not None and stats.dtype != torch.int64:
+        raise TypeError("stats must be int64")
+    q, k, v, o = describe(Q), describe(K), describe(V), describe(out)
+    _check(lib.pbs_attn_fwd_qperm(ctypes.byref(q), ctypes.byref(k), ctypes.byref(v), perm.data_ptr(),
+                                  qperm.data_ptr(), counts.data_ptr(), idx.data_ptr(), idx.shape[-1], blk, seg,
+                                  float(softmax_scale), ctypes.byref(o), _ptr(lse), _ptr(stats), _stream(stream)))
     return out, lse
 
 

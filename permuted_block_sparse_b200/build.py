@@ -14,7 +14,8 @@ CSRC = os.path.join(HERE, "csrc")
 BUILD_DIR = os.path.join(ROOT, "_build")
 LIB = os.path.join(HERE, "libpbs.so")
 SOURCES = ["api.cu", "permute.cu", "permute_seg.cu", "select.cu", "select_sample.cu", "attn_fwd.cu",
-           "attn_fwd_pair.cu", "permute_noalloc.cu"]
+           "attn_fwd_pair.cu", "permute_queries.cu",
+           "permute_noalloc.cu"]
 HEADERS = ["pbs_common.cuh", "pbs_internal.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O2", "--expt-relaxed-constexpr"]

@@ -163,7 +163,7 @@ int attn_common(const pbs_tensor* Qt, const pbs_tensor* Kt, const pbs_tensor* Vt
                 const int32_t* perm, const int32_t* counts, const int32_t* idx, int cap, int blk,
                 int seg, const float* gate_thr, int early_stop, float stop_tau, int per_segment,
                 float softmax_scale, pbs_tensor* Ot, float* lse, long long* stats, void* stream,
-                int cta_pair = 0) {
+                int cta_pair = 0, const int32_t* qperm = nullptr) {
   pbs::TensorDesc Q, K, V, O;
   int rc;
   if ((rc = check_tensor(Qt, "Q", &Q)) || (rc = check_tensor(Kt, "K", &K)) ||
@@ -188,6 +188,7 @@ int attn_common(const pbs_tensor* Qt, const pbs_tensor* Kt, const pbs_tensor* Vt
   p.perm = perm;
   p.counts = counts;
   p.idx = idx;
+  p.qperm = qperm;
   p.cap = cap;
   p.blk = blk;
   p.seg = seg;
@@ -207,6 +208,12 @@ int attn_common(const pbs_tensor* Qt, const pbs_tensor* Kt, const pbs_tensor* Vt
   if (e != cudaSuccess) return cuda_fail(e, "attn_fwd launch");
   return ok();
 }
+}  // namespace
+
+namespace {
+int select_impl(const pbs_tensor* Qt, const pbs_tensor* Kt, const int32_t* perm, const int32_t* qperm, int blk,
+                int seg, int mode, double density_or_tau, int band, int n_sink, int32_t* counts, int32_t* idx,
+                int cap, void* ws, size_t ws_bytes, void* stream);
 }  // namespace
 
 extern "C" {
@@ -231,6 +238,8 @@ size_t pbs_workspace_size(int op, const pbs_tensor* Qt, const pbs_tensor* Kt, in
       return nseg > 0 ? select_ws(Q, K, blk, nseg).total : 0;
     case PBS_OP_SELECT_SAMPLE:
       return sample_ws(Q).total;
+    case PBS_OP_PERMUTE_QUERIES:
+      return align256(pbs::permute_queries_ws_bytes(K));
     default:
       return 0;
   }
@@ -247,6 +256,20 @@ int pbs_permute_segmented(const pbs_tensor* Qt, const pbs_tensor* Kt, int blk, i
   cudaError_t e = pbs::launch_permute_segmented(Q, K, seg, n_sink, static_cast<double*>(ws), perm,
                                                 static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "permute_segmented launch");
+  return ok();
+}
+
+int pbs_permute_queries(const pbs_tensor* Qt, const pbs_tensor* Kt, int blk, int seg, int32_t* qperm, void* ws,
+                        size_t ws_bytes, void* stream) {
+  pbs::TensorDesc Q, K;
+  int rc;
+  if ((rc = pbs::api_validate_permute(Qt, Kt, blk, seg, 0, qperm, &Q, &K))) return rc;
+  const int64_t nseg = (Q.N + seg - 1) / seg;
+  if (nseg > 65535) return fail(PBS_ERR_UNSUPPORTED, "too many segments");
+  if ((rc = check_ws(ws, ws_bytes, align256(pbs::permute_queries_ws_bytes(K))))) return rc;
+  cudaError_t e = pbs::launch_permute_queries(Q, K, seg, static_cast<double*>(ws), qperm,
+                                              static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "permute_queries launch");
   return ok();
 }
 
@@ -301,6 +324,26 @@ int pbs_select_capacity(int64_t N, int blk, int seg, int mode, double density_or
 int pbs_select(const pbs_tensor* Qt, const pbs_tensor* Kt, const int32_t* perm, int blk, int seg,
                int mode, double density_or_tau, int band, int n_sink, int32_t* counts,
                int32_t* idx, int cap, void* ws, size_t ws_bytes, void* stream) {
+  return select_impl(Qt, Kt, perm, nullptr, blk, seg, mode, density_or_tau, band, n_sink, counts, idx, cap, ws,
+                     ws_bytes, stream);
+}
+
+int pbs_select_qperm(const pbs_tensor* Qt, const pbs_tensor* Kt, const int32_t* perm, const int32_t* qperm,
+                     int blk, int seg, int mode, double density_or_tau, int n_sink, int32_t* counts,
+                     int32_t* idx, int cap, void* ws, size_t ws_bytes, void* stream) {
+  if (!qperm) return fail(PBS_ERR_INVALID_ARG, "qperm is null");
+  if (mode != PBS_SELECT_TOPK && mode != PBS_SELECT_TAU)
+    return fail(PBS_ERR_UNSUPPORTED, "permuted queries take PBS_SELECT_TOPK or PBS_SELECT_TAU without flags");
+  return select_impl(Qt, Kt, perm, qperm, blk, seg, mode, density_or_tau, 0, n_sink, counts, idx, cap, ws,
+                     ws_bytes, stream);
+}
+
+}  // extern "C"
+
+namespace {
+int select_impl(const pbs_tensor* Qt, const pbs_tensor* Kt, const int32_t* perm, const int32_t* qperm, int blk,
+                int seg, int mode, double density_or_tau, int band, int n_sink, int32_t* counts, int32_t* idx,
+                int cap, void* ws, size_t ws_bytes, void* stream) {
   pbs::TensorDesc Q, K;
   int rc;
   if ((rc = check_tensor(Qt, "Q", &Q)) || (rc = check_tensor(Kt, "K", &K))) return rc;
@@ -369,7 +412,7 @@ int pbs_select(const pbs_tensor* Qt, const pbs_tensor* Kt, const int32_t* perm, 
     if (e != cudaSuccess) return cuda_fail(e, "select_sample launch");
     return ok();
   }
-  cudaError_t e = pbs::launch_pool_query_blocks(Q, blk, qbar, s);
+  cudaError_t e = pbs::launch_pool_query_blocks(Q, blk, qperm, seg, err, qbar, s);
   if (e != cudaSuccess) return cuda_fail(e, "pool_query_blocks launch");
   e = pbs::launch_pool_key_blocks(K, perm, static_cast<int>(perm_nseg), blk, seg, mode == PBS_SELECT_TAU, kperm,
                                   knat, inv, err, s);
@@ -396,6 +439,9 @@ int pbs_select(const pbs_tensor* Qt, const pbs_tensor* Kt, const int32_t* perm, 
   return ok();
 }
 
+}  // namespace
+
+extern "C" {
 
 int pbs_attn_fwd(const pbs_tensor* Qt, const pbs_tensor* Kt, const pbs_tensor* Vt,
                  const int32_t* perm, const int32_t* counts, const int32_t* idx, int cap, int blk,
@@ -435,6 +481,14 @@ int pbs_attn_fwd_ex(const pbs_tensor* Qt, const pbs_tensor* Kt, const pbs_tensor
 }
 
 void pbs_test_inject_timeout(unsigned limit_polls) { g_test_wait_limit.store(limit_polls); }
+
+int pbs_attn_fwd_qperm(const pbs_tensor* Qt, const pbs_tensor* Kt, const pbs_tensor* Vt, const int32_t* perm,
+                       const int32_t* qperm, const int32_t* counts, const int32_t* idx, int cap, int blk, int seg,
+                       float softmax_scale, pbs_tensor* Ot, float* lse, long long* stats, void* stream) {
+  if (!qperm) return fail(PBS_ERR_INVALID_ARG, "qperm is null");
+  return attn_common(Qt, Kt, Vt, perm, counts, idx, cap, blk, seg, nullptr, 0, 0.0f, 0, softmax_scale, Ot, lse,
+                     stats, stream, 0, qperm);
+}
 
 int pbs_check_device(void* stream) {
   cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));

@@ -79,6 +79,7 @@ struct Shared {
   uint32_t tmem_base;
   int abort;
   int n_union;
+  int jtop;                // last natural block of Pass 1
   int skip[2][2];
   float red[2][4];
   int vote[2][4];          // early stopping: per-warp "every row's gain is small"
@@ -86,12 +87,17 @@ struct Shared {
   int n_list[2];           // early stopping: listed tiles per head slot
 };
 
+// QP: S2O query permutation -- row r of query block i is the query at
+// qperm[i*BLK + r] (both heads' rows from their own qperm rows), Pass 1 runs
+// the natural blocks of the own segment up to the last of those queries
+// with an element-wise causal mask, and O / LSE go back to the queries'
+// positions.
 // ES: S2O early stopping -- each head's listed blocks are visited in the
 // order given and its Pass 2 is cut once a tile's gain is small.  The two
 // heads' lists are interleaved (one tile of each in turn, every tile for one
 // head); tiles of a head that has stopped are not loaded and only passed
 // through the rings.
-template <int D, int BLK, bool ES>
+template <int D, int BLK, bool ES, bool QP>
 __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
   using C = Cfg<D, BLK>;
   extern __shared__ unsigned char smem_raw[];
@@ -101,6 +107,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
   __shared__ Shared sh;
   __shared__ uint32_t bm[2][256];          // candidate bitmaps (ncand <= 8192)
   __shared__ int32_t rowbuf[kStages][BLK];
+  __shared__ int32_t qpos[2][QP ? BLK : 1];  // QP: the query position of each row
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int Hq = p.G * static_cast<int>(p.K.H);
@@ -120,7 +127,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
   const int spb = p.seg / BLK;
   const int s = i / spb;
   const int ncand = s * spb;
-  const int n_diag = i - s * spb + 1;
   const int64_t q0 = static_cast<int64_t>(i) * BLK;
   const int64_t N = p.Q.N;
 
@@ -223,6 +229,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
     }
     if (lane == 0) {
       sh.n_union = total;
+      sh.jtop = i;
       sh.abort = 0;
       sh.limit[0] = 0x7fffffff;
       sh.limit[1] = 0x7fffffff;
@@ -241,11 +248,36 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
       mbar_init(&sh.bar_fin, 1);
       fence_mbar_init();
     }
+    if (QP) {
+      // Rows' query positions (each must lie in the block's segment; an
+      // entry outside it sets the error word and is replaced by the
+      // segment's first position) and the last natural block they reach.
+      const int64_t seg_lo = static_cast<int64_t>(s) * p.seg, seg_hi = min(seg_lo + p.seg, N);
+      int64_t mx = seg_lo;
+      for (int h = 0; h < (has1 ? 2 : 1); ++h) {
+        const int32_t* qrow = p.qperm + (static_cast<int64_t>(b) * Hq + h0 + h) * N + q0;
+        for (int r = lane; r < BLK; r += 32) {
+          int64_t x = qrow[r];
+          if (x < seg_lo || x >= seg_hi) {
+            set_error(p.err, kErrDeviceCheck);
+            x = seg_lo;
+          }
+          qpos[h][r] = static_cast<int32_t>(x);
+          mx = max(mx, x);
+        }
+      }
+      for (int off = 16; off > 0; off >>= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+      if (lane == 0) sh.jtop = static_cast<int>(mx / BLK);
+    }
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sh.tmem_base;
+  // Pass 1 runs natural blocks jtop, jtop - 1, ..., down to the segment's
+  // first; jtop is i itself unless queries are permuted.
+  const int jtop = QP ? sh.jtop : i;
+  const int n_diag = jtop - s * spb + 1;
   const int T = n_diag + sh.n_union;
   // Poll limit of the role waits (the drain before tensor memory is freed
   // keeps the full limit).
@@ -301,7 +333,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
         const int r = id / CH, c = id % CH;
         const bool valid = r < BLK;
         cp_async16_zfill(dst + (c / 8) * (kM * 128) + sw128_offset(r, c % 8),
-                         valid ? qb + (q0 + r) * p.Q.sN + c * 8 : qb, valid);
+                         valid ? qb + (QP ? static_cast<int64_t>(qpos[h][r]) : q0 + r) * p.Q.sN + c * 8 : qb,
+                         valid);
       }
     }
     // (the failure-path test hook withholds this arrival, so the MMA role's
@@ -347,7 +380,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
         const bool ok = t < kStages || wait_slot(&sh.bar_kempty[st], ((t >> 1) - 1) & 1, t);
         if (named_sync_or(1, kProducerThreads, !ok)) break;   // all producer threads leave together
         const bool nat = t < n_diag;
-        const int id0 = nat ? i - t : static_cast<int>(sched[t - n_diag] & 0x3FFFFFFFu);
+        const int id0 = nat ? jtop - t : static_cast<int>(sched[t - n_diag] & 0x3FFFFFFFu);
         // a permuted block lies inside one segment (seg is a multiple of BLK)
         const int64_t lo = static_cast<int64_t>((id0 * BLK) / p.seg) * p.seg;
 #pragma unroll
@@ -571,6 +604,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
     const uint32_t tS = tmem + h * 128 + lane_off;
     const uint32_t tO = tmem + 256 + h * 128 + lane_off;
     const int hq = h0 + h;
+    // this row's query position (rows r >= BLK, present when BLK < 128, are never written)
+    const int64_t qp = QP ? static_cast<int64_t>(qpos[h][r < BLK ? r : 0]) : q0 + r;
     const bool active = h == 0 || has1;
     const float thr =
         (active && p.gate_thr) ? p.gate_thr[(static_cast<int64_t>(b) * Hq + hq) * p.nb + i] : -INFINITY;
@@ -629,7 +664,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
       // chunk's max exceeds m by more than 2^8, m moves up and the P columns
       // already written for this tile are rescaled in place (rare after the
       // first tile).  So P stays below 2^8 and S is read once here.
-      const bool causal = t == 0;
+      // Causal mask: columns above `vis` are not visible to this row.  In
+      // natural order only the diagonal tile (t == 0) needs it; with permuted
+      // queries every Pass-1 tile does, against the row's own position.
+      int vis = BLK;
+      if (QP) {
+        if (t < n_diag) vis = static_cast<int>(qp - static_cast<int64_t>(jtop - t) * BLK);
+      } else if (t == 0) {
+        vis = r;
+      }
+      const bool causal = QP ? __any_sync(0xffffffffu, vis < BLK - 1) : t == 0;
       float psum = 0.f, m_t = m_run;
 #pragma unroll 1
       for (int c = 0; c < BLK / 64; ++c) {
@@ -639,7 +683,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
         if (causal) {
 #pragma unroll
           for (int e = 0; e < 64; ++e) {
-            const float v = c * 64 + e > r ? -INFINITY : __uint_as_float(x[e]);
+            const float v = c * 64 + e > vis ? -INFINITY : __uint_as_float(x[e]);
             x[e] = __float_as_uint(v);
             cmax = fmaxf(cmax, v);
           }
@@ -659,7 +703,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
         const bool up = cm > (m_t == -INFINITY ? -INFINITY : m_t + kRescaleSlack);
         if (__any_sync(0xffffffffu, up)) {
           const float m_new = up ? cm : m_t;
-          const float beta = ex2(m_t - m_new);       // 0 when m_t was -inf
+          // 0 when m_t was -inf; 1 for a row that still has no visible key
+          const float beta = m_new == -INFINITY ? 1.0f : ex2(m_t - m_new);
           if (c > 0 && __any_sync(0xffffffffu, beta != 1.0f)) {
             tmem_st_wait();                           // earlier P stores of this thread landed
             for (int q = 0; q < 2 * c; ++q) {         // rescale this tile's P so far
@@ -711,7 +756,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
         tmem_st32(tS + c * 32, u);
       }
       const float m_new = m_t;
-      const float alpha = ex2(m_run - m_new);
+      // (a row that has seen no visible key yet keeps m = -inf and l = 0)
+      const float alpha = m_new == -INFINITY ? 1.0f : ex2(m_run - m_new);
       if (o_init && __any_sync(0xffffffffu, alpha != 1.0f)) {
         // PV of this head's previous tile has completed: the S-ready barrier
         // tracks every MMA issued before this tile's QK^T.
@@ -762,7 +808,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
     if (active && ok && o_init) {
       const float inv_l = 1.0f / l_run;
       __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(const_cast<void*>(p.O.ptr)) + b * p.O.sB +
-                          hq * p.O.sH + (q0 + r) * p.O.sN;
+                          hq * p.O.sH + qp * p.O.sN;
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
         uint32_t u[32];
@@ -780,7 +826,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
         }
       }
       if (p.lse && r < BLK)
-        p.lse[(static_cast<int64_t>(b) * Hq + hq) * N + q0 + r] = (m_run + log2f(l_run)) * 0.69314718055994531f;
+        p.lse[(static_cast<int64_t>(b) * Hq + hq) * N + qp] = (m_run + log2f(l_run)) * 0.69314718055994531f;
     }
     if (active && r == 0 && p.stats) {
       atomicAdd(reinterpret_cast<unsigned long long*>(p.stats), static_cast<unsigned long long>(n_qk));
@@ -795,7 +841,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
   }
 }
 
-template <int D, int BLK, bool ES>
+template <int D, int BLK, bool ES, bool QP>
 cudaError_t launch_typed(const AttnParams& p, cudaStream_t s) {
   using C = Cfg<D, BLK>;
   // schedule: at most min(candidates, 2 * cap) permuted tiles per item
@@ -805,19 +851,20 @@ cudaError_t launch_typed(const AttnParams& p, cudaStream_t s) {
   int smem = 1024 + C::kEnd + 4 * max_union;
   smem = smem < C::kMinSmem ? C::kMinSmem : smem;
   if (smem + 4096 > 227 * 1024) return cudaErrorInvalidValue;   // + static shared memory
-  cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D, BLK, ES>,
+  cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D, BLK, ES, QP>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const int npair = (p.G + 1) / 2;
   const int64_t items = static_cast<int64_t>(p.nb) * p.Q.B * p.K.H * npair;
   if (items >= (1ll << 31)) return cudaErrorInvalidValue;
-  attn_fwd_kernel<D, BLK, ES><<<static_cast<unsigned>(items), kThreads, smem, s>>>(p);
+  attn_fwd_kernel<D, BLK, ES, QP><<<static_cast<unsigned>(items), kThreads, smem, s>>>(p);
   return cudaGetLastError();
 }
 
 template <int D, int BLK>
 cudaError_t launch_mode(const AttnParams& p, cudaStream_t s) {
-  return p.early_stop ? launch_typed<D, BLK, true>(p, s) : launch_typed<D, BLK, false>(p, s);
+  if (p.qperm) return p.early_stop ? cudaErrorInvalidValue : launch_typed<D, BLK, false, true>(p, s);
+  return p.early_stop ? launch_typed<D, BLK, true, false>(p, s) : launch_typed<D, BLK, false, false>(p, s);
 }
 
 }  // namespace

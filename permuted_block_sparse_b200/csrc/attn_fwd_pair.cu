@@ -649,7 +649,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_pair_kernel(AttnParams p
 
 // Whether the CTA-pair kernel serves these parameters.
 bool attn_fwd_pair_applies(const AttnParams& p) {
-  if (!p.cta_pair || p.Q.D != kD || p.blk != kBlk || p.early_stop || p.gate_thr) return false;
+  if (!p.cta_pair || p.Q.D != kD || p.blk != kBlk || p.early_stop || p.gate_thr || p.qperm) return false;
   if (p.G % 4 != 0) return false;
   const int max_union = std::min(p.nb, 4 * p.cap);
   const int smem = 1024 + kEnd + 4 * max_union;

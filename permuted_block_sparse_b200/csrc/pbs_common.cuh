@@ -35,6 +35,38 @@ __device__ __forceinline__ uint32_t ordered_u32(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// Order-preserving map of a double onto unsigned 64-bit integers.
+__device__ __forceinline__ uint64_t ordered_u64(double x) {
+  const uint64_t u = static_cast<uint64_t>(__double_as_longlong(x));
+  return (u & 0x8000000000000000ull) ? ~u : (u | 0x8000000000000000ull);
+}
+
+// Bitonic sort by the whole CTA of n2 (a power of two) (key, idx) pairs in
+// shared memory, ascending in key and then idx: distinct idx make it a
+// total order, so equal keys keep ascending idx.
+__device__ __forceinline__ void cta_bitonic_sort(uint64_t* key, uint32_t* idx, int n2) {
+  for (int k = 2; k <= n2; k <<= 1) {
+    for (int jj = k >> 1; jj > 0; jj >>= 1) {
+      for (int i = threadIdx.x; i < n2; i += blockDim.x) {
+        const int ixj = i ^ jj;
+        if (ixj > i) {
+          const uint64_t a = key[i], c = key[ixj];
+          const uint32_t ia = idx[i], ic = idx[ixj];
+          const bool greater = a > c || (a == c && ia > ic);
+          const bool up = (i & k) == 0;
+          if (greater == up) {
+            key[i] = c;
+            key[ixj] = a;
+            idx[i] = ic;
+            idx[ixj] = ia;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+}
+
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)

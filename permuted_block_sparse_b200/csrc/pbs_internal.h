@@ -21,7 +21,12 @@ cudaError_t launch_score_sort(const TensorDesc& K, int seg, int n_sink, const fl
                               int32_t* perm, int* err, cudaStream_t s);
 
 // pbs_select launchers ----------------------------------------------------
-cudaError_t launch_pool_query_blocks(const TensorDesc& Q, int blk, float* qbar, cudaStream_t s);
+cudaError_t launch_pool_query_blocks(const TensorDesc& Q, int blk, const int32_t* qperm, int seg, int* err,
+                                     float* qbar, cudaStream_t s);
+// pbs_permute_queries: guide vectors and the per-segment query sort.
+size_t permute_queries_ws_bytes(const TensorDesc& K);
+cudaError_t launch_permute_queries(const TensorDesc& Q, const TensorDesc& K, int seg, double* ws, int32_t* qperm,
+                                   cudaStream_t s);
 cudaError_t launch_pool_key_blocks(const TensorDesc& K, const int32_t* perm, int perm_nseg, int blk,
                                    int seg, bool natural, float* kbar_perm, float* kbar_nat,
                                    int32_t* inv, int* err, cudaStream_t s);
@@ -57,6 +62,7 @@ struct AttnParams {
   const int32_t* perm;
   const int32_t* counts;
   const int32_t* idx;
+  const int32_t* qperm;   // NULL, or S2O's query permutation [B, Hq, N]
   int cap, blk, seg, nb, G;
   const float* gate_thr;
   int early_stop;         // S2O early stopping: lists in visiting order, cut by stop_tau

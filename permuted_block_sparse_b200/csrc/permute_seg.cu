@@ -60,12 +60,6 @@ __global__ void __launch_bounds__(256) pool_segment_queries_kernel(
   }
 }
 
-// Order-preserving map of a double onto unsigned 64-bit integers.
-__device__ __forceinline__ uint64_t ordered_u64(double x) {
-  const uint64_t u = static_cast<uint64_t>(__double_as_longlong(x));
-  return (u & 0x8000000000000000ull) ? ~u : (u | 0x8000000000000000ull);
-}
-
 // One CTA per (key segment j, query segment s, b * Hkv + hkv).  For j < s:
 // fp64 scores of j's keys against s's representative query, then a bitonic
 // sort of (descending score, ascending position) pairs in shared memory.
@@ -125,28 +119,8 @@ __global__ void __launch_bounds__(1024) score_sort_seg_kernel(
     idx[r] = 0xffffffffu;
   }
   __syncthreads();
-  // bitonic sort of (key, idx) pairs, lexicographic: a total order on
-  // distinct positions, so equal scores keep ascending position
-  for (int k = 2; k <= n2; k <<= 1) {
-    for (int jj = k >> 1; jj > 0; jj >>= 1) {
-      for (int i = threadIdx.x; i < n2; i += blockDim.x) {
-        const int ixj = i ^ jj;
-        if (ixj > i) {
-          const uint64_t a = key[i], c = key[ixj];
-          const uint32_t ia = idx[i], ic = idx[ixj];
-          const bool greater = a > c || (a == c && ia > ic);
-          const bool up = (i & k) == 0;
-          if (greater == up) {
-            key[i] = c;
-            key[ixj] = a;
-            idx[i] = ic;
-            idx[ixj] = ia;
-          }
-        }
-      }
-      __syncthreads();
-    }
-  }
+  // lexicographic on (key, idx): equal scores keep ascending position
+  cta_bitonic_sort(key, idx, n2);
   for (int r = threadIdx.x; r < len; r += blockDim.x) out[r] = static_cast<int32_t>(lo + idx[r]);
 }
 

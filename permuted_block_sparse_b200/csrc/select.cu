@@ -18,19 +18,33 @@
 namespace pbs {
 namespace {
 
-// Sum of `blk` consecutive rows: one CTA per (block, head, batch); thread =
-// (16-byte chunk, row lane); fp32.
+// Sum of the `blk` rows of query block i: one CTA per (block, head, batch);
+// thread = (16-byte chunk, row lane); fp32.  The rows are i*blk .. i*blk +
+// blk - 1, or with a query permutation (qperm, [B, H, N]) the positions
+// qperm[i*blk + r]; an entry outside block i's segment sets the error word
+// and is skipped.
 __global__ void __launch_bounds__(256) pool_query_blocks_kernel(
     const __nv_bfloat16* __restrict__ Q, int64_t sB, int64_t sH, int64_t sN, int D, int blk,
-    float* __restrict__ qbar) {
+    const int32_t* __restrict__ qperm, int64_t N, int seg, int* err, float* __restrict__ qbar) {
   const int i = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int nb = gridDim.x, H = gridDim.y;
   const int nchunk = D / 8, chunk = threadIdx.x % nchunk;
   const int lanes = blockDim.x / nchunk, rl = threadIdx.x / nchunk;
-  const __nv_bfloat16* base = Q + b * sB + h * sH + static_cast<int64_t>(i) * blk * sN;
+  const int64_t p0 = static_cast<int64_t>(i) * blk;
+  const __nv_bfloat16* base = Q + b * sB + h * sH;
+  const int32_t* qrow = qperm ? qperm + (static_cast<int64_t>(b) * H + h) * N + p0 : nullptr;
+  const int64_t seg_lo = (p0 / seg) * seg, seg_hi = min(seg_lo + seg, N);
   float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
   for (int r = rl; r < blk; r += lanes) {
-    const uint4 v = *reinterpret_cast<const uint4*>(base + r * sN + chunk * 8);
+    int64_t n = p0 + r;
+    if (qrow) {
+      n = qrow[r];
+      if (n < seg_lo || n >= seg_hi) {
+        set_error(err, kErrDeviceCheck);
+        continue;
+      }
+    }
+    const uint4 v = *reinterpret_cast<const uint4*>(base + n * sN + chunk * 8);
     const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v);
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
@@ -585,10 +599,12 @@ __global__ void __launch_bounds__(kSelThreads) select_tau_kernel(
 
 }  // namespace
 
-cudaError_t launch_pool_query_blocks(const TensorDesc& Q, int blk, float* qbar, cudaStream_t s) {
+cudaError_t launch_pool_query_blocks(const TensorDesc& Q, int blk, const int32_t* qperm, int seg, int* err,
+                                     float* qbar, cudaStream_t s) {
   dim3 grid(static_cast<unsigned>(Q.N / blk), static_cast<unsigned>(Q.H), static_cast<unsigned>(Q.B));
   pool_query_blocks_kernel<<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(Q.ptr), Q.sB,
-                                                 Q.sH, Q.sN, static_cast<int>(Q.D), blk, qbar);
+                                                 Q.sH, Q.sN, static_cast<int>(Q.D), blk, qperm, Q.N, seg, err,
+                                                 qbar);
   return cudaGetLastError();
 }
 

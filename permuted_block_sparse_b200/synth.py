@@ -67,6 +67,7 @@ class Workload:
     local_pmin: float = 32.0  # shortest and longest period of the pairs, in positions
     local_pmax: float = 32768.0
     perm_per_segment: bool = False   # one key permutation per query segment
+    query_perm: bool = False  # S2O's query permutation (queries sorted per segment by a guide vector)
     stripe_frac: float = 0.0
     c_lo: float = 4.0
     c_hi: float = 4.0
@@ -114,6 +115,12 @@ WORKLOADS = {
     # score, Pass 2 cut once a tile adds less than 2 % of the accumulated
     # mass.  The pages give no threshold; 2 % is an operating point at which
     # late query blocks of these inputs run about a fifth of their candidates.
+    # S2O's query permutation on the 32K shape: queries reordered inside
+    # each segment by their score against the KV head's guide vector, top-k
+    # 10% of the permuted key blocks per permuted query block.
+    "s2o_32k_qperm": Workload(
+        "s2o_32k_qperm", B=1, Hq=32, Hkv=8, N=32768, d=128, blk=128, seg=2048,
+        mode="topk", density=0.1, query_perm=True, stripe_frac=0.005, c_lo=3.0, c_hi=6.0),
     "s2o_32k_stop": Workload(
         "s2o_32k_stop", B=1, Hq=32, Hkv=8, N=32768, d=128, blk=128, seg=2048,
         mode="topk", density=1.0, stop_tau=0.02, stripe_frac=0.005, c_lo=3.0, c_hi=6.0),
