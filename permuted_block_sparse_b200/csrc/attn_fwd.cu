@@ -98,7 +98,9 @@ struct Shared {
 // head); tiles of a head that has stopped are not loaded and only passed
 // through the rings.
 template <int D, int BLK, bool ES, bool QP>
-__global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
+__global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p, const __grid_constant__ CUtensorMap mq,
+                                                                const __grid_constant__ CUtensorMap mk,
+                                                                const __grid_constant__ CUtensorMap mv) {
   using C = Cfg<D, BLK>;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
@@ -325,8 +327,22 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
         if (r < BLK) cp_async16(dst + cc_off + sw128_offset(r, cc % 8), base + x[k] * sN + cc * 8);
       }
     };
-    // Q tiles of both heads (rows >= BLK zero-filled when BLK < 128)
-    for (int h = 0; h < (has1 ? 2 : 1); ++h) {
+    // Q tiles of both heads: by TMA (one thread, 64-column boxes) where the
+    // rows are contiguous, else by cp.async (rows >= BLK zero-filled when
+    // BLK < 128; with permuted queries each row from its own position).
+    const bool tma_q = p.tma && !QP;
+    if (tma_q) {
+      if (pt == 0 && !p.test_wait_limit) {
+        mbar_expect_tx(&sh.bar_q, static_cast<uint32_t>((has1 ? 2 : 1) * C::kQBytes));
+        for (int h = 0; h < (has1 ? 2 : 1); ++h)
+          for (int c = 0; c < D / 64; ++c)
+            tma_rows_4d(sQ0 + h * C::kQBytes + c * (kM * 128), &mq, c * 64, static_cast<int>(q0), h0 + h, b,
+                        &sh.bar_q);
+      } else if (pt != 0 && !p.test_wait_limit) {
+        mbar_arrive(&sh.bar_q);
+      }
+    }
+    for (int h = 0; h < (has1 ? 2 : 1) && !tma_q; ++h) {
       const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(p.Q.ptr) + b * p.Q.sB + (h0 + h) * p.Q.sH;
       const uint32_t dst = sQ0 + h * C::kQBytes;
       for (int id = pt; id < kM * CH; id += kProducerThreads) {
@@ -339,7 +355,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
     }
     // (the failure-path test hook withholds this arrival, so the MMA role's
     // wait for Q runs out)
-    if (!p.test_wait_limit) cp_async_mbar_arrive(&sh.bar_q);
+    if (!p.test_wait_limit && !tma_q) cp_async_mbar_arrive(&sh.bar_q);
+    // A natural tile by TMA: one thread announces the bytes and issues the
+    // 64-column boxes; the other producer threads arrive.
+    auto tma_tile = [&](uint64_t* bar, uint32_t dst, const CUtensorMap* map, int id0) {
+      if (pt == 0) {
+        mbar_expect_tx(bar, static_cast<uint32_t>(C::kKVBytes));
+        for (int c = 0; c < D / 64; ++c) tma_rows_4d(dst + c * (BLK * 128), map, c * 64, id0 * BLK, hk, b, bar);
+      } else {
+        mbar_arrive(bar);
+      }
+    };
     // Row indices of a tile: natural rows, or the permutation's entries for
     // a permuted block.  Loaded one tile ahead into registers and checked
     // when used, so the load latency overlaps the previous tile.
@@ -400,15 +426,23 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
           rowbuf[st][r] = static_cast<int32_t>(x);
         }
         named_sync(1, kProducerThreads);
-        if (!ES || live(t)) gather_tile(sK + st * C::kKVBytes, kb, p.K.sN, rowbuf[st]);
-        cp_async_mbar_arrive(&sh.bar_k[st]);      // arrives when this thread's copies land
+        if (p.tma && nat) {
+          tma_tile(&sh.bar_k[st], sK + st * C::kKVBytes, &mk, id0);
+        } else {
+          if (!ES || live(t)) gather_tile(sK + st * C::kKVBytes, kb, p.K.sN, rowbuf[st]);
+          cp_async_mbar_arrive(&sh.bar_k[st]);    // arrives when this thread's copies land
+        }
       }
       {                                           // V of tile t
         const int sv = t & 1;
         const bool okv = t < kStages || wait_slot(&sh.bar_vempty[sv], ((t >> 1) - 1) & 1, t);
         if (named_sync_or(1, kProducerThreads, !okv)) break;
-        if (!ES || live(t)) gather_tile(sV + sv * C::kKVBytes, vb, p.V.sN, rowbuf[sv]);
-        cp_async_mbar_arrive(&sh.bar_v[sv]);
+        if (p.tma && t < n_diag) {
+          tma_tile(&sh.bar_v[sv], sV + sv * C::kKVBytes, &mv, jtop - t);
+        } else {
+          if (!ES || live(t)) gather_tile(sV + sv * C::kKVBytes, vb, p.V.sN, rowbuf[sv]);
+          cp_async_mbar_arrive(&sh.bar_v[sv]);
+        }
       }
       if (t + 1 < T) fetch_rows(t + 1);
     }
@@ -842,7 +876,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p) {
 }
 
 template <int D, int BLK, bool ES, bool QP>
-cudaError_t launch_typed(const AttnParams& p, cudaStream_t s) {
+cudaError_t launch_typed(const AttnParams& p0, cudaStream_t s) {
+  // Tensor maps for the TMA loads of Q and of natural K/V tiles (128-row
+  // boxes, so BLK = 128 only); without them every tile is gathered.
+  AttnParams p = p0;
+  CUtensorMap mq{}, mk{}, mv{};
+  p.tma = BLK == 128 && encode_rows_map(&mk, p.K) && encode_rows_map(&mv, p.V) && (QP || encode_rows_map(&mq, p.Q));
+  if (!p.tma || QP) mq = mk;                       // unused
   using C = Cfg<D, BLK>;
   // schedule: at most min(candidates, 2 * cap) permuted tiles per item
   // (with early stopping both lists in full, compacted first in the V ring)
@@ -857,7 +897,7 @@ cudaError_t launch_typed(const AttnParams& p, cudaStream_t s) {
   const int npair = (p.G + 1) / 2;
   const int64_t items = static_cast<int64_t>(p.nb) * p.Q.B * p.K.H * npair;
   if (items >= (1ll << 31)) return cudaErrorInvalidValue;
-  attn_fwd_kernel<D, BLK, ES, QP><<<static_cast<unsigned>(items), kThreads, smem, s>>>(p);
+  attn_fwd_kernel<D, BLK, ES, QP><<<static_cast<unsigned>(items), kThreads, smem, s>>>(p, mq, mk, mv);
   return cudaGetLastError();
 }
 

@@ -4,6 +4,7 @@
 // PTX ISA's description of each instruction.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -180,6 +181,25 @@ __device__ __forceinline__ void cp_async_mbar_arrive(uint64_t* bar) {
 // (tensor-core operand reads).
 __device__ __forceinline__ void fence_proxy_async() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// ---------------------------------------------------------------------- TMA
+// mbarrier arrive that also announces `bytes` of asynchronous copies.
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+// One box of a [B, H, N, D] bf16 tensor (coordinates d, n, h, b; the box
+// shape is the tensor map's) into this CTA's shared memory, completing on
+// `bar`.  Callers pass d = 0 or 64, so the innermost coordinate is always a
+// multiple of 16 bytes.  No multicast.
+__device__ __forceinline__ void tma_rows_4d(uint32_t dst, const CUtensorMap* map, int d, int n, int h, int b,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+      "[%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(d), "r"(n), "r"(h), "r"(b), "r"(smem_u32(bar))
+      : "memory");
 }
 
 // ------------------------------------------------------------------ tcgen05

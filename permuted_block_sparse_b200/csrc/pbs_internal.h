@@ -2,6 +2,8 @@
 // kernel translation units.  Host-only; not part of the public ABI.
 #pragma once
 
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -13,6 +15,12 @@ struct TensorDesc {       // validated pbs_tensor, strides in elements
   const void* ptr;
   int64_t B, H, N, D, sB, sH, sN;
 };
+
+// Tensor map of a [B, H, N, D] bf16 tensor for boxes of 64 columns x 128
+// rows, 128-byte swizzle, rows past N read as zeros; false if the tensor
+// cannot be described (a zero head or batch stride over several heads or
+// batches) or the driver entry point is missing.  (select_sample.cu)
+bool encode_rows_map(CUtensorMap* map, const TensorDesc& t);
 
 // pbs_permute launchers ---------------------------------------------------
 cudaError_t launch_pool_proxy_query(const TensorDesc& Q, int Hkv, int blk, float* qhat,
@@ -68,6 +76,7 @@ struct AttnParams {
   int early_stop;         // S2O early stopping: lists in visiting order, cut by stop_tau
   int perm_nseg;          // 1: one permutation per KV head; else one per query segment
   int cta_pair;           // run the CTA-pair kernel where it applies
+  int tma;                // set by the launcher: Q and natural K/V tiles by TMA
   // Failure-path test hook (0 in normal use): bound the role waits by this
   // many polls and withhold the "Q landed" arrival, so the kernel times out.
   uint32_t test_wait_limit;

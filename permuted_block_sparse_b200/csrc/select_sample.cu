@@ -75,22 +75,6 @@ struct SampleCfg {
 constexpr int kScoreThreads = 640;                            // warps 2-3 only join the teardown
 constexpr int kScoreConsumers = 512;                          // warps 4-19
 
-// mbarrier arrive that also announces `bytes` of asynchronous copies.
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
-               : "memory");
-}
-// One 64-column x 128-row box of a [B, H, N, D] bf16 tensor (coordinates
-// d, n, h, b) into shared memory, completing on `bar`.  d is 0 or 64, so the
-// innermost coordinate is always a multiple of 16 bytes.
-__device__ __forceinline__ void tma_rows_4d(uint32_t dst, const CUtensorMap* map, int d, int n, int h, int b,
-                                            uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
-      "[%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(d), "r"(n), "r"(h), "r"(b), "r"(smem_u32(bar))
-      : "memory");
-}
 
 template <int D>
 __global__ void __launch_bounds__(kScoreThreads, 1) sample_scores_kernel(
@@ -561,6 +545,8 @@ __global__ void __launch_bounds__(kSampleWarps * 32) sample_lists_kernel(
   }
 }
 
+}  // namespace
+
 // cuTensorMapEncodeTiled from the driver, looked up once through the runtime.
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   static const PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
@@ -594,8 +580,6 @@ bool encode_rows_map(CUtensorMap* map, const TensorDesc& t) {
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
-
-}  // namespace
 
 cudaError_t launch_select_sample(const SelectParams& p, const TensorDesc& Q, const TensorDesc& K,
                                  float scale_log2, double* col, double* sl, uint32_t* keep_col,
