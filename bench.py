@@ -71,7 +71,8 @@ def selection_label(w) -> str:
         return (f"topk density={w.density} in descending block score, early stop at gain < {w.stop_tau}"
                 + (", one key permutation per query segment" if w.perm_per_segment else ""))
     sel = f"topk density={w.density}" if w.mode == "topk" else f"tau={w.tau}"
-    return sel + (f" band={w.band}" if w.band else "") + (f" n_sink={w.n_sink}" if w.n_sink else "")
+    return (sel + (f" band={w.band}" if w.band else "") + (f" n_sink={w.n_sink}" if w.n_sink else "")
+            + (", queries permuted per segment by the guide vector (S2O)" if w.query_perm else ""))
 
 
 def arm_config(w) -> dict:
@@ -95,7 +96,12 @@ def permute_bytes(w):
     nseg = (w.N + w.seg - 1) // w.seg
     n_perm = w.B * w.Hkv * w.N * (nseg if w.perm_per_segment else 1)
     q_read = w.B * w.Hq * (w.N if w.perm_per_segment else w.blk) * w.d * 2
-    return w.B * w.Hkv * w.N * w.d * 2 + q_read + n_perm * 4
+    k_read = w.B * w.Hkv * w.N * w.d * 2
+    if w.query_perm:
+        # the query permutation reads K again (guide vectors) and Q once, and
+        # writes qperm
+        return 2 * k_read + q_read + w.B * w.Hq * w.N * w.d * 2 + n_perm * 4 + w.B * w.Hq * w.N * 4
+    return k_read + q_read + n_perm * 4
 
 
 def select_bytes(w, cap):
@@ -224,10 +230,18 @@ def oracle_baseline(w, Q, K, V, budget_s: float = 20.0, n_blocks: int = 48):
         else:
             perm1 = oracle.permute(Q[:, qh], K[:, kv], w.blk, w.seg, w.n_sink)
             perm = np.zeros((w.B, w.Hkv, w.N), np.int32)
+        qsel = Q
+        if w.query_perm:
+            # the query permutation of the sampled heads (all heads of KV head
+            # 0, or all) is part of the permutation step
+            qp1 = oracle.permute_queries(Q[:, qh], K[:, kv], w.seg)
+            qperm = np.broadcast_to(np.arange(w.N, dtype=np.int32), (w.B, w.Hq, w.N)).copy()
+            qperm[:, :qp1.shape[1]] = qp1
+            qsel = oracle.gather_queries(Q, qperm)
         t_perm = time.perf_counter() - t0
         perm[:, :perm1.shape[1]] = perm1
         t0 = time.perf_counter()
-        counts, lists = oracle.select(Q, K, perm, w.blk, w.seg, w.mode, density=w.density, tau=w.tau,
+        counts, lists = oracle.select(qsel, K, perm, w.blk, w.seg, w.mode, density=w.density, tau=w.tau,
                                       band=w.band, n_sink=w.n_sink, rows=blocks,
                                       list_order="score" if w.stop_tau > 0 else "ascending")
         t_sel = time.perf_counter() - t0
@@ -236,6 +250,10 @@ def oracle_baseline(w, Q, K, V, budget_s: float = 20.0, n_blocks: int = 48):
     for key in blocks:
         if w.stop_tau > 0:
             oracle.attn_early_stop(Q, K, V, perm, lists, w.blk, w.seg, w.stop_tau, [key])
+        elif w.query_perm:
+            b_, h_, i_ = key
+            oracle.attn_block_qperm(Q, K, V, perm, qperm, lists.get(key, np.zeros(0, np.int32)), b_, h_, i_,
+                                    w.blk, w.seg, 1.0 / math.sqrt(w.d))
         else:
             oracle.attn_blocks(Q, K, V, perm, lists, w.blk, w.seg, [key], gate_thr=thr)
         done.append(key)
@@ -317,6 +335,13 @@ def run_pbs(args):
     permute = pbs.pbs_permute_segmented if segperm else pbs.pbs_permute
     stats = torch.zeros(2, dtype=torch.int64, device=dev)
     launches_per_step = 6   # 2 permute + 3 select + 1 attention kernels
+    qperm_on = w.query_perm        # S2O's query permutation
+    qperm = ws_q = None
+    if qperm_on:
+        qperm = torch.empty((w.B, w.Hq, w.N), dtype=torch.int32, device=dev)
+        ws_q = torch.empty(pbs.workspace_size(pbs.PBS_OP_PERMUTE_QUERIES, Q, K, w.blk, w.seg) + 256,
+                           dtype=torch.uint8, device=dev)
+        launches_per_step = 9   # 2 + 3 permute (keys, queries) + 3 select + 1 attention
     # Block-max gating workloads: no permutation or selection step; every
     # earlier block is listed and the thresholds (calibrated offline by the
     # oracle, stored beside the tests) decide per tile.
@@ -343,9 +368,14 @@ def run_pbs(args):
             e[0].record(s)
         if not gate and not sample:
             permute(Q, K, w.blk, w.seg, w.n_sink, perm=perm, ws=ws_p)
+        if qperm_on:
+            pbs.pbs_permute_queries(Q, K, w.blk, w.seg, qperm=qperm, ws=ws_q)
         if record:
             e[1].record(s)
-        if not gate:
+        if qperm_on:
+            pbs.pbs_select_qperm(Q, K, perm, qperm, w.blk, w.seg, w.mode, dt, w.n_sink, cap=cap, counts=counts,
+                                 idx=idx, ws=ws_s)
+        elif not gate:
             pbs.pbs_select(Q, K, None if sample else perm, w.blk, w.seg, w.mode, dt, w.band, w.n_sink, cap=cap,
                            counts=counts, idx=idx, ws=ws_s, score_order=early)
         if record:
@@ -353,6 +383,8 @@ def run_pbs(args):
         if early:
             pbs.pbs_attn_fwd_early_stop(Q, K, V, perm, counts, idx, w.blk, w.seg, w.stop_tau, out=O, lse=lse,
                                         stats=st)
+        elif qperm_on:
+            pbs.pbs_attn_fwd_qperm(Q, K, V, perm, qperm, counts, idx, w.blk, w.seg, out=O, lse=lse, stats=st)
         else:
             pbs.pbs_attn_fwd(Q, K, V, perm, counts, idx, w.blk, w.seg, out=O, lse=lse, stats=st, gate_thr=thr)
         if record:
@@ -465,7 +497,10 @@ def run_pbs(args):
     # overlaps the copies of one KV head's unit with the kernels of another
     # on three streams; the result must equal the device-resident run's O.
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and qperm_on:
+        e2e = {"value": None, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0,
+               "note": "the host-memory prefill driver does not take a query permutation"}
+    elif not args.no_e2e:
         from permuted_block_sparse_b200.host_pipeline import HostPrefill
         Qh = torch.from_numpy(Qn).to(torch.bfloat16).pin_memory()
         Kh = torch.from_numpy(Kn).to(torch.bfloat16).pin_memory()

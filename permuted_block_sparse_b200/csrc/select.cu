@@ -196,14 +196,15 @@ __device__ __forceinline__ double block_max_f64(double v, double* red) {
 
 // Block scores S[b, hq, i, pb] = Qbar_i . Kbar_pb for every candidate
 // pb < candidates(i), as a register-tiled fp32 GEMM per (batch, query head):
-// 64 x 64 output tiles, 4 x 4 per thread, d in chunks of 32.  Tiles wholly
-// above the candidate triangle are skipped.  On lattice inputs every
-// partial sum is exact, so any accumulation order gives the same scores.
-constexpr int kTile = 64;
+// 128 x 128 output tiles, 8 x 8 per thread (four 16-byte shared loads per
+// 64 FMAs), d in chunks of 32, accumulated in d order.  Tiles wholly above
+// the candidate triangle are skipped.  On lattice inputs every partial sum
+// is exact, so any accumulation order gives the same scores.
+constexpr int kTile = 128;
 
-__global__ void __launch_bounds__(256) block_scores_kernel(SelectParams p, const float* __restrict__ qbar,
-                                                           const float* __restrict__ kbar_perm,
-                                                           float* __restrict__ S) {
+__global__ void __launch_bounds__(256, 2) block_scores_kernel(SelectParams p, const float* __restrict__ qbar,
+                                                              const float* __restrict__ kbar_perm,
+                                                              float* __restrict__ S) {
   const int ct = blockIdx.x, rt = blockIdx.y, bh = blockIdx.z;
   const int b = bh / p.Hq, h = bh % p.Hq, hk = h / (p.Hq / p.Hkv);
   const int spb = p.seg / p.blk;
@@ -213,11 +214,11 @@ __global__ void __launch_bounds__(256) block_scores_kernel(SelectParams p, const
   __shared__ __align__(16) float qs[32][kTile + 4];     // [d][row]
   __shared__ __align__(16) float ks[32][kTile + 4];     // [d][candidate]
   const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
-  float acc[4][4];
+  float acc[8][8];
 #pragma unroll
-  for (int u = 0; u < 4; ++u)
+  for (int u = 0; u < 8; ++u)
 #pragma unroll
-    for (int v = 0; v < 4; ++v) acc[u][v] = 0.f;
+    for (int v = 0; v < 8; ++v) acc[u][v] = 0.f;
   const float* qsrc = qbar + (static_cast<int64_t>(b) * p.Hq + h) * p.nb * p.D;
   const float* ksrc = kbar_perm + (static_cast<int64_t>(b) * p.Hkv + hk) * p.nb * p.D;
   for (int d0 = 0; d0 < p.D; d0 += 32) {
@@ -234,25 +235,29 @@ __global__ void __launch_bounds__(256) block_scores_kernel(SelectParams p, const
     __syncthreads();
 #pragma unroll 4
     for (int dd = 0; dd < 32; ++dd) {
-      const float4 a = *reinterpret_cast<const float4*>(&qs[dd][ty * 4]);
-      const float4 c = *reinterpret_cast<const float4*>(&ks[dd][tx * 4]);
-      const float av[4] = {a.x, a.y, a.z, a.w}, cv[4] = {c.x, c.y, c.z, c.w};
+      // rows ty*4 .. +3 and 64 + ty*4 .. +3; candidates tx*4 .. +3 and 64 + tx*4 .. +3
+      const float4 a0 = *reinterpret_cast<const float4*>(&qs[dd][ty * 4]);
+      const float4 a1 = *reinterpret_cast<const float4*>(&qs[dd][64 + ty * 4]);
+      const float4 c0 = *reinterpret_cast<const float4*>(&ks[dd][tx * 4]);
+      const float4 c1 = *reinterpret_cast<const float4*>(&ks[dd][64 + tx * 4]);
+      const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      const float cv[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
 #pragma unroll
-      for (int u = 0; u < 4; ++u)
+      for (int u = 0; u < 8; ++u)
 #pragma unroll
-        for (int v = 0; v < 4; ++v) acc[u][v] = fmaf(av[u], cv[v], acc[u][v]);
+        for (int v = 0; v < 8; ++v) acc[u][v] = fmaf(av[u], cv[v], acc[u][v]);
     }
     __syncthreads();
   }
   float* out = S + (static_cast<int64_t>(b) * p.Hq + h) * p.nb * p.nb;
 #pragma unroll
-  for (int u = 0; u < 4; ++u) {
-    const int i = rt * kTile + ty * 4 + u;
+  for (int u = 0; u < 8; ++u) {
+    const int i = rt * kTile + (u < 4 ? ty * 4 + u : 64 + ty * 4 + u - 4);
     if (i >= p.nb) continue;
     const int nc = (i / spb) * spb;
 #pragma unroll
-    for (int v = 0; v < 4; ++v) {
-      const int pb = pb0 + tx * 4 + v;
+    for (int v = 0; v < 8; ++v) {
+      const int pb = pb0 + (v < 4 ? tx * 4 + v : 64 + tx * 4 + v - 4);
       if (pb < nc) out[static_cast<int64_t>(i) * p.nb + pb] = acc[u][v];
     }
   }
@@ -327,15 +332,35 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32) select_topk_kernel(
   auto key_hi = [&](int t) -> uint32_t {
     return ((fbits[t >> 5] >> (t & 31)) & 1u) ? 0u : ~ordered_u32(S[t]);
   };
+  // Rows of up to 32 * kCache candidates keep their keys in registers
+  // (lane l holds candidates l, l + 32, ...), so the row is read once.
+  constexpr int kCache = 32;
+  const bool cached = ncand <= 32 * kCache;
+  uint32_t kr[kCache];
+  if (cached) {
+#pragma unroll
+    for (int j = 0; j < kCache; ++j) {
+      const int t = lane + 32 * j;
+      kr[j] = t < ncand ? key_hi(t) : 0xffffffffu;
+    }
+  }
   uint32_t prefix = 0, pmask = 0;
   int rank = want;
   if (want > 0) {
     for (int shift = 24; shift >= 0; shift -= 8) {
       for (int q = lane; q < 256; q += 32) hist[q] = 0u;
       __syncwarp();
-      for (int t = lane; t < ncand; t += 32) {
-        const uint32_t k = key_hi(t);
-        if ((k & pmask) == prefix) atomicAdd(&hist[(k >> shift) & 255u], 1u);
+      if (cached) {
+#pragma unroll
+        for (int j = 0; j < kCache; ++j) {
+          const uint32_t k = kr[j];
+          if (lane + 32 * j < ncand && (k & pmask) == prefix) atomicAdd(&hist[(k >> shift) & 255u], 1u);
+        }
+      } else {
+        for (int t = lane; t < ncand; t += 32) {
+          const uint32_t k = key_hi(t);
+          if ((k & pmask) == prefix) atomicAdd(&hist[(k >> shift) & 255u], 1u);
+        }
       }
       __syncwarp();
       uint32_t loc[8], sum = 0;
@@ -375,9 +400,9 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32) select_topk_kernel(
   }
   int32_t* out = idx + row * p.cap;
   int written = 0, ties = 0;
-  for (int base = 0; base < ncand && want > 0; base += 32) {
-    const int t = base + lane;
-    const uint32_t k = t < ncand ? key_hi(t) : 0xffffffffu;
+  // Write the chosen ids in ascending order: keys below the threshold, and
+  // the first `rank` keys equal to it.
+  auto emit = [&](int t, uint32_t k) {
     const bool lt = t < ncand && k < prefix;
     const bool eq = t < ncand && k == prefix;
     const uint32_t eqm = __ballot_sync(0xffffffffu, eq);
@@ -387,6 +412,18 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32) select_topk_kernel(
     if (take) out[written + __popc(tm & ((1u << lane) - 1u))] = t;
     written += __popc(tm);
     ties += __popc(eqm);
+  };
+  if (want > 0 && cached) {
+#pragma unroll
+    for (int j = 0; j < kCache; ++j) {
+      if (32 * j >= ncand) break;
+      emit(lane + 32 * j, kr[j]);
+    }
+  } else if (want > 0) {
+    for (int base = 0; base < ncand; base += 32) {
+      const int t = base + lane;
+      emit(t, t < ncand ? key_hi(t) : 0xffffffffu);
+    }
   }
   if (lane == 0) counts[row] = want;
 }
