@@ -56,91 +56,47 @@ __global__ void __launch_bounds__(256) pool_proxy_query_kernel(
 // One CTA per (segment, hkv, b), kSortThreads threads.  Scores every key of
 // the segment with one fp32 dot product against qhat (lanes of a row group
 // read 16 bytes each, a row is one coalesced 128/256-byte read; eight rows
-// per thread in flight), packs (descending score, ascending position) into
-// one 64-bit key and sorts the keys: sorting unique composite keys is a
-// total order, so the result equals a stable descending sort by score.
+// per thread in flight), then sorts the segment by descending score with a
+// stable least-significant-digit radix sort of the 32-bit order-inverted
+// scores (four passes of 8 bits).  The keys start in ascending position and
+// every pass keeps equal digits in their current order, so equal scores end
+// in ascending position: a stable descending sort by score.
 //
-// The sort is bitonic with E keys per thread in registers (thread t holds
-// elements t*E .. t*E+E-1): exchanges between elements of one thread are
-// register swaps, between threads of one warp (partner distance below 32*E)
-// warp shuffles, and only the longer distances go through shared memory
-// with a barrier -- 10 of the 78 stages for a 4096-key segment.
+// A pass over n = kSortThreads * E keys: warp w owns positions
+// [w*32*E, (w+1)*32*E), element (e, lane) at w*32*E + e*32 + lane.  Each
+// warp ranks its keys among equal digits with a match over lanes and
+// running per-digit counters (e in order), a block-wide scan over
+// (digit, warp) in digit-major order gives every warp's offset for every
+// digit, and the keys scatter to offset + rank in a second buffer.
 constexpr int kSortThreads = 512;
-
-template <int E>
-__device__ __forceinline__ void bitonic_regs(uint64_t (&v)[E], int n2, uint64_t* sm) {
-  const int tid = threadIdx.x, lane = tid & 31;
-  for (int k = 2; k <= n2; k <<= 1) {
-    // partner distances j >= E: another thread
-    for (int j = k >> 1; j >= E; j >>= 1) {
-      if (j < 32 * E) {
-        // partner in another lane of this warp: lane ^ (j / E), same e
-        const int lx = j / E;
-        const bool lower = (lane & lx) == 0;
-#pragma unroll
-        for (int e = 0; e < E; ++e) {
-          const bool up = ((tid * E + e) & k) == 0;
-          const uint64_t o = __shfl_xor_sync(0xffffffffu, v[e], lx);
-          const uint64_t mn = v[e] < o ? v[e] : o, mx = v[e] < o ? o : v[e];
-          v[e] = (lower == up) ? mn : mx;
-        }
-      } else {
-        // partner in another warp: through shared memory
-#pragma unroll
-        for (int e = 0; e < E; ++e) sm[tid * E + e] = v[e];
-        __syncthreads();
-#pragma unroll
-        for (int e = 0; e < E; ++e) {
-          const int i = tid * E + e;
-          const bool up = (i & k) == 0, lower = (i & j) == 0;
-          const uint64_t o = sm[i ^ j];
-          const uint64_t mn = v[e] < o ? v[e] : o, mx = v[e] < o ? o : v[e];
-          v[e] = (lower == up) ? mn : mx;
-        }
-        __syncthreads();
-      }
-    }
-    // partner distances j < E: this thread's own registers (static indices)
-#pragma unroll
-    for (int j = E / 2; j > 0; j >>= 1) {
-      if (j < k) {
-#pragma unroll
-        for (int e = 0; e < E; ++e) {
-          if ((e & j) == 0) {
-            const bool up = ((tid * E + e) & k) == 0;
-            const uint64_t a = v[e], c = v[e | j];
-            if ((a > c) == up) {
-              v[e] = c;
-              v[e | j] = a;
-            }
-          }
-        }
-      }
-    }
-  }
-}
+constexpr int kSortWarps = kSortThreads / 32;
 
 template <int E>
 __global__ void __launch_bounds__(kSortThreads, 2) score_sort_kernel(
     const __nv_bfloat16* __restrict__ K, int64_t sB, int64_t sH, int64_t sN, int64_t N, int D,
     int seg, int n_sink, const float* __restrict__ qhat, int32_t* __restrict__ perm) {
+  constexpr int n = kSortThreads * E;
   extern __shared__ __align__(16) unsigned char smem_raw[];
+  uint32_t* skey = reinterpret_cast<uint32_t*>(smem_raw);                 // [2][n]
+  uint16_t* sidx = reinterpret_cast<uint16_t*>(skey + 2 * n);             // [2][n]
+  uint32_t* hist = reinterpret_cast<uint32_t*>(sidx + 2 * n);             // [kSortWarps][256]
+  float* q = reinterpret_cast<float*>(hist + kSortWarps * 256);
+  __shared__ uint32_t wsum[kSortWarps];
   const int t = blockIdx.x, hkv = blockIdx.y, b = blockIdx.z, Hkv = gridDim.y;
   const int64_t lo = static_cast<int64_t>(t) * seg;
   const int len = static_cast<int>(min(static_cast<int64_t>(seg), N - lo));
-  // the whole CTA sorts kSortThreads * E >= len keys; the padding keys
-  // (all ones) sort after every real one
-  const int n2 = kSortThreads * E;
-  uint64_t* keys = reinterpret_cast<uint64_t*>(smem_raw);
-  float* q = reinterpret_cast<float*>(keys + kSortThreads * E);
   for (int c = threadIdx.x; c < D; c += blockDim.x)
     q[c] = qhat[(static_cast<int64_t>(b) * Hkv + hkv) * D + c];
-  for (int r = len + threadIdx.x; r < kSortThreads * E; r += blockDim.x) keys[r] = ~0ull;
+  // padding keys (all ones) come after every real key in the initial order
+  for (int r = threadIdx.x; r < n; r += blockDim.x) {
+    skey[r] = 0xffffffffu;
+    sidx[r] = static_cast<uint16_t>(r);
+  }
   __syncthreads();
 
   const int lanes_per_row = D / 8;           // 16 (D=128) or 8 (D=64)
   const int rows_per_warp = 32 / lanes_per_row;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarp = blockDim.x >> 5;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int sub = lane / lanes_per_row, cl = lane % lanes_per_row;
   const __nv_bfloat16* base = K + b * sB + hkv * sH;
   float qv[8];
@@ -149,7 +105,7 @@ __global__ void __launch_bounds__(kSortThreads, 2) score_sort_kernel(
   // kRowsInFlight rows per thread are loaded before any is used, so each
   // thread keeps that many 16-byte reads in flight.
   constexpr int kRowsInFlight = 8;
-  const int step = nwarp * rows_per_warp;
+  const int step = kSortWarps * rows_per_warp;
   for (int r0 = warp * rows_per_warp; r0 < len; r0 += kRowsInFlight * step) {
     uint4 v[kRowsInFlight];
 #pragma unroll
@@ -172,22 +128,78 @@ __global__ void __launch_bounds__(kSortThreads, 2) score_sort_kernel(
         acc += __shfl_xor_sync(0xffffffffu, acc, off);
       if (r < len && cl == 0) {
         const float sc = (lo + r < n_sink) ? __int_as_float(0x7f800000) : acc;
-        keys[r] = (static_cast<uint64_t>(~ordered_u32(sc)) << 32) | static_cast<uint32_t>(r);
+        skey[r] = ~ordered_u32(sc);                // ascending key = descending score
       }
     }
   }
   __syncthreads();
-  uint64_t v[E];
+
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  int cur = 0;
+  for (int shift = 0; shift < 32; shift += 8) {
+    const uint32_t* kin = skey + cur * n;
+    const uint16_t* iin = sidx + cur * n;
+    uint32_t* kout = skey + (cur ^ 1) * n;
+    uint16_t* iout = sidx + (cur ^ 1) * n;
+    uint32_t* h = hist + warp * 256;
+    for (int d = lane; d < 256; d += 32) h[d] = 0u;
+    __syncwarp();
+    uint32_t key[E], rank[E];
+    uint16_t ix[E];
 #pragma unroll
-  for (int e = 0; e < E; ++e) v[e] = keys[threadIdx.x * E + e];
-  __syncthreads();
-  bitonic_regs<E>(v, n2, keys);
-  int32_t* out = perm + (static_cast<int64_t>(b) * Hkv + hkv) * N + lo;
+    for (int e = 0; e < E; ++e) {
+      const int pos = warp * 32 * E + e * 32 + lane;
+      key[e] = kin[pos];
+      ix[e] = iin[pos];
+      const uint32_t dg = (key[e] >> shift) & 255u;
+      const uint32_t peers = __match_any_sync(0xffffffffu, dg);
+      const uint32_t before = h[dg];
+      rank[e] = before + __popc(peers & lt_mask);
+      __syncwarp();
+      if ((peers & lt_mask) == 0u) h[dg] = before + __popc(peers);   // the lowest peer lane
+      __syncwarp();
+    }
+    __syncthreads();
+    // exclusive scan over (digit, warp), digit-major: thread tid covers
+    // digit tid / 2, warps (tid % 2) * 8 .. + 7
+    {
+      const int dg = threadIdx.x >> 1, w0 = (threadIdx.x & 1) * 8;
+      uint32_t c[8], tot = 0;
 #pragma unroll
-  for (int e = 0; e < E; ++e) {
-    const int r = threadIdx.x * E + e;
-    if (r < len) out[r] = static_cast<int32_t>(lo + static_cast<uint32_t>(v[e] & 0xffffffffu));
+      for (int j = 0; j < 8; ++j) {
+        c[j] = hist[(w0 + j) * 256 + dg];
+        tot += c[j];
+      }
+      uint32_t incl = tot;
+      for (int off = 1; off < 32; off <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += y;
+      }
+      if (lane == 31) wsum[warp] = incl;
+      __syncthreads();
+      uint32_t wpre = 0;
+      for (int w = 0; w < warp; ++w) wpre += wsum[w];
+      uint32_t run = wpre + incl - tot;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        hist[(w0 + j) * 256 + dg] = run;           // now this warp's offset for the digit
+        run += c[j];
+      }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      const uint32_t dg = (key[e] >> shift) & 255u;
+      const uint32_t dst = h[dg] + rank[e];
+      kout[dst] = key[e];
+      iout[dst] = ix[e];
+    }
+    __syncthreads();
+    cur ^= 1;
   }
+  const uint16_t* order = sidx + cur * n;
+  int32_t* out = perm + (static_cast<int64_t>(b) * Hkv + hkv) * N + lo;
+  for (int r = threadIdx.x; r < len; r += blockDim.x) out[r] = static_cast<int32_t>(lo + order[r]);
 }
 
 }  // namespace
@@ -206,7 +218,8 @@ cudaError_t launch_score_sort(const TensorDesc& K, int seg, int n_sink, const fl
   const int64_t nseg = (K.N + seg - 1) / seg;
   dim3 grid(static_cast<unsigned>(nseg), static_cast<unsigned>(K.H), static_cast<unsigned>(K.B));
   auto run = [&](auto kernel, int E) -> cudaError_t {
-    const size_t smem = static_cast<size_t>(kSortThreads) * E * 8 + K.D * 4;
+    const size_t n = static_cast<size_t>(kSortThreads) * E;
+    const size_t smem = n * 2 * 4 + n * 2 * 2 + kSortWarps * 256 * 4 + K.D * 4;
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     kernel<<<grid, kSortThreads, smem, s>>>(static_cast<const __nv_bfloat16*>(K.ptr), K.sB, K.sH, K.sN, K.N,
