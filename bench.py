@@ -44,6 +44,9 @@ def parse():
     ap.add_argument("--no-dense", action="store_true", help="skip the dense same-kernel comparison run")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
+    ap.add_argument("--seq-len", type=int, default=0,
+                    help="run the workload's settings at this sequence length instead of its own "
+                         "(scaled-down cases for counter captures; not a bench line)")
     return ap.parse_args()
 
 
@@ -310,6 +313,11 @@ def run_pbs(args):
 
     from permuted_block_sparse_b200 import shard
     w = synth.WORKLOADS[args.workload]
+    if args.seq_len:
+        if w.mode == "gate" or args.seq_len % w.blk:
+            raise SystemExit("--seq-len: a multiple of the block size, and not for the gate workloads "
+                             "(their thresholds are calibrated at the workload's own length)")
+        w = w.with_(N=args.seq_len)
     Qn, Kn, Vn, _ = synth.make_inputs(w, seed=shard.seed_for_rank(w.seed, rank))
     Q = torch.from_numpy(Qn).to(torch.bfloat16).to(dev)
     K = torch.from_numpy(Kn).to(torch.bfloat16).to(dev)
@@ -452,7 +460,7 @@ def run_pbs(args):
         pbs.pbs_check_device()
         dms = a.elapsed_time(b) / reps
         dense = {"ms": dms, "tflops": causal_tiles * tile_flops(w) / (dms * 1e-3) / 1e12,
-                 "speedup_of_sparse_step": dms / ms_step}
+                 "speedup_of_sparse_step": dms / ms_step, "speedup_of_sparse_attention": dms / ms_attn}
         # Attention coverage (outside the timed region): the share of each
         # row's full causal softmax mass on its key set is exp(LSE over the
         # key set - LSE over all causal keys).  The permuted selection of the

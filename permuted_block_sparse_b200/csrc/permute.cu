@@ -27,16 +27,25 @@ __global__ void __launch_bounds__(256) pool_proxy_query_kernel(
   const int rl = threadIdx.x / nchunk;
   float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
   const int rows = G * blk;
-  for (int r = rl; r < rows; r += lanes) {
-    const int h = hkv * G + r / blk;
-    const int64_t n = N - blk + (r % blk);
-    const uint4 v = *reinterpret_cast<const uint4*>(Q + b * sB + h * sH + n * sN + chunk * 8);
-    const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v);
+  // eight rows per thread in flight, then added in row order
+  for (int r0 = rl; r0 < rows; r0 += 8 * lanes) {
+    uint4 v[8];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      float2 f = __bfloat1622float2(p[e]);
-      acc[2 * e] += f.x;
-      acc[2 * e + 1] += f.y;
+    for (int u = 0; u < 8; ++u) {
+      const int r = r0 + u * lanes;
+      const int h = hkv * G + r / blk;
+      const int64_t n = N - blk + (r % blk);
+      v[u] = r < rows ? *reinterpret_cast<const uint4*>(Q + b * sB + h * sH + n * sN + chunk * 8) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v[u]);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        float2 f = __bfloat1622float2(p[e]);
+        acc[2 * e] += f.x;
+        acc[2 * e + 1] += f.y;
+      }
     }
   }
   __shared__ float red[256 * 8];
