@@ -356,12 +356,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p, con
     // (the failure-path test hook withholds this arrival, so the MMA role's
     // wait for Q runs out)
     if (!p.test_wait_limit && !tma_q) cp_async_mbar_arrive(&sh.bar_q);
-    // A natural tile by TMA: one thread announces the bytes and issues the
-    // 64-column boxes; the other producer threads arrive.
-    auto tma_tile = [&](uint64_t* bar, uint32_t dst, const CUtensorMap* map, int id0) {
+    // A tile of BLK contiguous rows (from row0) by TMA: one thread announces
+    // the bytes and issues the 64-column boxes; the other producer threads
+    // arrive.
+    auto tma_tile = [&](uint64_t* bar, uint32_t dst, const CUtensorMap* map, int row0) {
       if (pt == 0) {
         mbar_expect_tx(bar, static_cast<uint32_t>(C::kKVBytes));
-        for (int c = 0; c < D / 64; ++c) tma_rows_4d(dst + c * (BLK * 128), map, c * 64, id0 * BLK, hk, b, bar);
+        for (int c = 0; c < D / 64; ++c) tma_rows_4d(dst + c * (BLK * 128), map, c * 64, row0, hk, b, bar);
       } else {
         mbar_arrive(bar);
       }
@@ -401,6 +402,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p, con
     // would put the gather's latency in front of every kept tile's PV.
     // (A dropped tile's V is gathered but never multiplied.)
     for (int t = 0; t < T; ++t) {
+      // first row of the tile when its rows are contiguous (natural blocks;
+      // a permuted block whose entries happen to run in order, as with the
+      // identity permutation), loaded by TMA; else -1 and gathered row by row
+      int row0 = -1;
       {                                           // K of tile t
         const int st = t & 1;
         const bool ok = t < kStages || wait_slot(&sh.bar_kempty[st], ((t >> 1) - 1) & 1, t);
@@ -426,8 +431,21 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p, con
           rowbuf[st][r] = static_cast<int32_t>(x);
         }
         named_sync(1, kProducerThreads);
-        if (p.tma && nat) {
-          tma_tile(&sh.bar_k[st], sK + st * C::kKVBytes, &mk, id0);
+        if (nat) row0 = id0 * BLK;
+        if constexpr (!ES) {
+          if (p.tma && !nat) {
+            const int32_t x0 = rowbuf[st][0];
+            bool run = true;
+#pragma unroll
+            for (int q = 0; q < RPT; ++q) {
+              const int r = pt + q * kProducerThreads;
+              if (r < BLK) run = run && rowbuf[st][r] == x0 + r;
+            }
+            if (!named_sync_or(1, kProducerThreads, !run)) row0 = x0;
+          }
+        }
+        if (p.tma && row0 >= 0) {
+          tma_tile(&sh.bar_k[st], sK + st * C::kKVBytes, &mk, row0);
         } else {
           if (!ES || live(t)) gather_tile(sK + st * C::kKVBytes, kb, p.K.sN, rowbuf[st]);
           cp_async_mbar_arrive(&sh.bar_k[st]);    // arrives when this thread's copies land
@@ -437,8 +455,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p, con
         const int sv = t & 1;
         const bool okv = t < kStages || wait_slot(&sh.bar_vempty[sv], ((t >> 1) - 1) & 1, t);
         if (named_sync_or(1, kProducerThreads, !okv)) break;
-        if (p.tma && t < n_diag) {
-          tma_tile(&sh.bar_v[sv], sV + sv * C::kKVBytes, &mv, jtop - t);
+        if (p.tma && row0 >= 0) {
+          tma_tile(&sh.bar_v[sv], sV + sv * C::kKVBytes, &mv, row0);
         } else {
           if (!ES || live(t)) gather_tile(sV + sv * C::kKVBytes, vb, p.V.sN, rowbuf[sv]);
           cp_async_mbar_arrive(&sh.bar_v[sv]);
