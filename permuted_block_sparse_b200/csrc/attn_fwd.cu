@@ -137,6 +137,47 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p, con
   const uint32_t sV = smem_u32(smem + C::kV);
 
   // ------------------------------------------------------------------ setup
+  // Barriers first, so that the loads that need no schedule -- Q and, in
+  // natural query order, the diagonal block's K and V (tile 0) -- start by
+  // TMA while warp 0 builds the schedule.
+  if (tid == 32) {
+    sh.abort = 0;
+    sh.limit[0] = 0x7fffffff;
+    sh.limit[1] = 0x7fffffff;
+    mbar_init(&sh.bar_q, kProducerThreads);
+    for (int st = 0; st < kStages; ++st) {
+      mbar_init(&sh.bar_k[st], kProducerThreads);
+      mbar_init(&sh.bar_v[st], kProducerThreads);
+      mbar_init(&sh.bar_kempty[st], 1);
+      mbar_init(&sh.bar_vempty[st], 1);
+    }
+    for (int h = 0; h < 2; ++h) {
+      mbar_init(&sh.bar_s[h], 1);
+      mbar_init(&sh.bar_p[h], 4);               // one arrival per softmax warp
+      mbar_init(&sh.bar_o[h], 1);
+    }
+    mbar_init(&sh.bar_fin, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  // (the failure-path test hook withholds the Q loads; with early stopping
+  // warp 0 compacts the lists in the V ring during set-up, so tile 0 waits)
+  const bool early = p.tma && !QP && !p.test_wait_limit;
+  const bool early_kv = early && !ES;
+  if (tid == 32 && early) {
+    mbar_expect_tx(&sh.bar_q, static_cast<uint32_t>((has1 ? 2 : 1) * C::kQBytes));
+    for (int h = 0; h < (has1 ? 2 : 1); ++h)
+      for (int c = 0; c < D / 64; ++c)
+        tma_rows_4d(sQ0 + h * C::kQBytes + c * (kM * 128), &mq, c * 64, static_cast<int>(q0), h0 + h, b, &sh.bar_q);
+  }
+  if (tid == 32 && early_kv) {
+    mbar_expect_tx(&sh.bar_k[0], static_cast<uint32_t>(C::kKVBytes));
+    for (int c = 0; c < D / 64; ++c)
+      tma_rows_4d(sK + c * (BLK * 128), &mk, c * 64, i * BLK, hk, b, &sh.bar_k[0]);
+    mbar_expect_tx(&sh.bar_v[0], static_cast<uint32_t>(C::kKVBytes));
+    for (int c = 0; c < D / 64; ++c)
+      tma_rows_4d(sV + c * (BLK * 128), &mv, c * 64, i * BLK, hk, b, &sh.bar_v[0]);
+  }
   if (warp == 0) {
     tmem_alloc(&sh.tmem_base, 512);
     tmem_relinquish();
@@ -198,15 +239,33 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p, con
         sh.n_list[1] = nl[1];
       }
     }
-    for (int h = 0; h < 2 && !ES; ++h) {
-      const int32_t* list = p.idx + ((static_cast<int64_t>(b) * Hq + h0 + h) * p.nb + i) * p.cap;
-      for (int e = lane; e < cnt[h]; e += 32) {
-        const int pb = list[e];
-        if (pb < 0 || pb >= ncand) {
-          set_error(p.err, kErrDeviceCheck);
-          continue;
+    if (!ES) {
+      // both heads' entries in batches of 8 per lane, all loads in flight
+      // before the first is used (one memory round trip per 256 entries)
+      constexpr int kBatch = 8;
+      const int32_t* list0 = p.idx + ((static_cast<int64_t>(b) * Hq + h0) * p.nb + i) * p.cap;
+      const int32_t* list1 = list0 + static_cast<int64_t>(p.nb) * p.cap;   // next head's row (read only if cnt[1] > 0)
+      for (int base = 0; base < max(cnt[0], cnt[1]); base += 32 * kBatch) {
+        int pb[2][kBatch];
+#pragma unroll
+        for (int j = 0; j < kBatch; ++j) {
+          const int e = base + lane + 32 * j;
+          pb[0][j] = e < cnt[0] ? list0[e] : 0;
+          pb[1][j] = e < cnt[1] ? list1[e] : 0;
         }
-        atomicOr(&bm[h][pb >> 5], 1u << (pb & 31));
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+#pragma unroll
+          for (int j = 0; j < kBatch; ++j) {
+            if (base + lane + 32 * j >= cnt[h]) continue;
+            const int v = pb[h][j];
+            if (v < 0 || v >= ncand) {
+              set_error(p.err, kErrDeviceCheck);
+              continue;
+            }
+            atomicOr(&bm[h][v >> 5], 1u << (v & 31));
+          }
+        }
       }
     }
     __syncwarp();
@@ -232,23 +291,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p, con
     if (lane == 0) {
       sh.n_union = total;
       sh.jtop = i;
-      sh.abort = 0;
-      sh.limit[0] = 0x7fffffff;
-      sh.limit[1] = 0x7fffffff;
-      mbar_init(&sh.bar_q, kProducerThreads);
-      for (int st = 0; st < kStages; ++st) {
-        mbar_init(&sh.bar_k[st], kProducerThreads);
-        mbar_init(&sh.bar_v[st], kProducerThreads);
-        mbar_init(&sh.bar_kempty[st], 1);
-        mbar_init(&sh.bar_vempty[st], 1);
-      }
-      for (int h = 0; h < 2; ++h) {
-        mbar_init(&sh.bar_s[h], 1);
-        mbar_init(&sh.bar_p[h], 4);             // one arrival per softmax warp
-        mbar_init(&sh.bar_o[h], 1);
-      }
-      mbar_init(&sh.bar_fin, 1);
-      fence_mbar_init();
     }
     if (QP) {
       // Rows' query positions (each must lie in the block's segment; an
@@ -332,15 +374,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p, con
     // BLK < 128; with permuted queries each row from its own position).
     const bool tma_q = p.tma && !QP;
     if (tma_q) {
-      if (pt == 0 && !p.test_wait_limit) {
-        mbar_expect_tx(&sh.bar_q, static_cast<uint32_t>((has1 ? 2 : 1) * C::kQBytes));
-        for (int h = 0; h < (has1 ? 2 : 1); ++h)
-          for (int c = 0; c < D / 64; ++c)
-            tma_rows_4d(sQ0 + h * C::kQBytes + c * (kM * 128), &mq, c * 64, static_cast<int>(q0), h0 + h, b,
-                        &sh.bar_q);
-      } else if (pt != 0 && !p.test_wait_limit) {
-        mbar_arrive(&sh.bar_q);
-      }
+      // thread 0 issued the Q boxes during set-up; the others arrive
+      if (pt != 0 && !p.test_wait_limit) mbar_arrive(&sh.bar_q);
     }
     for (int h = 0; h < (has1 ? 2 : 1) && !tma_q; ++h) {
       const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(p.Q.ptr) + b * p.Q.sB + (h0 + h) * p.Q.sH;
@@ -359,8 +394,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p, con
     // A tile of BLK contiguous rows (from row0) by TMA: one thread announces
     // the bytes and issues the 64-column boxes; the other producer threads
     // arrive.
-    auto tma_tile = [&](uint64_t* bar, uint32_t dst, const CUtensorMap* map, int row0) {
+    auto tma_tile = [&](uint64_t* bar, uint32_t dst, const CUtensorMap* map, int row0, bool issued) {
       if (pt == 0) {
+        if (issued) return;                  // tile 0's boxes went out during set-up
         mbar_expect_tx(bar, static_cast<uint32_t>(C::kKVBytes));
         for (int c = 0; c < D / 64; ++c) tma_rows_4d(dst + c * (BLK * 128), map, c * 64, row0, hk, b, bar);
       } else {
@@ -445,7 +481,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p, con
           }
         }
         if (p.tma && row0 >= 0) {
-          tma_tile(&sh.bar_k[st], sK + st * C::kKVBytes, &mk, row0);
+          tma_tile(&sh.bar_k[st], sK + st * C::kKVBytes, &mk, row0, early_kv && t == 0);
         } else {
           if (!ES || live(t)) gather_tile(sK + st * C::kKVBytes, kb, p.K.sN, rowbuf[st]);
           cp_async_mbar_arrive(&sh.bar_k[st]);    // arrives when this thread's copies land
@@ -456,7 +492,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p, con
         const bool okv = t < kStages || wait_slot(&sh.bar_vempty[sv], ((t >> 1) - 1) & 1, t);
         if (named_sync_or(1, kProducerThreads, !okv)) break;
         if (p.tma && row0 >= 0) {
-          tma_tile(&sh.bar_v[sv], sV + sv * C::kKVBytes, &mv, row0);
+          tma_tile(&sh.bar_v[sv], sV + sv * C::kKVBytes, &mv, row0, early_kv && t == 0);
         } else {
           if (!ES || live(t)) gather_tile(sV + sv * C::kKVBytes, vb, p.V.sN, rowbuf[sv]);
           cp_async_mbar_arrive(&sh.bar_v[sv]);
