@@ -97,7 +97,7 @@ struct Shared {
 // heads' lists are interleaved (one tile of each in turn, every tile for one
 // head); tiles of a head that has stopped are not loaded and only passed
 // through the rings.
-template <int D, int BLK, bool ES, bool QP>
+template <int D, int BLK, bool ES, bool QP, bool GT>
 __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p, const __grid_constant__ CUtensorMap mq,
                                                                 const __grid_constant__ CUtensorMap mk,
                                                                 const __grid_constant__ CUtensorMap mv) {
@@ -696,7 +696,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p, con
     const int64_t qp = QP ? static_cast<int64_t>(qpos[h][r < BLK ? r : 0]) : q0 + r;
     const bool active = h == 0 || has1;
     const float thr =
-        (active && p.gate_thr) ? p.gate_thr[(static_cast<int64_t>(b) * Hq + hq) * p.nb + i] : -INFINITY;
+        (GT && active) ? p.gate_thr[(static_cast<int64_t>(b) * Hq + hq) * p.nb + i] : -INFINITY;
     float m_run = -INFINITY, l_run = 0.f;
     bool o_init = false;
     int k = 0, n_qk = 0, n_gated = 0;
@@ -716,7 +716,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p, con
       // -inf (no more causal tiles than the calibration keeps) can never drop
       // a tile, so its warpgroup skips the gate altogether: thr is the same
       // for every thread of the warpgroup, so this costs no divergence.
-      if (p.gate_thr && t != 0 && thr > -INFINITY) {
+      if (GT && t != 0 && thr > -INFINITY) {
         float rm = -INFINITY;
 #pragma unroll 1
         for (int c = 0; c < BLK / 64; ++c) {
@@ -929,7 +929,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p, con
   }
 }
 
-template <int D, int BLK, bool ES, bool QP>
+template <int D, int BLK, bool ES, bool QP, bool GT>
 cudaError_t launch_typed(const AttnParams& p0, cudaStream_t s) {
   // Tensor maps for the TMA loads of Q and of natural K/V tiles (128-row
   // boxes, so BLK = 128 only); without them every tile is gathered.
@@ -945,20 +945,23 @@ cudaError_t launch_typed(const AttnParams& p0, cudaStream_t s) {
   int smem = 1024 + C::kEnd + 4 * max_union;
   smem = smem < C::kMinSmem ? C::kMinSmem : smem;
   if (smem + 4096 > 227 * 1024) return cudaErrorInvalidValue;   // + static shared memory
-  cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D, BLK, ES, QP>,
+  cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D, BLK, ES, QP, GT>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const int npair = (p.G + 1) / 2;
   const int64_t items = static_cast<int64_t>(p.nb) * p.Q.B * p.K.H * npair;
   if (items >= (1ll << 31)) return cudaErrorInvalidValue;
-  attn_fwd_kernel<D, BLK, ES, QP><<<static_cast<unsigned>(items), kThreads, smem, s>>>(p, mq, mk, mv);
+  attn_fwd_kernel<D, BLK, ES, QP, GT><<<static_cast<unsigned>(items), kThreads, smem, s>>>(p, mq, mk, mv);
   return cudaGetLastError();
 }
 
 template <int D, int BLK>
 cudaError_t launch_mode(const AttnParams& p, cudaStream_t s) {
-  if (p.qperm) return p.early_stop ? cudaErrorInvalidValue : launch_typed<D, BLK, false, true>(p, s);
-  return p.early_stop ? launch_typed<D, BLK, true, false>(p, s) : launch_typed<D, BLK, false, false>(p, s);
+  // (the gate's code is compiled only into the kernel that gates)
+  if (p.qperm)
+    return p.early_stop || p.gate_thr ? cudaErrorInvalidValue : launch_typed<D, BLK, false, true, false>(p, s);
+  if (p.early_stop) return p.gate_thr ? cudaErrorInvalidValue : launch_typed<D, BLK, true, false, false>(p, s);
+  return p.gate_thr ? launch_typed<D, BLK, false, false, true>(p, s) : launch_typed<D, BLK, false, false, false>(p, s);
 }
 
 }  // namespace
