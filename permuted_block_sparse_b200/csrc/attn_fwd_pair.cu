@@ -499,24 +499,22 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_pair_kernel(AttnParams p
           uint32_t x[64], u[32];
           tmem_ld64(tS + c * 64, x);
           float cmax = -INFINITY;
+          // Causal tiles: columns above the row's last visible key become -inf
+          // (exponential 0), then the same pass as every other tile.
           if (causal) {
 #pragma unroll
-            for (int e = 0; e < 64; ++e) {
-              const float v = c * 64 + e > r ? -INFINITY : __uint_as_float(x[e]);
-              x[e] = __float_as_uint(v);
-              cmax = fmaxf(cmax, v);
-            }
-          } else {
-            float mm[8];
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-              mm[q] = fmax3(__uint_as_float(x[q]), __uint_as_float(x[8 + q]), __uint_as_float(x[16 + q]));
-              mm[q] = fmax3(mm[q], __uint_as_float(x[24 + q]), __uint_as_float(x[32 + q]));
-              mm[q] = fmax3(mm[q], __uint_as_float(x[40 + q]), __uint_as_float(x[48 + q]));
-              mm[q] = fmaxf(mm[q], __uint_as_float(x[56 + q]));
-            }
-            cmax = fmax3(fmax3(mm[0], mm[1], mm[2]), fmax3(mm[3], mm[4], mm[5]), fmaxf(mm[6], mm[7]));
+            for (int e = 0; e < 64; ++e)
+              if (c * 64 + e > r) x[e] = __float_as_uint(-INFINITY);
           }
+          float mm[8];
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            mm[q] = fmax3(__uint_as_float(x[q]), __uint_as_float(x[8 + q]), __uint_as_float(x[16 + q]));
+            mm[q] = fmax3(mm[q], __uint_as_float(x[24 + q]), __uint_as_float(x[32 + q]));
+            mm[q] = fmax3(mm[q], __uint_as_float(x[40 + q]), __uint_as_float(x[48 + q]));
+            mm[q] = fmaxf(mm[q], __uint_as_float(x[56 + q]));
+          }
+          cmax = fmax3(fmax3(mm[0], mm[1], mm[2]), fmax3(mm[3], mm[4], mm[5]), fmaxf(mm[6], mm[7]));
           const float cm = cmax * p.scale_log2;
           const bool up = cm > (m_t == -INFINITY ? -INFINITY : m_t + kRescaleSlack);
           if (__any_sync(0xffffffffu, up)) {
@@ -539,35 +537,25 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_pair_kernel(AttnParams p
             m_t = m_new;
           }
           const float m_use = m_t == -INFINITY ? 0.f : m_t;
-          if (causal) {
+          unsigned long long ps2[4] = {0ull, 0ull, 0ull, 0ull};
+          const unsigned long long sc2 = f2_pack(p.scale_log2, p.scale_log2);
+          const unsigned long long nm2 = f2_pack(-m_use, -m_use);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              const float a0 = ex2(fmaf(__uint_as_float(x[2 * e]), p.scale_log2, -m_use));
-              const float a1 = ex2(fmaf(__uint_as_float(x[2 * e + 1]), p.scale_log2, -m_use));
-              psum += a0 + a1;
-              u[e] = pack_bf16x2(a0, a1);
-            }
-          } else {
-            unsigned long long ps2[4] = {0ull, 0ull, 0ull, 0ull};
-            const unsigned long long sc2 = f2_pack(p.scale_log2, p.scale_log2);
-            const unsigned long long nm2 = f2_pack(-m_use, -m_use);
-#pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              const unsigned long long y =
-                  f2_fma(f2_pack(__uint_as_float(x[2 * e]), __uint_as_float(x[2 * e + 1])), sc2, nm2);
-              float y0, y1;
-              f2_unpack(y, y0, y1);
-              const float a0 = ex2(y0), a1 = ex2(y1);
-              ps2[e & 3] = f2_add(ps2[e & 3], f2_pack(a0, a1));
-              u[e] = cvt_bf16x2(a0, a1);
-            }
-            float s0, s1, s2, s3, s4, s5, s6, s7;
-            f2_unpack(ps2[0], s0, s1);
-            f2_unpack(ps2[1], s2, s3);
-            f2_unpack(ps2[2], s4, s5);
-            f2_unpack(ps2[3], s6, s7);
-            psum += ((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7));
+          for (int e = 0; e < 32; ++e) {
+            const unsigned long long y =
+                f2_fma(f2_pack(__uint_as_float(x[2 * e]), __uint_as_float(x[2 * e + 1])), sc2, nm2);
+            float y0, y1;
+            f2_unpack(y, y0, y1);
+            const float a0 = ex2(y0), a1 = ex2(y1);
+            ps2[e & 3] = f2_add(ps2[e & 3], f2_pack(a0, a1));
+            u[e] = cvt_bf16x2(a0, a1);
           }
+          float s0, s1, s2, s3, s4, s5, s6, s7;
+          f2_unpack(ps2[0], s0, s1);
+          f2_unpack(ps2[1], s2, s3);
+          f2_unpack(ps2[2], s4, s5);
+          f2_unpack(ps2[3], s6, s7);
+          psum += ((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7));
           tmem_st32(tS + c * 32, u);
         }
         const float m_new = m_t;
