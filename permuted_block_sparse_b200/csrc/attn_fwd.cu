@@ -67,6 +67,36 @@ struct Cfg {
   static constexpr int kMinSmem = 120 * 1024;
 };
 
+// Rare softmax paths, kept out of line so that the softmax loop's
+// instruction footprint stays small (called by whole warps).
+// Rescale the first n16 x 16 P columns of this tile (bf16 pairs) by beta,
+// after this thread's earlier P stores have landed.
+__device__ __noinline__ void rescale_p(uint32_t tS, int n16, float beta) {
+  tmem_st_wait();
+  for (int q = 0; q < n16; ++q) {
+    uint32_t w[16];
+    tmem_ld16(tS + q * 16, w);
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[e]));
+      w[e] = pack_bf16x2(f.x * beta, f.y * beta);
+    }
+    tmem_st16(tS + q * 16, w);
+  }
+}
+// Rescale this row's O accumulator (D fp32 columns) by alpha.
+template <int D>
+__device__ __noinline__ void rescale_o(uint32_t tO, float alpha) {
+#pragma unroll 1
+  for (int c = 0; c < D / 32; ++c) {
+    uint32_t u[32];
+    tmem_ld32(tO + c * 32, u);
+#pragma unroll
+    for (int e = 0; e < 32; ++e) u[e] = __float_as_uint(__uint_as_float(u[e]) * alpha);
+    tmem_st32(tO + c * 32, u);
+  }
+}
+
 __device__ __forceinline__ float warp_max(float v) {
   for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
   return v;
@@ -791,19 +821,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p, con
           const float m_new = up ? cm : m_t;
           // 0 when m_t was -inf; 1 for a row that still has no visible key
           const float beta = m_new == -INFINITY ? 1.0f : ex2(m_t - m_new);
-          if (c > 0 && __any_sync(0xffffffffu, beta != 1.0f)) {
-            tmem_st_wait();                           // earlier P stores of this thread landed
-            for (int q = 0; q < 2 * c; ++q) {         // rescale this tile's P so far
-              uint32_t w[16];
-              tmem_ld16(tS + q * 16, w);             // columns q*16 .. q*16+15 hold P
-#pragma unroll
-              for (int e = 0; e < 16; ++e) {
-                const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[e]));
-                w[e] = pack_bf16x2(f.x * beta, f.y * beta);
-              }
-              tmem_st16(tS + q * 16, w);
-            }
-          }
+          if (c > 0 && __any_sync(0xffffffffu, beta != 1.0f)) rescale_p(tS, 2 * c, beta);
           psum *= beta;
           m_t = m_new;
         }
@@ -834,18 +852,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p, con
       const float m_new = m_t;
       // (a row that has seen no visible key yet keeps m = -inf and l = 0)
       const float alpha = m_new == -INFINITY ? 1.0f : ex2(m_run - m_new);
-      if (o_init && __any_sync(0xffffffffu, alpha != 1.0f)) {
-        // PV of this head's previous tile has completed: the S-ready barrier
-        // tracks every MMA issued before this tile's QK^T.
-#pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t u[32];
-          tmem_ld32(tO + c * 32, u);
-#pragma unroll
-          for (int e = 0; e < 32; ++e) u[e] = __float_as_uint(__uint_as_float(u[e]) * alpha);
-          tmem_st32(tO + c * 32, u);
-        }
-      }
+      // (PV of this head's previous tile has completed: the S-ready barrier
+      // tracks every MMA issued before this tile's QK^T)
+      if (o_init && __any_sync(0xffffffffu, alpha != 1.0f)) rescale_o<D>(tO, alpha);
       l_run = l_run * alpha + psum;
       m_run = m_new;
       // Early stopping (Pass 2 only): this tile's gain per row is psum / l,
