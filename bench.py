@@ -372,13 +372,15 @@ def run_pbs(args):
 
     def step(record=False, st=None):
         e = [torch.cuda.Event(enable_timing=True) for _ in range(4)] if record else None
+        if record and gate:
+            e[1] = e[2] = e[0]      # no permutation or selection phase: no events between
         if record:
             e[0].record(s)
         if not gate and not sample:
             permute(Q, K, w.blk, w.seg, w.n_sink, perm=perm, ws=ws_p)
         if qperm_on:
             pbs.pbs_permute_queries(Q, K, w.blk, w.seg, qperm=qperm, ws=ws_q)
-        if record:
+        if record and not gate:
             e[1].record(s)
         if qperm_on:
             pbs.pbs_select_qperm(Q, K, perm, qperm, w.blk, w.seg, w.mode, dt, w.n_sink, cap=cap, counts=counts,
@@ -386,7 +388,7 @@ def run_pbs(args):
         elif not gate:
             pbs.pbs_select(Q, K, None if sample else perm, w.blk, w.seg, w.mode, dt, w.band, w.n_sink, cap=cap,
                            counts=counts, idx=idx, ws=ws_s, score_order=early)
-        if record:
+        if record and not gate:
             e[2].record(s)
         if early:
             pbs.pbs_attn_fwd_early_stop(Q, K, V, perm, counts, idx, w.blk, w.seg, w.stop_tau, out=O, lse=lse,
