@@ -106,6 +106,7 @@ struct Shared {
   uint64_t bar_q;
   uint64_t bar_k[kStages], bar_v[kStages], bar_kempty[kStages], bar_vempty[kStages];
   uint64_t bar_s[2], bar_p[2], bar_o[2], bar_fin;
+  uint64_t bar_sched;      // the schedule is built (the LAZY kernels)
   uint32_t tmem_base;
   int abort;
   int n_union;
@@ -187,9 +188,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p, con
       mbar_init(&sh.bar_o[h], 1);
     }
     mbar_init(&sh.bar_fin, 1);
+    mbar_init(&sh.bar_sched, 32);               // every lane of the building warp
     fence_mbar_init();
   }
+  if (warp == 0) {
+    tmem_alloc(&sh.tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
   __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sh.tmem_base;
   // (the failure-path test hook withholds the Q loads; with early stopping
   // warp 0 compacts the lists in the V ring during set-up, so tile 0 waits)
   const bool early = p.tma && !QP && !p.test_wait_limit;
@@ -208,9 +217,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p, con
     for (int c = 0; c < D / 64; ++c)
       tma_rows_4d(sV + c * (BLK * 128), &mv, c * 64, i * BLK, hk, b, &sh.bar_v[0]);
   }
-  if (warp == 0) {
-    tmem_alloc(&sh.tmem_base, 512);
-    tmem_relinquish();
+  // LAZY (natural query order, no early stopping, no gate): a producer warp builds
+  // the schedule while the diagonal tile -- block i itself, natural, both
+  // heads, needing no schedule -- already runs: its QK^T, softmax and PV go
+  // ahead, and each role waits for the schedule only when it needs the tiles
+  // after it.  Otherwise warp 0 builds it before anything starts.
+  constexpr bool LAZY = !QP && !ES && !GT;     // (with the gate it measured slower)
+  auto build_schedule = [&]() {
     // union of the two heads' lists as a bitmap, then an ascending schedule
     int cnt[2] = {0, 0};
     for (int h = 0; h < 2; ++h) {
@@ -343,16 +356,23 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p, con
       for (int off = 16; off > 0; off >>= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, off));
       if (lane == 0) sh.jtop = static_cast<int>(mx / BLK);
     }
+    if (LAZY) {
+      __syncwarp();
+      mbar_arrive(&sh.bar_sched);               // each lane: its schedule writes are released
+    }
+  };
+  if (!LAZY && warp == 0) build_schedule();
+  if (!LAZY) {
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
   }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = sh.tmem_base;
   // Pass 1 runs natural blocks jtop, jtop - 1, ..., down to the segment's
   // first; jtop is i itself unless queries are permuted.
   const int jtop = QP ? sh.jtop : i;
   const int n_diag = jtop - s * spb + 1;
-  const int T = n_diag + sh.n_union;
+  // tiles of the item (LAZY: known to each role once it has waited for the schedule)
+  int T = LAZY ? 0 : n_diag + sh.n_union;
   // Poll limit of the role waits (the drain before tensor memory is freed
   // keeps the full limit).
   const uint32_t lim = p.test_wait_limit ? p.test_wait_limit : kSpinLimit;
@@ -421,6 +441,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p, con
     // (the failure-path test hook withholds this arrival, so the MMA role's
     // wait for Q runs out)
     if (!p.test_wait_limit && !tma_q) cp_async_mbar_arrive(&sh.bar_q);
+    if constexpr (LAZY) {
+      if (warp == 2) build_schedule();
+      named_sync(1, kProducerThreads);          // the schedule is built
+      T = n_diag + sh.n_union;
+    }
     // A tile of BLK contiguous rows (from row0) by TMA: one thread announces
     // the bytes and issues the 64-column boxes; the other producer threads
     // arrive.
@@ -557,6 +582,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p, con
       // All loop state lives in registers: per-head arrays are indexed only
       // by the unrolled head loop's constant, per-stage values are separate
       // scalars chosen by the stage bit.
+      // LAZY: a first pass of the event loop runs tile 0 alone (T = 1 here),
+      // then the schedule is awaited and the loop goes on over every tile.
+      bool phase_a = LAZY;
+      if (phase_a) T = 1;
       // Per head: next tile needing QK^T, tile whose PV is pending, QK count.
       int nq[2] = {T, T}, pend[2] = {-1, -1}, kh[2] = {0, 0};
       bool o_init[2] = {false, false};
@@ -606,6 +635,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p, con
       // (previous PV_h issued, K landed) can go, goes.  QK_h(t) is always
       // issued after PV_h of the head's previous tile, so P (which lives in
       // S's columns) has been consumed before S is overwritten.
+      for (;;) {
       while (ok) {
         bool pending = false, progress = false;
         const bool all_stopped = ES && hstop[0] && (nh < 2 || hstop[1]);
@@ -704,6 +734,21 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p, con
           ok = !__shfl_sync(0xffffffffu, *abort_flag, 0);
         }
       }
+      if (phase_a && ok) {
+        // tile 0 is done (its PV issued): wait for the schedule, go on from tile 1
+        phase_a = false;
+        // (every lane waits, so each has acquired the schedule)
+        ok = __all_sync(0xffffffffu, mbar_wait_or_abort(&sh.bar_sched, 0, p.err, abort_flag, lim));
+        if (ok) {
+          T = n_diag + sh.n_union;
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+            if (h < nh) nq[h] = next_tile(h, 1);
+          continue;
+        }
+      }
+      break;
+      }
       if (leader) {
 #pragma unroll
         for (int h = 0; h < 2; ++h)
@@ -734,7 +779,22 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p, con
     // to its end with every wait returning at once, so the warpgroup takes
     // the same named barriers without a vote each tile.
     bool ok = true;
-    for (int t = 0; active && t < T; ++t) {
+    // LAZY: tile 0 first (T = 1 here), then the schedule is awaited
+    bool sched_seen = !LAZY;
+    if (!sched_seen) T = 1;
+    for (int t = 0; active; ++t) {
+      if (t >= T) {
+        if (sched_seen) break;
+        sched_seen = true;
+        // one vote, so the warpgroup stays together on its named barriers
+        const bool w = mbar_wait_or_abort(&sh.bar_sched, 0, p.err, abort_flag, lim);
+        if (named_sync_or(2 + h, 128, !w)) {
+          ok = false;
+          break;                                    // (after an abort the schedule may be unwritten)
+        }
+        T = n_diag + sh.n_union;
+        if (t >= T) break;
+      }
       if (!((tile_mask(t) >> h) & 1u)) continue;
       if (!mbar_wait_or_abort(&sh.bar_s[h], k & 1, p.err, abort_flag, lim)) ok = false;
       tc_fence_after();
