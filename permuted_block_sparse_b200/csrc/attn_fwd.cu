@@ -25,8 +25,10 @@
 // ordered lists are interleaved instead, each tile serving one head.)
 // Roles (384 threads):
 //   warp 0       tcgen05 MMA issuer (one thread) and tensor-memory owner;
-//   warps 1-3    producer: 16-byte cp.async row gathers of Q once and of the
-//                K and V tiles into a 2-stage ring of 128B-swizzled tiles;
+//   warps 1-3    producer: Q once and the K and V tiles into 2-stage rings
+//                of 128B-swizzled tiles -- by TMA where a tile's rows are
+//                contiguous (Q, natural blocks, in-order permuted blocks),
+//                else by 16-byte cp.async row gathers;
 //   warps 4-7    softmax for head slot 0, warps 8-11 for head slot 1: each
 //                thread owns one query row of S and O in tensor memory.
 // Tensor memory (512 columns): S0 | S1 | O0 | O1, 128 columns each; P (bf16)
@@ -36,8 +38,9 @@
 // PVs, so each gather has about two tiles of time to land.  The MMA thread
 // is event driven: it issues whichever QK^T or PV is ready, so that while
 // one softmax warpgroup works on its tile the tensor core works for the
-// other head.  All waits are bounded; a shared abort flag makes
-// every role of the CTA give up together.
+// other head.  Causal tiles only mask columns to -inf and then take the
+// same softmax pass as every other tile.  All waits are bounded; a shared
+// abort flag makes every role of the CTA give up together.
 #include <math.h>
 
 #include <algorithm>
