@@ -131,7 +131,7 @@ struct Shared {
 // heads' lists are interleaved (one tile of each in turn, every tile for one
 // head); tiles of a head that has stopped are not loaded and only passed
 // through the rings.
-template <int D, int BLK, bool ES, bool QP, bool GT>
+template <int D, int BLK, bool ES, bool QP, bool GT, bool LZ>
 __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p, const __grid_constant__ CUtensorMap mq,
                                                                 const __grid_constant__ CUtensorMap mk,
                                                                 const __grid_constant__ CUtensorMap mv) {
@@ -225,7 +225,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p, con
   // heads, needing no schedule -- already runs: its QK^T, softmax and PV go
   // ahead, and each role waits for the schedule only when it needs the tiles
   // after it.  Otherwise warp 0 builds it before anything starts.
-  constexpr bool LAZY = !QP && !ES && !GT;     // (with the gate it measured slower)
+  // (chosen by the launcher where the own segment holds more than the
+  // diagonal block; with one block per segment, as in the gate workloads and
+  // the dense run, and with the gate it measured slower)
+  constexpr bool LAZY = LZ && !QP && !ES && !GT;
   auto build_schedule = [&]() {
     // union of the two heads' lists as a bitmap, then an ascending schedule
     int cnt[2] = {0, 0};
@@ -989,7 +992,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p, con
   }
 }
 
-template <int D, int BLK, bool ES, bool QP, bool GT>
+template <int D, int BLK, bool ES, bool QP, bool GT, bool LZ = false>
 cudaError_t launch_typed(const AttnParams& p0, cudaStream_t s) {
   // Tensor maps for the TMA loads of Q and of natural K/V tiles (128-row
   // boxes, so BLK = 128 only); without them every tile is gathered.
@@ -1005,13 +1008,13 @@ cudaError_t launch_typed(const AttnParams& p0, cudaStream_t s) {
   int smem = 1024 + C::kEnd + 4 * max_union;
   smem = smem < C::kMinSmem ? C::kMinSmem : smem;
   if (smem + 4096 > 227 * 1024) return cudaErrorInvalidValue;   // + static shared memory
-  cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D, BLK, ES, QP, GT>,
+  cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D, BLK, ES, QP, GT, LZ>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const int npair = (p.G + 1) / 2;
   const int64_t items = static_cast<int64_t>(p.nb) * p.Q.B * p.K.H * npair;
   if (items >= (1ll << 31)) return cudaErrorInvalidValue;
-  attn_fwd_kernel<D, BLK, ES, QP, GT><<<static_cast<unsigned>(items), kThreads, smem, s>>>(p, mq, mk, mv);
+  attn_fwd_kernel<D, BLK, ES, QP, GT, LZ><<<static_cast<unsigned>(items), kThreads, smem, s>>>(p, mq, mk, mv);
   return cudaGetLastError();
 }
 
@@ -1021,7 +1024,9 @@ cudaError_t launch_mode(const AttnParams& p, cudaStream_t s) {
   if (p.qperm)
     return p.early_stop || p.gate_thr ? cudaErrorInvalidValue : launch_typed<D, BLK, false, true, false>(p, s);
   if (p.early_stop) return p.gate_thr ? cudaErrorInvalidValue : launch_typed<D, BLK, true, false, false>(p, s);
-  return p.gate_thr ? launch_typed<D, BLK, false, false, true>(p, s) : launch_typed<D, BLK, false, false, false>(p, s);
+  if (p.gate_thr) return launch_typed<D, BLK, false, false, true>(p, s);
+  return p.seg > p.blk ? launch_typed<D, BLK, false, false, false, true>(p, s)
+                       : launch_typed<D, BLK, false, false, false, false>(p, s);
 }
 
 }  // namespace
