@@ -173,7 +173,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(AttnParams p, con
   // ------------------------------------------------------------------ setup
   // Barriers first, so that the loads that need no schedule -- Q and, in
   // natural query order, the diagonal block's K and V (tile 0) -- start by
-  // TMA while warp 0 builds the schedule.
+  // TMA while the schedule is being built.
   if (tid == 32) {
     sh.abort = 0;
     sh.limit[0] = 0x7fffffff;
