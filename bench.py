@@ -342,14 +342,17 @@ def run_pbs(args):
     ws_s = torch.empty(pbs.workspace_size(op_s, Q, K, w.blk, w.seg) + 256, dtype=torch.uint8, device=dev)
     permute = pbs.pbs_permute_segmented if segperm else pbs.pbs_permute
     stats = torch.zeros(2, dtype=torch.int64, device=dev)
-    launches_per_step = 6   # 2 permute + 3 select + 1 attention kernels
+    # 2 permute kernels; select: query pooling, key pooling (one launch per
+    # key permutation), block scores, top-k / cumulative-mass selection;
+    # 1 attention kernel
+    launches_per_step = 2 + 3 + (nseg if segperm else 1) + 1
     qperm_on = w.query_perm        # S2O's query permutation
     qperm = ws_q = None
     if qperm_on:
         qperm = torch.empty((w.B, w.Hq, w.N), dtype=torch.int32, device=dev)
         ws_q = torch.empty(pbs.workspace_size(pbs.PBS_OP_PERMUTE_QUERIES, Q, K, w.blk, w.seg) + 256,
                            dtype=torch.uint8, device=dev)
-        launches_per_step = 9   # 2 + 3 permute (keys, queries) + 3 select + 1 attention
+        launches_per_step = 10  # 2 + 3 permute (keys, queries) + 4 select + 1 attention
     # Block-max gating workloads: no permutation or selection step; every
     # earlier block is listed and the thresholds (calibrated offline by the
     # oracle, stored beside the tests) decide per tile.
