@@ -117,6 +117,21 @@ def select_bytes(w, cap):
     return w.B * w.Hq * w.N * w.d * 2 + w.B * w.Hkv * w.N * w.d * 2 + 2 * pooled + lists
 
 
+def step_launches(w) -> int:
+    """Kernels one step of the workload launches (all in this library)."""
+    if w.mode == "gate":
+        return 1                                 # attention alone
+    if w.mode == "sample":
+        return 4                                 # 3 selection kernels + attention
+    if w.query_perm:
+        return 10                                # 2 + 3 permutation (keys, queries) + 4 selection + attention
+    # 2 permutation kernels; selection: query pooling, key pooling (one
+    # launch per key permutation), block scores, top-k / cumulative-mass
+    # selection; attention
+    nperm = (w.N + w.seg - 1) // w.seg if w.perm_per_segment else 1
+    return 2 + 3 + nperm + 1
+
+
 def _gbs(nbytes, ms):
     return None if nbytes is None or ms <= 0 else nbytes / (ms * 1e-3) / 1e9
 
@@ -342,17 +357,13 @@ def run_pbs(args):
     ws_s = torch.empty(pbs.workspace_size(op_s, Q, K, w.blk, w.seg) + 256, dtype=torch.uint8, device=dev)
     permute = pbs.pbs_permute_segmented if segperm else pbs.pbs_permute
     stats = torch.zeros(2, dtype=torch.int64, device=dev)
-    # 2 permute kernels; select: query pooling, key pooling (one launch per
-    # key permutation), block scores, top-k / cumulative-mass selection;
-    # 1 attention kernel
-    launches_per_step = 2 + 3 + (nseg if segperm else 1) + 1
+    launches_per_step = step_launches(w)
     qperm_on = w.query_perm        # S2O's query permutation
     qperm = ws_q = None
     if qperm_on:
         qperm = torch.empty((w.B, w.Hq, w.N), dtype=torch.int32, device=dev)
         ws_q = torch.empty(pbs.workspace_size(pbs.PBS_OP_PERMUTE_QUERIES, Q, K, w.blk, w.seg) + 256,
                            dtype=torch.uint8, device=dev)
-        launches_per_step = 10  # 2 + 3 permute (keys, queries) + 4 select + 1 attention
     # Block-max gating workloads: no permutation or selection step; every
     # earlier block is listed and the thresholds (calibrated offline by the
     # oracle, stored beside the tests) decide per tile.
@@ -366,10 +377,8 @@ def run_pbs(args):
         counts.copy_(torch.arange(w.nb, dtype=torch.int32, device=dev).expand(w.B, w.Hq, w.nb))
         cap = max(w.nb - 1, 1)
         idx = torch.arange(cap, dtype=torch.int32, device=dev).expand(w.B, w.Hq, w.nb, cap).contiguous()
-        launches_per_step = 1
     if sample:
         perm.copy_(torch.arange(w.N, dtype=torch.int32, device=dev).expand(w.B, w.Hkv, w.N))
-        launches_per_step = 4   # 3 select + 1 attention kernels
 
     ev = {k: [] for k in ("p0", "p1", "s1", "a1")}
 

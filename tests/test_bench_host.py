@@ -66,3 +66,19 @@ def test_dense_flops_and_labels():
     assert bench.dense_causal_flops(w) == 2.0 * 128 * 131072 ** 2 * 32
     assert "topk density=0.1" in bench.selection_label(w) and "n_sink=128" in bench.selection_label(w)
     assert bench.selection_label(synth.WORKLOADS["sample_32k_local"]).startswith("SampleAttention-style")
+
+
+def test_step_launches():
+    """The kernels one bench step launches, as the library's entry points
+    issue them: 2 permutation, 4 selection (one key-pooling launch per key
+    permutation), 1 attention."""
+    W = synth.WORKLOADS
+    assert bench.step_launches(W["llama8b_128k_sink"]) == 7
+    assert bench.step_launches(W["llama8b_32k_tau"]) == 7
+    assert bench.step_launches(W["s2o_32k_stop"]) == 7
+    w = W["s2o_32k_segperm"]
+    assert bench.step_launches(w) == 6 + w.N // w.seg
+    assert bench.step_launches(W["s2o_32k_qperm"]) == 10
+    assert bench.step_launches(W["sample_32k_local"]) == 4
+    for name in ("gate_b8_2k", "gate_b8_4k", "gate_b1_64k"):
+        assert bench.step_launches(W[name]) == 1
